@@ -1,0 +1,510 @@
+"""Benchmark of the DSA hot path: one step = one pass of the whole path over one batch.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode_b8] [--impl ours|reference]
+
+A decode step runs, through the C ABI: dsa_index_keys on the new keys (written into the
+resident FP8 K-cache) and on the queries, dsa_index_scores, dsa_topk and dsa_sparse_mla. A
+prefill step runs the same calls over all T queries and S keys. Inputs are seeded synthetic
+tensors of the workload's shapes (dsa_inputs); the caches are resident device state.
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on the launching
+stream with a 256 MiB L2-flush write between steps (outside the events); the K step times are
+summed, ranks barrier + synchronise before and after, and rank 0 reports the max over ranks.
+Under torchrun each rank runs its own replica of the workload (independent sequences, no
+collective on the data path): weak scaling.
+
+The reference arm (--impl reference) times the CPU oracle on the host cores on a bounded sample
+of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import dsa_inputs as DI  # noqa: E402
+
+METRIC = "indexer scores/s (query·key pairs) + sparse-MLA decode tok/s; % FP8 or HBM roofline"
+UNIT = "query·key pairs/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------------------ work accounting
+def work_units(inp):
+    """Algorithmic units of one step: causal (query, key) pairs scored, queries decoded, and the
+    per-kernel algorithmic bytes / flops (the roofline numerators)."""
+    from math import prod
+    nv = np.clip(np.minimum(inp.q_pos.astype(np.int64) + 1, inp.kv_len[:, None]), 0, None)
+    pairs = int(nv.sum())
+    k = inp.workload.topk
+    sel = int(np.minimum(nv, k).sum())
+    BT = int(prod(inp.q_pos.shape))
+    new_keys = BT if inp.workload.decode else inp.idx_k.shape[0] * inp.idx_k.shape[1]
+    return {
+        "pairs": pairs,
+        "queries": BT,
+        "selected": sel,
+        # per kernel: bytes read + written that the operation cannot avoid
+        "index_keys_bytes": (BT * 64 + new_keys) * (512 + 132) + (BT + new_keys) * 4,
+        "index_scores_bytes": pairs * (132 + 4) + BT * 64 * (128 + 4 + 4),
+        "index_scores_flops": pairs * 64 * 128 * 2,
+        "topk_bytes": pairs * 4 + BT * k * 4,
+        "sparse_mla_bytes": sel * 1152 + BT * 128 * (576 + 512) * 2 + BT * k * 4,
+        "sparse_mla_flops": sel * 128 * (576 + 512) * 2,
+    }
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------------------ clocks sampling
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------ our arm
+class Step:
+    """Device-resident state and the ABI calls of one step."""
+
+    def __init__(self, inp, device):
+        import torch
+        import sparse_attention_keys_b200 as dsa
+        self.dsa, self.torch, self.inp = dsa, torch, inp
+        wl = inp.workload
+        B, T = inp.q_pos.shape
+        S = wl.s_max
+        self.B, self.T, self.S, self.k = B, T, S, wl.topk
+        dev = device
+        self.table = dsa.dsa_rope_table(16384).to(dev)
+        # resident caches
+        self.kcache = torch.zeros((B, S, 128), dtype=torch.uint8, device=dev)
+        self.kscale = torch.zeros((B, S), dtype=torch.float32, device=dev)
+        self.kv = torch.from_numpy(inp.mla_kv).view(torch.bfloat16).to(dev) if inp.mla_kv is not None else None
+        # step inputs (device copies) and their pinned host sources
+        if wl.decode:
+            # the new token of each sequence is the key at its query position
+            new_k = np.stack([inp.idx_k[b, inp.q_pos[b, 0]] for b in range(B)])
+            new_pos = inp.q_pos[:, 0].astype(np.int32)
+            new_dst = (np.arange(B) * S + new_pos).astype(np.int64)
+            # pre-fill the cache for every earlier position (state from previous steps)
+            kx = torch.from_numpy(inp.idx_k.reshape(B * S, 128)).to(dev)
+            kp = torch.from_numpy(np.tile(np.arange(S, dtype=np.int32), B)).to(dev)
+            dsa.dsa_index_keys(kx, kp, self.table, out_fp8=self.kcache, out_scale=self.kscale,
+                               dst_row=torch.arange(B * S, dtype=torch.int64, device=dev))
+            del kx, kp
+        else:
+            new_k = inp.idx_k.reshape(B * S, 128)
+            new_pos = np.tile(np.arange(S, dtype=np.int32), B)
+            new_dst = np.arange(B * S, dtype=np.int64)
+        host = {
+            "qx": inp.idx_q.reshape(B * T, 64, 128), "qpos_flat": inp.q_pos.reshape(-1).astype(np.int32),
+            "w": inp.idx_w, "q_pos": inp.q_pos, "kv_len": inp.kv_len,
+            "kx": new_k.astype(np.float32), "kpos": new_pos, "kdst": new_dst,
+        }
+        if inp.mla_q is not None:
+            host["mq"] = inp.mla_q
+        self.h = {n: torch.from_numpy(np.ascontiguousarray(a)).pin_memory() for n, a in host.items()}
+        self.d = {n: t.to(dev) for n, t in self.h.items()}
+        if "mq" in self.d:
+            self.d["mq"] = self.d["mq"].view(torch.bfloat16)
+        # outputs
+        self.q8 = torch.empty((B * T, 64, 128), dtype=torch.uint8, device=dev)
+        self.qs = torch.empty((B * T, 64), dtype=torch.float32, device=dev)
+        self.ld = (S + 3) // 4 * 4
+        self.scores = torch.empty((B, T, self.ld), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((B, T, self.k), dtype=torch.int32, device=dev)
+        self.out = torch.empty((B, T, 128, 512), dtype=torch.bfloat16, device=dev) if self.kv is not None else None
+        self.lse = torch.empty((B, T, 128), dtype=torch.float32, device=dev) if self.kv is not None else None
+        ws = dsa.dsa_sparse_mla_workspace_size(B, T, self.k) if self.kv is not None else 0
+        self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
+        self.flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.h_idx = torch.empty((B, T, self.k), dtype=torch.int32).pin_memory()
+        self.h_out = torch.empty((B, T, 128, 512), dtype=torch.bfloat16).pin_memory() if self.out is not None else None
+        self.h_lse = torch.empty((B, T, 128), dtype=torch.float32).pin_memory() if self.out is not None else None
+        self.launches_per_step = 4 + (1 if self.kv is not None else 0) + (
+            1 if ws > 0 else 0)
+
+    def h2d(self):
+        for n, t in self.h.items():
+            dst = self.d[n]
+            if dst.dtype != t.dtype:
+                dst = dst.view(t.dtype)
+            dst.copy_(t, non_blocking=True)
+
+    def d2h(self):
+        self.h_idx.copy_(self.idx, non_blocking=True)
+        if self.out is not None:
+            self.h_out.copy_(self.out, non_blocking=True)
+            self.h_lse.copy_(self.lse, non_blocking=True)
+
+    def bytes_h2d(self):
+        return sum(t.numel() * t.element_size() for t in self.h.values())
+
+    def bytes_d2h(self):
+        n = self.h_idx.numel() * 4
+        if self.out is not None:
+            n += self.h_out.numel() * 2 + self.h_lse.numel() * 4
+        return n
+
+    def run(self, ev=None):
+        """One step. ev: optional dict name -> list of (start, end) event pairs to record."""
+        dsa, d = self.dsa, self.d
+
+        def rec(name, fn):
+            if ev is None:
+                fn()
+                return
+            s = self.torch.cuda.Event(enable_timing=True)
+            e = self.torch.cuda.Event(enable_timing=True)
+            s.record()
+            fn()
+            e.record()
+            ev.setdefault(name, []).append((s, e))
+
+        B, T = self.B, self.T
+        rec("index_keys", lambda: (
+            dsa.dsa_index_keys(d["kx"], d["kpos"], self.table, out_fp8=self.kcache, out_scale=self.kscale,
+                               dst_row=d["kdst"]),
+            dsa.dsa_index_keys(d["qx"], d["qpos_flat"], self.table, out_fp8=self.q8, out_scale=self.qs)))
+        rec("index_scores", lambda: dsa.dsa_index_scores(
+            self.q8.view(B, T, 64, 128), self.qs.view(B, T, 64), d["w"], self.kcache, self.kscale, d["q_pos"],
+            d["kv_len"], scores=self.scores, ld=self.ld))
+        rec("topk", lambda: dsa.dsa_topk(self.scores, d["q_pos"], d["kv_len"], self.k, idx=self.idx))
+        if self.kv is not None:
+            rec("sparse_mla", lambda: dsa.dsa_sparse_mla(d["mq"], self.kv, self.idx, out=self.out, lse=self.lse,
+                                                         workspace=self.ws))
+
+    def l2_flush(self):
+        self.flush.zero_()
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as tdist
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    inp = DI.make_inputs(args.workload, seed=rank)
+    units = work_units(inp)
+    st = Step(inp, dev)
+    import sparse_attention_keys_b200 as dsa
+
+    for _ in range(args.warmup):
+        st.l2_flush()
+        st.run()
+    torch.cuda.synchronize()
+    status = dsa.dsa_get_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after warm-up: {dsa.dsa_status_string(status)}")
+
+    def barrier():
+        if world > 1:
+            tdist.barrier()
+        torch.cuda.synchronize()
+
+    # ---- device-timed region (inputs resident in HBM)
+    kev = {}
+    steps = []
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        for _ in range(args.steps):
+            st.l2_flush()
+            s = torch.cuda.Event(enable_timing=True)
+            e = torch.cuda.Event(enable_timing=True)
+            s.record()
+            st.run(kev)
+            e.record()
+            steps.append((s, e))
+        barrier()
+    clocks = clk.summary()
+    t_dev = sum(s.elapsed_time(e) for s, e in steps) / 1e3          # seconds
+    per_kernel = {n: sum(a.elapsed_time(b) for a, b in v) / len(v) / 1e3 for n, v in kev.items()}
+
+    # ---- end to end through host buffers (pinned H2D of the step inputs, D2H of the results)
+    for _ in range(max(1, args.warmup)):
+        st.l2_flush()
+        st.h2d(); st.run(); st.d2h()
+    barrier()
+    e2e = []
+    for _ in range(args.steps):
+        st.l2_flush()
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record()
+        st.h2d()
+        st.run()
+        st.d2h()
+        e.record()
+        e2e.append((s, e))
+    barrier()
+    t_e2e = sum(s.elapsed_time(e) for s, e in e2e) / 1e3
+    status = dsa.dsa_get_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after timing: {dsa.dsa_status_string(status)}")
+
+    # ---- max over ranks
+    if world > 1:
+        tt = torch.tensor([t_dev, t_e2e], dtype=torch.float64, device=dev)
+        tdist.all_reduce(tt, op=tdist.ReduceOp.MAX)
+        t_dev, t_e2e = tt.tolist()
+    if rank != 0:
+        return None
+
+    peaks = load_peaks()
+    total_pairs = units["pairs"] * args.steps * world
+    value = total_pairs / t_dev
+    tok_s = units["queries"] * args.steps * world / t_dev
+    # dominant kernel and its roofline
+    dom = max(per_kernel, key=per_kernel.get)
+    roof = roofline_entry(dom, per_kernel[dom], units, peaks, args)
+    wl = inp.workload
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": t_dev / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3 scores / bf16 attention, fp32 accumulate",
+        "data": "synthetic (seeded N(0,1) of the workload shapes; resident caches)",
+        "config": {"workload": wl.name, "desc": wl.note, "batch": int(inp.q_pos.shape[0]),
+                   "queries_per_seq": int(inp.q_pos.shape[1]), "s_max": wl.s_max, "topk": wl.topk,
+                   "pairs_per_step": units["pairs"], "parallelism": f"replicas x{world}",
+                   "l2": "256 MiB flush write between timed steps"},
+        "mla_decode_tok_s": tok_s if wl.decode else None,
+        "kernel_ms": {n: v * 1e3 for n, v in per_kernel.items()},
+        "roofline": roof,
+        "e2e": {"value": total_pairs / t_e2e, "unit": UNIT, "h2d_bytes_per_step": st.bytes_h2d(),
+                "d2h_bytes_per_step": st.bytes_d2h(), "ms_per_step": t_e2e / args.steps * 1e3},
+        "gpu_launches": st.launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_budget)
+    return line
+
+
+def roofline_entry(name, seconds, units, peaks, args):
+    traffic = load_traffic(name, args.workload)
+    if name in ("index_scores",) and not DI.WORKLOADS[args.workload].decode:
+        flops = units["index_scores_flops"]
+        peak = 2.0 * peaks["bf16_tflops"]            # e4m3 dense = 2 x measured bf16 (nominal ratio)
+        ach = flops / seconds / 1e12
+        return {"kernel": name, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": ach / peak, "traffic": traffic,
+                "peak_source": f"{peaks['source']} bf16 x2 (e4m3 nominal ratio)", "algorithmic_flops": flops}
+    nbytes = units[f"{name}_bytes"]
+    ach = nbytes / seconds / 1e9
+    return {"kernel": name, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": ach / peaks["hbm_gbs"], "traffic": traffic, "peak_source": f"{peaks['source']} hbm_gbs",
+            "algorithmic_bytes": nbytes}
+
+
+def load_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary for this kernel and workload, if one
+    exists and matches the current build (else null)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(f"{kernel}/{workload}")
+    if not e:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------------------ oracle timing
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_step(inp, seqs, table, caches):
+    """The oracle's pass over sequences `seqs` of one step (new keys and queries quantised,
+    scores, top-k, sparse MLA). Returns the (query, key) pairs processed."""
+    from oracle import dsa_oracle as O
+    k8_all, ks_all = caches
+    pairs = 0
+    for b in seqs:
+        sl = slice(b, b + 1)
+        q8, qs = O.index_keys(inp.idx_q[sl], inp.q_pos[sl][..., None], table)
+        if inp.workload.decode:
+            p = int(inp.q_pos[b, 0])
+            k8_all[b, p], ks_all[b, p] = O.index_keys(inp.idx_k[b, p], p, table)
+        sc = O.index_scores(q8, qs, inp.idx_w[sl], k8_all[sl], ks_all[sl], inp.q_pos[sl], inp.kv_len[sl])
+        idx = O.topk_indices(sc, inp.q_pos[sl], inp.kv_len[sl], inp.workload.topk)
+        if inp.mla_q is not None:
+            O.sparse_mla(inp.mla_q[sl], inp.mla_kv[sl], idx)
+        pairs += int(O.valid_len(inp.q_pos[sl], inp.kv_len[sl]).sum())
+    return pairs
+
+
+def _oracle_setup(workload):
+    from oracle import dsa_oracle as O
+    inp = DI.make_inputs(workload)
+    table = O.rope_table(16384)
+    if not inp.workload.decode:
+        raise SystemExit("the oracle baseline is defined for the decode workloads")
+    B, S = inp.idx_k.shape[:2]
+    k8 = np.zeros((B, S, 128), np.uint8)
+    ks = np.zeros((B, S), np.float32)
+    return inp, table, (k8, ks)
+
+
+def cpu_baseline(workload, budget_s=15.0):
+    """Time the oracle as it stands on this host, on whole sequences of the workload until about
+    `budget_s` seconds of CPU work are done; value in the metric's unit."""
+    inp, table, caches = _oracle_setup(workload)
+    B = inp.q_pos.shape[0]
+    pairs = 0
+    seqs_done = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        b = seqs_done % B
+        pairs += oracle_step(inp, [b], table, caches)
+        seqs_done += 1
+    dt = time.perf_counter() - t0
+    return {"value": pairs / dt, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{seqs_done} sequences of {workload} (full path per sequence: new key and query "
+                      f"quantised, scores, top-{inp.workload.topk}, sparse MLA) in {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    inp, table, caches = _oracle_setup(args.workload)
+    B = inp.q_pos.shape[0]
+    # one step = a bounded sample: two sequences of the workload's batch
+    sample = [0, 1] if B > 1 else [0]
+    for _ in range(args.warmup):
+        oracle_step(inp, sample, table, caches)
+    t0 = time.perf_counter()
+    pairs = 0
+    for _ in range(args.steps):
+        pairs += oracle_step(inp, sample, table, caches)
+    dt = time.perf_counter() - t0
+    value = pairs / dt
+    wl = inp.workload
+    cores = _blas_threads()
+    sample_desc = f"{len(sample)} of {B} sequences of {wl.name} per step (full path per sequence)"
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+        "data": "synthetic (seeded N(0,1) of the workload shapes)",
+        "config": {"workload": wl.name, "desc": wl.note, "batch": B, "s_max": wl.s_max, "topk": wl.topk,
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample_desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode_b8", choices=sorted(DI.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        if world > 1:
+            import datetime
+            import torch
+            import torch.distributed as tdist
+            torch.cuda.set_device(local_rank)
+            tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                     device_id=torch.device("cuda", local_rank))
+        try:
+            line = run_ours(args, rank, world, local_rank)
+        finally:
+            if world > 1:
+                import torch.distributed as tdist
+                tdist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

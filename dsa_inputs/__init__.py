@@ -69,8 +69,8 @@ def bf16_bits_from_f32(x: np.ndarray) -> np.ndarray:
     This is storage-format conversion of the synthetic draw, not method arithmetic.
     """
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    rounding_bias = ((u >> 16) & 1) + 0x7FFF
+    u = x.view(np.uint32)
+    rounding_bias = ((u >> 16) & np.uint32(1)) + np.uint32(0x7FFF)   # finite inputs: no overflow
     return ((u + rounding_bias) >> 16).astype(np.uint16)
 
 
@@ -134,6 +134,17 @@ def make_inputs(name_or_wl, seed: int = 0, with_mla: bool | None = None) -> Inpu
         hot_rows = np.sort(rng.choice(S, n_hot, replace=False))
         k[:, hot_rows, :] *= np.float32(wl.hot_key_gain)
     return Inputs(wl, q, k, w, q_pos, kv_len, mla_q, mla_kv, hot_rows)
+
+
+def filler_e4m3(shape, seed: int):
+    """Seeded e4m3 codes and fp32 block scales for rows no test checks (full-size launches where
+    only sampled rows are compared). Uses torch's fp32 -> float8_e4m3fn cast as a data source."""
+    import torch
+    g = torch.Generator().manual_seed(seed)
+    v = (torch.randn(shape, generator=g) * 100.0).clamp_(-448.0, 448.0)
+    codes = v.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    scales = (0.005 + 0.015 * torch.rand(shape[:-1], generator=g)).numpy().astype(np.float32)
+    return codes, scales
 
 
 def make_custom(batch: int, queries: int, s_max: int, topk: int, *, decode: bool, seed: int = 0,

@@ -1,0 +1,192 @@
+/*
+ * dsa.h - C ABI of libdsa, the B200 (sm_100a) hot path of DeepSeek Sparse Attention.
+ *
+ * The path: lightning-indexer transform of queries and keys (non-interleaved YaRN RoPE on the
+ * first 64 features, (1/sqrt 128) H_128, FP8-e4m3 quantisation with one fp32 scale per
+ * 128-element block, K-cache write) -> index scores I[t,s] = sum_j w[t,j] ReLU(q[t,j].k[s]) ->
+ * causal per-query top-k -> sparse MQA-style latent attention over the selected positions.
+ *
+ * Sources (web pages on DeepSeek-V3.2-Exp):
+ *   [news]    "DeepSeek fixes RoPE mismatch in the V3.2-Exp inference demo": index-score
+ *             formula, ReLU, 128-element FP8 blocks, non-interleaved indexer RoPE.
+ *   [rope]    "DeepSeek-V3.2-Exp - RoPE coefficients": YaRN precompute excerpt, ModelArgs.
+ *   [dense]   "DeepSeek-V3.2-Exp - Dense transformer block, Sparse latent attention": the
+ *             43-step equation list (indexer steps, sparse attention steps, m = 1 + 0.1 ln 40).
+ *   [rotate]  "DeepSeek-V3.2-Exp - Rotate first features": Indexer.forward (model.py 457-487),
+ *             apply_rotary_emb (model.py 405-425).
+ *   [sim]     "DeepSeek-V3.2-Exp - Similarities": absorbed MQA decode (model.py 590-606).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers unless a comment says "host". The caller owns
+ *     every buffer; the library allocates nothing in these calls and keeps no per-call state.
+ *   - Calls are asynchronous and ordered on `stream` (NULL = the legacy default stream).
+ *   - Return value: DSA_OK, or an error code for arguments rejected on the host before any
+ *     launch (nothing is launched then) or a failed launch. Errors found on the device
+ *     (index or position out of range, a bounded wait that ran out) are recorded in a device
+ *     status word and reported by dsa_get_device_status().
+ *   - Pointers must be 16-byte aligned; sizes are in elements unless stated.
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - No C++ exception crosses this boundary and nothing aborts or traps.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+typedef struct CUstream_st* dsa_stream_t; /* a cudaStream_t */
+
+/* Status codes */
+#define DSA_OK 0
+#define DSA_ERR_INVALID_ARG 1   /* null/misaligned pointer or bad size; nothing launched       */
+#define DSA_ERR_UNSUPPORTED 2   /* device is not sm_100 (B200 class)                           */
+#define DSA_ERR_CUDA 3          /* a CUDA runtime call or kernel launch failed                 */
+#define DSA_ERR_TIMEOUT 4       /* device: a bounded wait gave up (status word)                */
+#define DSA_ERR_DEVICE_BOUNDS 5 /* device: a position or index outside its buffer (status word) */
+#define DSA_ERR_WORKSPACE 6     /* workspace pointer null or smaller than the size query says   */
+
+/* Fixed model dimensions (ModelArgs of DeepSeek-V3.2-Exp, [rope] model-args excerpt; [dense]) */
+#define DSA_INDEX_HEADS 64      /* H_I */
+#define DSA_INDEX_DIM 128       /* indexer head dim = one FP8 block */
+#define DSA_ROPE_PAIRS 32       /* qk_rope_head_dim / 2 */
+#define DSA_MLA_HEADS 128
+#define DSA_MLA_LATENT 512      /* kv_lora_rank: the value / output width */
+#define DSA_MLA_ROPE 64
+#define DSA_MLA_QK 576          /* latent + rotary key width */
+#define DSA_MAX_POS 1048576     /* positions accepted by dsa_rope_table / dsa_index_keys */
+#define DSA_TOPK_MAX_ROW 32768  /* longest score row dsa_topk accepts (kept in shared memory) */
+
+/* Flags */
+#define DSA_HADAMARD 0x1u      /* dsa_index_keys: apply (1/sqrt 128) H_128 after RoPE ([dense]
+                                  indexer steps; rotate_activation in Indexer.forward)         */
+#define DSA_FILL_MASKED 0x2u   /* dsa_index_scores: write -inf at masked (s > pos) entries of
+                                  each row up to S_max (the mask add of Indexer.forward)       */
+
+/*
+ * dsa_rope_table - HOST function. Writes the (cos, sin) table of the 32 rotary frequencies,
+ * fp32 [max_pos][32][2], into the HOST buffer `table`.
+ * Frequencies: theta^(-2i/64), theta = 1e4, blended by YaRN (factor 40, beta_fast 32, beta_slow 1,
+ * original length 4096; always on because max_seq_len 16384 > 4096) as in the precompute excerpt
+ * of [rope]; the correction-range and ramp helpers (omitted on the page) follow the YaRN paper.
+ * angle = fp32(pos * fp32(freq)); cos/sin evaluated in double and rounded to fp32.
+ * Returns DSA_ERR_INVALID_ARG if table is NULL or max_pos is outside [1, DSA_MAX_POS].
+ */
+DSA_API int dsa_rope_table(float* table, int max_pos);
+
+/*
+ * dsa_index_keys - indexer query/key transform and block FP8 quantisation
+ * ([rotate] Indexer.forward: RoPE on q_pe/k_pe with interleaved=False, rotate_activation,
+ * act_quant, k_cache / k_scale_cache write; [news] 128-element blocks).
+ *
+ *   x        fp32 [rows][heads][128]   rows = tokens; heads = 64 for queries, 1 for keys
+ *   pos      int32 [rows]              absolute position of each row (0 <= pos < max_pos)
+ *   rope_cs  fp32 [max_pos][32][2]     table from dsa_rope_table (copied to the device)
+ *   flags    DSA_HADAMARD or 0
+ *   out_fp8  uint8 e4m3 codes; out_scale fp32 scales (one per 128-block)
+ *   dst_row  int64 [rows] or NULL. NULL: outputs are dense, [rows][heads][128] and
+ *            [rows][heads]. Otherwise row r is written to out_fp8 + dst_row[r]*heads*128 and
+ *            out_scale + dst_row[r]*heads (e.g. dst_row = b*S_max + pos for a K-cache
+ *            [B][S_max][128]); dst_row values must be >= 0 and distinct and lie inside
+ *            the caller's buffers (not checked).
+ * Per 128-block: features j<32 pair with j+32 and rotate by pos*freq_j (fp32 arithmetic);
+ * features 64..127 pass through; optional Hadamard; amax = max(|y|, 1e-4);
+ * scale = amax / 448 (IEEE fp32 division); code = e4m3 round-to-nearest-even, saturating, of
+ * the IEEE fp32 quotient y / scale.
+ * A pos outside [0, max_pos) sets DSA_ERR_DEVICE_BOUNDS and leaves that row unwritten.
+ */
+DSA_API int dsa_index_keys(const float* x, int64_t rows, int heads, const int32_t* pos,
+                   const float* rope_cs, int max_pos, uint32_t flags,
+                   uint8_t* out_fp8, float* out_scale, const int64_t* dst_row,
+                   dsa_stream_t stream);
+
+/*
+ * dsa_index_scores - lightning-indexer scores (fp8_index in Indexer.forward; [dense]
+ * S^I_{t,s} = 1/(sqrt 64 sqrt 128) sum_h w_{t,h} ReLU(Q^I_{h,t} . k^I_s)).
+ *
+ *   q8       uint8 e4m3 [B][T][64][128]     q_scale fp32 [B][T][64]
+ *   w        fp32 [B][T][64]                raw head weights (weights_proj output)
+ *   k8       uint8 e4m3 [B][S_max][128]     K-cache;  k_scale fp32 [B][S_max]
+ *   q_pos    int32 [B][T]   position of each query; kv_len int32 [B] keys present
+ *   scores   fp32 [B][T][ld], ld >= S_max, ld a multiple of 4
+ * scores[b][t][s] = k_scale[b][s] * sum_j w'[b][t][j] * max(0, sum_i q8[b][t][j][i]*k8[b][s][i])
+ * with w' = w * 64^-0.5 * q_scale * softmax_scale (softmax_scale = 128^-0.5 in the model), for
+ * every visible s: s <= q_pos[b][t] and s < kv_len[b] (the causal mask; decode passes the last
+ * position). Other entries are left untouched, or set to -inf with DSA_FILL_MASKED.
+ * Products accumulate in fp32 on the tensor cores (kind::f8f6f4).
+ * Constraints: B, T >= 1; 1 <= S_max; q_pos and kv_len within [0, S_max] (kv_len) and
+ * [-1, S_max) (q_pos; -1 = no visible key). Not checked on the device beyond masking.
+ */
+DSA_API int dsa_index_scores(const uint8_t* q8, const float* q_scale, const float* w,
+                     const uint8_t* k8, const float* k_scale,
+                     const int32_t* q_pos, const int32_t* kv_len,
+                     int B, int T, int S_max, float softmax_scale,
+                     float* scores, int64_t ld, uint32_t flags, dsa_stream_t stream);
+
+/*
+ * dsa_topk - per query, the min(k, n_valid) visible positions with the largest scores
+ * (index_score.topk(min(index_topk, end_pos)) after the mask in Indexer.forward; [dense]
+ * top_2048). n_valid = min(q_pos+1, kv_len). Only visible entries of `scores` are read.
+ *
+ *   scores fp32 [B][T][ld];  idx int32 [B][T][k] (output)
+ * Ties go to the smaller position. The selected positions are written in ascending order,
+ * then -1 up to k. NaN scores are not allowed. -0.0 and +0.0 compare equal.
+ * Constraints: 1 <= k; every row's n_valid <= DSA_TOPK_MAX_ROW (ld may be larger).
+ */
+DSA_API int dsa_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int32_t* kv_len,
+             int B, int T, int k, int32_t* idx, dsa_stream_t stream);
+
+/*
+ * dsa_sparse_mla - sparse MQA-style latent attention over the selected positions
+ * ([sim] MQA decode: scores over the latent and rotary parts, index mask, softmax, latent-
+ * weighted sum; [dense] sparse attention steps S' = S m^2 / sqrt 192; the MLA prefill excerpt
+ * in [rope] computed in the same absorbed form).
+ *
+ *   q      bf16 [B][T][128][576]   absorbed query: 512 latent features then 64 rotary
+ *   kv     bf16 [B][S_max][576]    latent cache row = 512 latent features then 64 rotary key
+ *   idx    int32 [B][T][k]         selected positions (distinct; -1 = unused slot)
+ *   out    bf16 [B][T][128][512];  lse fp32 [B][T][128] or NULL (natural log)
+ *   workspace / ws_bytes: device scratch of at least dsa_sparse_mla_workspace_size(B, T, k)
+ *          bytes (may be NULL when that size is 0)
+ * For each (b, t, head h): z_u = softmax_scale * q[h] . kv[idx_u] over all 576 features,
+ * p = softmax(z) over the slots with idx_u >= 0, out[h] = sum_u p_u * kv[idx_u][0:512].
+ * In the model softmax_scale = 192^-0.5 * (1 + 0.1 ln 40)^2. A row with no selected position
+ * writes zeros and lse = -inf. An idx >= S_max sets DSA_ERR_DEVICE_BOUNDS (that slot is skipped).
+ */
+DSA_API int dsa_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
+                   int B, int T, int S_max, int k, float softmax_scale,
+                   uint16_t* out, float* lse, void* workspace, size_t ws_bytes,
+                   dsa_stream_t stream);
+
+/* Bytes of device scratch dsa_sparse_mla needs for this shape (0 when it needs none). */
+DSA_API size_t dsa_sparse_mla_workspace_size(int B, int T, int k);
+
+/*
+ * dsa_get_device_status - synchronises `stream`, returns the first error recorded by a kernel
+ * since the last call (DSA_OK if none) and clears it. DSA_ERR_CUDA if the sync itself fails.
+ */
+DSA_API int dsa_get_device_status(dsa_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+DSA_API const char* dsa_status_string(int code);
+
+/* 1 if the current device is sm_100 (B200 class) and the library's kernels can run on it. */
+DSA_API int dsa_device_supported(void);
+
+/* Library version string. */
+DSA_API const char* dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

@@ -204,6 +204,14 @@ def act_quant(x):
     return e4m3_encode(q), scale
 
 
+def index_keys_prequant(x, pos, table, hadamard: bool = True) -> np.ndarray:
+    """The fp32 rows act_quant receives in index_keys (RoPE_64, optional Hadamard, rounded to fp32)."""
+    y = rope_noninterleaved(x, pos, table)
+    if hadamard:
+        y = hadamard_rotate(y)
+    return y.astype(np.float32)
+
+
 def index_keys(x, pos, table, hadamard: bool = True):
     """Indexer q or k transform of Indexer.forward up to act_quant.
 
@@ -211,10 +219,7 @@ def index_keys(x, pos, table, hadamard: bool = True):
     RoPE_64 (non-interleaved) then, if ``hadamard``, (1/sqrt 128) H_128, both in float64;
     READING: the rotated row is rounded to fp32 (the activation dtype) before act_quant.
     """
-    y = rope_noninterleaved(x, pos, table)
-    if hadamard:
-        y = hadamard_rotate(y)
-    return act_quant(y.astype(np.float32))
+    return act_quant(index_keys_prequant(x, pos, table, hadamard))
 
 
 # ----------------------------------------------------------------------------------------------
@@ -250,7 +255,8 @@ def index_scores(q8, q_scale, w, k8, k_scale, q_pos, kv_len,
     for b in range(B):
         for t0 in range(0, T, 64):        # query rows in groups, only to bound memory
             t1 = min(T, t0 + 64)
-            dots = np.einsum("thd,sd->ths", q[b, t0:t1], k[b])      # exact
+            n = t1 - t0
+            dots = (q[b, t0:t1].reshape(n * H, -1) @ k[b].T).reshape(n, H, S)   # exact
             relu = np.maximum(dots, 0.0)
             score = np.einsum("th,ths->ts", wf[b, t0:t1], relu) * ks[b][None, :]
             for t in range(t0, t1):
@@ -272,7 +278,8 @@ def index_score_magnitude(q8, q_scale, w, k8, k_scale, q_pos, kv_len,
     for b in range(B):
         for t0 in range(0, T, 64):
             t1 = min(T, t0 + 64)
-            relu = np.maximum(np.einsum("thd,sd->ths", q[b, t0:t1], k[b]), 0.0)
+            n = t1 - t0
+            relu = np.maximum((q[b, t0:t1].reshape(n * H, -1) @ k[b].T).reshape(n, H, -1), 0.0)
             out[b, t0:t1] = np.einsum("th,ths->ts", wf[b, t0:t1], relu) * ks[b][None, :]
     return out
 

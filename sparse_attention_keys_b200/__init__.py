@@ -1,0 +1,208 @@
+"""Python binding of libdsa, the sm_100a hot path of DeepSeek Sparse Attention.
+
+Thin ctypes marshalling over the C ABI declared in include/dsa.h: every function takes torch
+tensors (device memory owned by the caller, or allocated here with torch.empty as plumbing),
+passes raw pointers and sizes, and raises DsaError on a non-zero status. All arithmetic runs in
+the library's CUDA kernels; there is no fallback path. Names follow the C entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "DsaError", "lib", "lib_path", "DSA_HADAMARD", "DSA_FILL_MASKED", "INDEXER_SOFTMAX_SCALE",
+    "MLA_SOFTMAX_SCALE", "dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk",
+    "dsa_sparse_mla", "dsa_sparse_mla_workspace_size", "dsa_get_device_status", "dsa_status_string",
+    "dsa_device_supported", "dsa_version",
+]
+
+DSA_OK = 0
+DSA_HADAMARD = 0x1
+DSA_FILL_MASKED = 0x2
+MAX_POS = 16384                 # max_seq_len of the model (ModelArgs)
+INDEXER_SOFTMAX_SCALE = 128 ** -0.5
+MLA_SOFTMAX_SCALE = 192 ** -0.5 * (1.0 + 0.1 * __import__("math").log(40.0)) ** 2
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libdsa.so")
+
+
+class DsaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {dsa_status_string(code) if _lib is not None else code}")
+
+
+def _load():
+    if not os.path.exists(lib_path):
+        raise ImportError(f"libdsa.so not built at {lib_path}; run `python -m sparse_attention_keys_b200.build`")
+    L = ctypes.CDLL(lib_path)
+    vp, i32, i64, u32, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint32,
+                                  ctypes.c_float, ctypes.c_size_t)
+    L.dsa_rope_table.argtypes = [vp, i32]
+    L.dsa_index_keys.argtypes = [vp, i64, i32, vp, vp, i32, u32, vp, vp, vp, vp]
+    L.dsa_index_scores.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, f32, vp, i64, u32, vp]
+    L.dsa_topk.argtypes = [vp, i64, vp, vp, i32, i32, i32, vp, vp]
+    L.dsa_sparse_mla.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
+    L.dsa_sparse_mla_workspace_size.argtypes = [i32, i32, i32]
+    L.dsa_sparse_mla_workspace_size.restype = sz
+    L.dsa_get_device_status.argtypes = [vp]
+    L.dsa_status_string.argtypes = [i32]
+    L.dsa_status_string.restype = ctypes.c_char_p
+    L.dsa_device_supported.argtypes = []
+    L.dsa_version.restype = ctypes.c_char_p
+    for f in ("dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk", "dsa_sparse_mla",
+              "dsa_get_device_status", "dsa_device_supported"):
+        getattr(L, f).restype = ctypes.c_int
+    return L
+
+
+_lib = _load()
+lib = _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(rc: int, what: str):
+    if rc != DSA_OK:
+        raise DsaError(rc, what)
+
+
+def _need(t, dtype, name, device=True):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def dsa_status_string(code: int) -> str:
+    return _lib.dsa_status_string(int(code)).decode()
+
+
+def dsa_version() -> str:
+    return _lib.dsa_version().decode()
+
+
+def dsa_device_supported() -> bool:
+    return bool(_lib.dsa_device_supported())
+
+
+def dsa_rope_table(max_pos: int = MAX_POS) -> torch.Tensor:
+    """(cos, sin) YaRN table, fp32 [max_pos, 32, 2], in HOST memory (computed by the library)."""
+    out = torch.empty((max_pos, 32, 2), dtype=torch.float32)
+    _check(_lib.dsa_rope_table(_ptr(out), int(max_pos)), "dsa_rope_table")
+    return out
+
+
+def dsa_index_keys(x, pos, rope_cs, flags: int = DSA_HADAMARD, out_fp8=None, out_scale=None,
+                   dst_row=None, stream=None):
+    """x fp32 [rows, heads, 128] (or [rows, 128] for keys) -> (codes uint8, scales fp32).
+
+    With dst_row (int64 [rows]) the outputs are written into the given cache tensors at those rows.
+    """
+    _need(x, torch.float32, "x")
+    _need(pos, torch.int32, "pos")
+    _need(rope_cs, torch.float32, "rope_cs")
+    if x.shape[-1] != 128:
+        raise ValueError("last dim of x must be 128")
+    rows = x.shape[0]
+    heads = 1 if x.dim() == 2 else int(x[0].numel() // 128)
+    if pos.numel() != rows:
+        raise ValueError("pos must have one entry per row of x")
+    if dst_row is None:
+        if out_fp8 is None:
+            out_fp8 = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+        if out_scale is None:
+            out_scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    else:
+        _need(dst_row, torch.int64, "dst_row")
+        if out_fp8 is None or out_scale is None:
+            raise ValueError("dst_row needs the destination out_fp8 and out_scale tensors")
+    _need(out_fp8, torch.uint8, "out_fp8")
+    _need(out_scale, torch.float32, "out_scale")
+    rc = _lib.dsa_index_keys(_ptr(x), rows, heads, _ptr(pos), _ptr(rope_cs), rope_cs.shape[0], int(flags),
+                             _ptr(out_fp8), _ptr(out_scale), _ptr(dst_row), _stream(stream))
+    _check(rc, "dsa_index_keys")
+    return out_fp8, out_scale
+
+
+def dsa_index_scores(q8, q_scale, w, k8, k_scale, q_pos, kv_len, softmax_scale: float = INDEXER_SOFTMAX_SCALE,
+                     scores=None, ld=None, flags: int = 0, stream=None):
+    """q8 [B,T,64,128] u8, q_scale/w [B,T,64] f32, k8 [B,S,128] u8, k_scale [B,S] f32,
+    q_pos [B,T] i32, kv_len [B] i32 -> scores fp32 [B,T,ld]."""
+    for t, dt, n in ((q8, torch.uint8, "q8"), (q_scale, torch.float32, "q_scale"), (w, torch.float32, "w"),
+                     (k8, torch.uint8, "k8"), (k_scale, torch.float32, "k_scale"), (q_pos, torch.int32, "q_pos"),
+                     (kv_len, torch.int32, "kv_len")):
+        _need(t, dt, n)
+    B, T = q8.shape[0], q8.shape[1]
+    S = k8.shape[1]
+    if ld is None:
+        ld = (S + 3) // 4 * 4
+    if scores is None:
+        scores = torch.empty((B, T, ld), dtype=torch.float32, device=q8.device)
+    _need(scores, torch.float32, "scores")
+    rc = _lib.dsa_index_scores(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale), _ptr(q_pos),
+                               _ptr(kv_len), B, T, S, float(softmax_scale), _ptr(scores), int(ld), int(flags),
+                               _stream(stream))
+    _check(rc, "dsa_index_scores")
+    return scores
+
+
+def dsa_topk(scores, q_pos, kv_len, k: int, idx=None, stream=None):
+    """scores fp32 [B,T,ld] -> idx int32 [B,T,k] (ascending positions, -1 padded)."""
+    _need(scores, torch.float32, "scores")
+    _need(q_pos, torch.int32, "q_pos")
+    _need(kv_len, torch.int32, "kv_len")
+    B, T, ld = scores.shape
+    if idx is None:
+        idx = torch.empty((B, T, k), dtype=torch.int32, device=scores.device)
+    _need(idx, torch.int32, "idx")
+    rc = _lib.dsa_topk(_ptr(scores), int(ld), _ptr(q_pos), _ptr(kv_len), B, T, int(k), _ptr(idx), _stream(stream))
+    _check(rc, "dsa_topk")
+    return idx
+
+
+def dsa_sparse_mla_workspace_size(B: int, T: int, k: int) -> int:
+    return int(_lib.dsa_sparse_mla_workspace_size(int(B), int(T), int(k)))
+
+
+def dsa_sparse_mla(q, kv, idx, softmax_scale: float = MLA_SOFTMAX_SCALE, out=None, lse=None, workspace=None,
+                   want_lse: bool = True, stream=None):
+    """q bf16 [B,T,128,576], kv bf16 [B,S,576], idx int32 [B,T,k] -> (out bf16 [B,T,128,512], lse fp32)."""
+    _need(q, torch.bfloat16, "q")
+    _need(kv, torch.bfloat16, "kv")
+    _need(idx, torch.int32, "idx")
+    B, T = q.shape[0], q.shape[1]
+    S = kv.shape[1]
+    k = idx.shape[-1]
+    if out is None:
+        out = torch.empty((B, T, 128, 512), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, T, 128), dtype=torch.float32, device=q.device)
+    ws_bytes = dsa_sparse_mla_workspace_size(B, T, k)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    rc = _lib.dsa_sparse_mla(_ptr(q), _ptr(kv), _ptr(idx), B, T, S, int(k), float(softmax_scale), _ptr(out),
+                             _ptr(lse), _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                             _stream(stream))
+    _check(rc, "dsa_sparse_mla")
+    return out, lse
+
+
+def dsa_get_device_status(stream=None) -> int:
+    return int(_lib.dsa_get_device_status(_stream(stream)))

@@ -1,0 +1,267 @@
+// C ABI of libdsa: argument validation, the device status word, and dispatch to the kernels.
+// Declarations and contracts: include/dsa.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "dsa.h"
+#include "kernels.h"
+
+namespace {
+
+__device__ int g_dsa_status = 0;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceCache {
+  bool init = false;
+  bool supported = false;
+  int sms = 0;
+  int* status = nullptr;
+};
+DeviceCache g_dev[kMaxDevices];
+std::mutex g_mu;
+
+DeviceCache* device_cache() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  DeviceCache& c = g_dev[dev];
+  if (!c.init) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!c.init) {
+      cudaDeviceProp prop;
+      if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return nullptr;
+      c.supported = prop.major == 10 && prop.minor == 0;
+      c.sms = prop.multiProcessorCount;
+      void* addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_dsa_status) != cudaSuccess) return nullptr;
+      c.status = static_cast<int*>(addr);
+      c.init = true;
+    }
+  }
+  return &c;
+}
+
+// Common prologue: device is sm_100 and the status word is reachable.
+int prologue(int** status) {
+  DeviceCache* c = device_cache();
+  if (!c) return DSA_ERR_CUDA;
+  if (!c->supported) return DSA_ERR_UNSUPPORTED;
+  *status = c->status;
+  return DSA_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+namespace dsa_host {
+
+int* status_word() {
+  DeviceCache* c = device_cache();
+  return c ? c->status : nullptr;
+}
+
+int check_launch() { return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int device_sm_count() {
+  DeviceCache* c = device_cache();
+  return (c && c->sms > 0) ? c->sms : 148;
+}
+
+bool encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, void* base, uint64_t inner,
+                          uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                          CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dtype, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace dsa_host
+
+// ------------------------------------------------------------------------------------------------
+// Host-side RoPE table: YaRN frequencies of the "RoPE coefficients" precompute excerpt; the
+// correction range and linear ramp follow the YaRN paper (their bodies are omitted on the page).
+// ------------------------------------------------------------------------------------------------
+namespace {
+
+double yarn_correction_dim(double rotations, int dim, double base, double max_pos) {
+  return dim * log(max_pos / (rotations * 2.0 * M_PI)) / (2.0 * log(base));
+}
+
+void yarn_freqs(double out[DSA_ROPE_PAIRS]) {
+  const int dim = 2 * DSA_ROPE_PAIRS;            // qk_rope_head_dim = 64
+  const double base = 10000.0, factor = 40.0;
+  const double beta_fast = 32.0, beta_slow = 1.0, original = 4096.0;
+  const int max_seq_len = 16384;
+  double low = floor(yarn_correction_dim(beta_fast, dim, base, original));
+  double high = ceil(yarn_correction_dim(beta_slow, dim, base, original));
+  if (low < 0) low = 0;
+  if (high > dim - 1) high = dim - 1;
+  if (low == high) high += 0.001;
+  for (int i = 0; i < DSA_ROPE_PAIRS; ++i) {
+    const double f = 1.0 / pow(base, (2.0 * i) / dim);
+    double ramp = (i - low) / (high - low);
+    ramp = ramp < 0 ? 0 : (ramp > 1 ? 1 : ramp);
+    const double smooth = 1.0 - ramp;
+    out[i] = (max_seq_len > original) ? f / factor * (1.0 - smooth) + f * smooth : f;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int dsa_rope_table(float* table, int max_pos) {
+  if (!table || max_pos < 1 || max_pos > DSA_MAX_POS) return DSA_ERR_INVALID_ARG;
+  double f[DSA_ROPE_PAIRS];
+  yarn_freqs(f);
+  float f32[DSA_ROPE_PAIRS];
+  for (int i = 0; i < DSA_ROPE_PAIRS; ++i) f32[i] = (float)f[i];
+  for (int p = 0; p < max_pos; ++p) {
+    for (int i = 0; i < DSA_ROPE_PAIRS; ++i) {
+      const float ang = (float)p * f32[i];           // fp32 product, as the page's float32 outer
+      table[((size_t)p * DSA_ROPE_PAIRS + i) * 2 + 0] = (float)cos((double)ang);
+      table[((size_t)p * DSA_ROPE_PAIRS + i) * 2 + 1] = (float)sin((double)ang);
+    }
+  }
+  return DSA_OK;
+}
+
+int dsa_index_keys(const float* x, int64_t rows, int heads, const int32_t* pos, const float* rope_cs,
+                   int max_pos, uint32_t flags, uint8_t* out_fp8, float* out_scale,
+                   const int64_t* dst_row, dsa_stream_t stream) {
+  if (rows < 0 || heads < 1 || heads > 4096 || max_pos < 1 || max_pos > DSA_MAX_POS ||
+      (flags & ~DSA_HADAMARD) != 0)
+    return DSA_ERR_INVALID_ARG;
+  if (rows == 0) return DSA_OK;
+  if (!x || !pos || !rope_cs || !out_fp8 || !out_scale) return DSA_ERR_INVALID_ARG;
+  if (!dsa_host::aligned16(x) || !dsa_host::aligned16(rope_cs) || !dsa_host::aligned16(out_fp8) ||
+      !dsa_host::aligned16(out_scale) || (dst_row && !dsa_host::aligned16(dst_row)) ||
+      !dsa_host::aligned16(pos))
+    return DSA_ERR_INVALID_ARG;
+  int* status;
+  int rc = prologue(&status);
+  if (rc != DSA_OK) return rc;
+  return dsa::launch_index_keys(x, rows, heads, pos, rope_cs, max_pos, flags, out_fp8, out_scale,
+                                dst_row, (cudaStream_t)stream, status);
+}
+
+int dsa_index_scores(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8,
+                     const float* k_scale, const int32_t* q_pos, const int32_t* kv_len, int B, int T,
+                     int S_max, float softmax_scale, float* scores, int64_t ld, uint32_t flags,
+                     dsa_stream_t stream) {
+  if (B < 1 || T < 1 || S_max < 1 || ld < S_max || (ld & 3) != 0 || (flags & ~DSA_FILL_MASKED) != 0 ||
+      !(softmax_scale > 0.f) || !isfinite(softmax_scale))
+    return DSA_ERR_INVALID_ARG;
+  if ((int64_t)B * T * 64 > 0x7fffffffLL || (int64_t)B * S_max > 0x7fffffffLL) return DSA_ERR_INVALID_ARG;
+  if (!q8 || !q_scale || !w || !k8 || !k_scale || !q_pos || !kv_len || !scores) return DSA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q8, q_scale, w, k8, k_scale, q_pos, kv_len, scores};
+  for (const void* p : ptrs)
+    if (!dsa_host::aligned16(p)) return DSA_ERR_INVALID_ARG;
+  int* status;
+  int rc = prologue(&status);
+  if (rc != DSA_OK) return rc;
+  return dsa::launch_index_scores(q8, q_scale, w, k8, k_scale, q_pos, kv_len, B, T, S_max, softmax_scale,
+                                  scores, ld, flags, (cudaStream_t)stream, status);
+}
+
+int dsa_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int32_t* kv_len, int B, int T,
+             int k, int32_t* idx, dsa_stream_t stream) {
+  if (B < 1 || T < 1 || k < 1 || ld < 1 || (ld & 3) != 0) return DSA_ERR_INVALID_ARG;
+  if ((int64_t)B * T > 0x7fffffffLL) return DSA_ERR_INVALID_ARG;
+  if (!scores || !q_pos || !kv_len || !idx) return DSA_ERR_INVALID_ARG;
+  if (!dsa_host::aligned16(scores) || !dsa_host::aligned16(q_pos) || !dsa_host::aligned16(kv_len) ||
+      !dsa_host::aligned16(idx))
+    return DSA_ERR_INVALID_ARG;
+  int* status;
+  int rc = prologue(&status);
+  if (rc != DSA_OK) return rc;
+  return dsa::launch_topk(scores, ld, q_pos, kv_len, B, T, k, idx, (cudaStream_t)stream, status);
+}
+
+size_t dsa_sparse_mla_workspace_size(int B, int T, int k) {
+  if (B < 1 || T < 1 || k < 1) return 0;
+  return dsa::sparse_mla_workspace_size(B, T, k);
+}
+
+int dsa_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T, int S_max,
+                   int k, float softmax_scale, uint16_t* out, float* lse, void* workspace,
+                   size_t ws_bytes, dsa_stream_t stream) {
+  if (B < 1 || T < 1 || S_max < 1 || k < 1 || !(softmax_scale > 0.f) || !isfinite(softmax_scale))
+    return DSA_ERR_INVALID_ARG;
+  if ((int64_t)B * T * 2 * 1024 > 0x7fffffffLL) return DSA_ERR_INVALID_ARG;
+  if (!q || !kv || !idx || !out) return DSA_ERR_INVALID_ARG;
+  if (!dsa_host::aligned16(q) || !dsa_host::aligned16(kv) || !dsa_host::aligned16(idx) ||
+      !dsa_host::aligned16(out) || (lse && !dsa_host::aligned16(lse)) ||
+      (workspace && !dsa_host::aligned16(workspace)))
+    return DSA_ERR_INVALID_ARG;
+  int* status;
+  int rc = prologue(&status);
+  if (rc != DSA_OK) return rc;
+  return dsa::launch_sparse_mla(q, kv, idx, B, T, S_max, k, softmax_scale, out, lse, workspace, ws_bytes,
+                                (cudaStream_t)stream, status);
+}
+
+int dsa_get_device_status(dsa_stream_t stream) {
+  DeviceCache* c = device_cache();
+  if (!c) return DSA_ERR_CUDA;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return DSA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, c->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return DSA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(c->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return DSA_ERR_CUDA;
+  }
+  return v;
+}
+
+const char* dsa_status_string(int code) {
+  switch (code) {
+    case DSA_OK: return "DSA_OK";
+    case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG";
+    case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED";
+    case DSA_ERR_CUDA: return "DSA_ERR_CUDA";
+    case DSA_ERR_TIMEOUT: return "DSA_ERR_TIMEOUT";
+    case DSA_ERR_DEVICE_BOUNDS: return "DSA_ERR_DEVICE_BOUNDS";
+    case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE";
+    default: return "DSA_ERR_UNKNOWN";
+  }
+}
+
+int dsa_device_supported(void) {
+  DeviceCache* c = device_cache();
+  return (c && c->supported) ? 1 : 0;
+}
+
+const char* dsa_version(void) { return "dsa-b200 0.1.0"; }
+
+}  // extern "C"

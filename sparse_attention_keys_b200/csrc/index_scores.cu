@@ -1,0 +1,268 @@
+// dsa_index_scores: lightning-indexer scores on the FP8 tensor cores (tcgen05, kind::f8f6f4).
+//
+// Computes I[b,t,s] = k_scale[b,s] * sum_j w'[b,t,j] * ReLU(q8[b,t,j,:] . k8[b,s,:]) for every
+// visible s (s <= q_pos, s < kv_len), w' = w * 64^-0.5 * q_scale * softmax_scale: the fp8_index
+// call and weight fold of Indexer.forward ("DeepSeek-V3.2-Exp - Rotate first features",
+// model.py 457-487 excerpt) and S^I of the lightning-indexer steps (dense-block page).
+//
+// Tile: the MMA's M = 128 keys (A = K-cache rows, K-major, 128 B each = one 128B-swizzle atom
+// row), N = NQ queries x 64 heads (B = the queries' FP8 head rows), K = 128 (4 MMAs of K=32).
+// Each TMEM lane then holds one key and its N (query, head) dot products, so the ReLU and the
+// weighted head-sum are an in-thread reduction over TMEM columns and the [T, 64, S] tensor of
+// per-head products never leaves the SM. The CTA keeps its NQ queries resident and streams
+// 16 KB key tiles through a TMA ring (one warp), one thread issues the MMAs into two TMEM
+// accumulators (ping-pong), and four epilogue warps drain TMEM while the next tile multiplies.
+// Key tiles above the causal diagonal of the CTA's queries are never loaded.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kKeysPerTile = 128;
+constexpr int kTileBytes = kKeysPerTile * 128;      // 16 KB of e4m3 keys
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = (kEpiWarps + 2) * 32;      // + TMA warp + MMA warp
+
+template <int NQ>
+struct ScoresCfg {
+  static constexpr int N = NQ * 64;                 // MMA N: (query, head) columns
+  static constexpr int kStages = NQ >= 4 ? 6 : 4;
+  static constexpr int kQBytes = N * 128;
+  static constexpr int kTmemCols = 2 * N;           // two accumulators
+  static constexpr int kSmemBytes = 1024 /*align slack*/ + kQBytes + kStages * kTileBytes + 1024;
+};
+
+struct ScoresParams {
+  const float* q_scale;
+  const float* w;
+  const float* k_scale;
+  const int32_t* q_pos;
+  const int32_t* kv_len;
+  float* scores;
+  int64_t ld;
+  int B, T, S_max;
+  int groups;          // query groups per sequence = ceil(T / NQ)
+  int ksplit;          // CTAs sharing one query group's key tiles
+  int tiles_per_split;
+  float wscale;        // 64^-0.5 * softmax_scale
+  uint32_t flags;
+  int* status;
+};
+
+}  // namespace
+
+template <int NQ>
+__global__ void __launch_bounds__(kThreads, 1)
+    index_scores_kernel(const __grid_constant__ CUtensorMap qmap,
+                        const __grid_constant__ CUtensorMap kmap, const ScoresParams p) {
+  using Cfg = ScoresCfg<NQ>;
+  constexpr int N = Cfg::N;
+  constexpr int STAGES = Cfg::kStages;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_smem = smem;                                   // [N rows][128 B], 128B swizzle
+  uint8_t* k_smem = smem + Cfg::kQBytes;                    // STAGES x [128 rows][128 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(k_smem + STAGES * kTileBytes);
+  uint64_t* full = bars;                                    // [STAGES] TMA -> MMA
+  uint64_t* empty = bars + STAGES;                          // [STAGES] MMA -> TMA
+  uint64_t* acc_full = bars + 2 * STAGES;                   // [2]      MMA -> epilogue
+  uint64_t* acc_empty = bars + 2 * STAGES + 2;              // [2]      epilogue -> MMA
+  uint64_t* q_full = bars + 2 * STAGES + 4;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+  __shared__ float wq[NQ][64];
+  __shared__ int nvalid[NQ];
+  __shared__ int ntiles_sh;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Heavy (late, long-context) query groups first so the causal tail is short.
+  const int unit = blockIdx.x / p.ksplit;
+  const int split = blockIdx.x - unit * p.ksplit;
+  const int b = unit / p.groups;
+  const int g = p.groups - 1 - (unit - b * p.groups);
+  const int t0 = g * NQ;
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], kEpiWarps * 32); }
+    mbar_init(q_full, 1);
+    fence_barrier_init();
+  }
+  if (warp == kEpiWarps + 1) {           // MMA warp owns the TMEM allocation
+    tmem_alloc(&tmem_base_sh, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i < NQ * 64; i += kThreads) {   // folded head weights
+    const int q = i >> 6, j = i & 63;
+    const int t = t0 + q;
+    float v = 0.f;
+    if (t < p.T) {
+      const int64_t o = ((int64_t)b * p.T + t) * 64 + j;
+      v = __fmul_rn(__fmul_rn(p.w[o], p.q_scale[o]), p.wscale);
+    }
+    wq[q][j] = v;
+  }
+  if (threadIdx.x < NQ) {
+    const int t = t0 + threadIdx.x;
+    int n = 0;
+    if (t < p.T) n = max(0, min(min(p.q_pos[(int64_t)b * p.T + t] + 1, p.kv_len[b]), p.S_max));
+    nvalid[threadIdx.x] = n;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0) {
+    int nmax = 0;
+    for (int q = 0; q < NQ; ++q) nmax = max(nmax, nvalid[q]);
+    ntiles_sh = (nmax + kKeysPerTile - 1) / kKeysPerTile;
+  }
+  __syncthreads();
+  const uint32_t tmem_base = tmem_base_sh;
+  const int kt_begin = split * p.tiles_per_split;
+  const int kt_end = min(ntiles_sh, kt_begin + p.tiles_per_split);
+  const int my_tiles = max(0, kt_end - kt_begin);
+
+  if (warp == kEpiWarps) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && my_tiles > 0) {
+      prefetch_tensormap(&qmap);
+      prefetch_tensormap(&kmap);
+      mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
+      tma_load_2d(q_smem, &qmap, q_full, 0, (b * p.T + t0) * 64);
+      for (int i = 0; i < my_tiles; ++i) {
+        const int s = i % STAGES;
+        if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) + 1) & 1, &abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(&full[s], kTileBytes);
+        tma_load_2d(k_smem + s * kTileBytes, &kmap, &full[s], 0,
+                    b * p.S_max + (kt_begin + i) * kKeysPerTile);
+      }
+    }
+  } else if (warp == kEpiWarps + 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && my_tiles > 0) {
+      constexpr uint32_t idesc = idesc_f32acc(0 /*E4M3*/, 0 /*E4M3*/, 128, N, 0, 0);
+      const uint32_t q_addr = smem_u32(q_smem);
+      bool ok = mbar_wait(q_full, 0, &abort_flag, p.status);
+      for (int i = 0; ok && i < my_tiles; ++i) {
+        const int s = i % STAGES, a = i & 1;
+        if (i >= 2 && !mbar_wait(&acc_empty[a], ((i >> 1) + 1) & 1, &abort_flag, p.status)) break;
+        if (!mbar_wait(&full[s], (i / STAGES) & 1, &abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(k_smem + s * kTileBytes);
+        const uint32_t d_tmem = tmem_base + a * N;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          mma_f8f6f4_ss(d_tmem, sdesc_kmajor_sw128(k_addr + kk * 32), sdesc_kmajor_sw128(q_addr + kk * 32),
+                        idesc, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&empty[s]);       // the K stage may be refilled once these MMAs have read it
+        mma_commit(&acc_full[a]);    // accumulator a is ready for the epilogue
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (warps 0-3)
+    const int row_in_tile = warp * 32 + lane;                 // TMEM lane = key within the tile
+    for (int i = 0; i < my_tiles; ++i) {
+      const int a = i & 1;
+      if (!mbar_wait(&acc_full[a], (i >> 1) & 1, &abort_flag, p.status)) break;
+      tc_fence_after();
+      const int key = (kt_begin + i) * kKeysPerTile + row_in_tile;
+      const float ks = key < p.S_max ? p.k_scale[(int64_t)b * p.S_max + key] : 0.f;
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        uint32_t r0[32], r1[32];
+        const uint32_t taddr = tmem_base + ((uint32_t)(warp * 32) << 16) + a * N + q * 64;
+        tmem_ld32(taddr, r0);
+        tmem_ld32(taddr + 32, r1);
+        tmem_ld_wait();
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc = fmaf(wq[q][j], fmaxf(__uint_as_float(r0[j]), 0.f), acc);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc = fmaf(wq[q][32 + j], fmaxf(__uint_as_float(r1[j]), 0.f), acc);
+        const int t = t0 + q;
+        if (t < p.T) {
+          float* dst = p.scores + ((int64_t)b * p.T + t) * p.ld;
+          if (key < nvalid[q]) dst[key] = acc * ks;
+          else if ((p.flags & DSA_FILL_MASKED) && key < p.S_max) dst[key] = -INFINITY;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[a]);
+    }
+    if (p.flags & DSA_FILL_MASKED) {      // tiles of this split above the causal limit
+      const int kt_stop = min((p.S_max + kKeysPerTile - 1) / kKeysPerTile, kt_begin + p.tiles_per_split);
+      for (int kt = max(kt_begin, kt_end); kt < kt_stop; ++kt) {
+        const int key = kt * kKeysPerTile + row_in_tile;
+        if (key >= p.S_max) continue;
+        for (int q = 0; q < NQ; ++q) {
+          const int t = t0 + q;
+          if (t < p.T) p.scores[((int64_t)b * p.T + t) * p.ld + key] = -INFINITY;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kEpiWarps + 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+template <int NQ>
+static int launch_scores_nq(const uint8_t* q8, const uint8_t* k8, const ScoresParams& base,
+                            cudaStream_t stream) {
+  using Cfg = ScoresCfg<NQ>;
+  CUtensorMap qmap, kmap;
+  if (!dsa_host::encode_tensor_map_2d(&qmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, (void*)q8, 128,
+                                      (uint64_t)base.B * base.T * 64, 128, 128, NQ * 64,
+                                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !dsa_host::encode_tensor_map_2d(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, (void*)k8, 128,
+                                      (uint64_t)base.B * base.S_max, 128, 128, kKeysPerTile,
+                                      CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  ScoresParams p = base;
+  p.groups = (base.T + NQ - 1) / NQ;
+  const int tiles_max = (base.S_max + kKeysPerTile - 1) / kKeysPerTile;
+  const int64_t units = (int64_t)base.B * p.groups;
+  const int target = 4 * dsa_host::device_sm_count();
+  int ksplit = (int)((target + units - 1) / units);
+  ksplit = max(1, min(ksplit, tiles_max));
+  p.ksplit = ksplit;
+  p.tiles_per_split = (tiles_max + ksplit - 1) / ksplit;
+  p.ksplit = (tiles_max + p.tiles_per_split - 1) / p.tiles_per_split;
+  const int64_t grid = units * p.ksplit;
+  if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    if (cudaFuncSetAttribute(index_scores_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::kSmemBytes) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    configured[dev] = true;
+  }
+  index_scores_kernel<NQ><<<(unsigned)grid, kThreads, Cfg::kSmemBytes, stream>>>(qmap, kmap, p);
+  return dsa_host::check_launch();
+}
+
+int launch_index_scores(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8,
+                        const float* k_scale, const int32_t* q_pos, const int32_t* kv_len, int B,
+                        int T, int S_max, float softmax_scale, float* scores, int64_t ld,
+                        uint32_t flags, cudaStream_t stream, int* status) {
+  ScoresParams p{};
+  p.q_scale = q_scale; p.w = w; p.k_scale = k_scale; p.q_pos = q_pos; p.kv_len = kv_len;
+  p.scores = scores; p.ld = ld; p.B = B; p.T = T; p.S_max = S_max;
+  p.wscale = 0.125f * softmax_scale;   // 64^-0.5 (n_heads**-0.5 in Indexer.forward)
+  p.flags = flags; p.status = status;
+  if (T >= 4) return launch_scores_nq<4>(q8, k8, p, stream);
+  return launch_scores_nq<1>(q8, k8, p, stream);
+}
+
+}  // namespace dsa

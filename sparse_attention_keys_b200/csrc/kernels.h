@@ -1,0 +1,27 @@
+// Internal launchers behind the C ABI (dsa_abi.cu validates arguments, then calls these).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace dsa {
+
+int launch_index_keys(const float* x, int64_t rows, int heads, const int32_t* pos,
+                      const float* rope_cs, int max_pos, uint32_t flags, uint8_t* out_fp8,
+                      float* out_scale, const int64_t* dst_row, cudaStream_t stream, int* status);
+
+int launch_index_scores(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8,
+                        const float* k_scale, const int32_t* q_pos, const int32_t* kv_len, int B,
+                        int T, int S_max, float softmax_scale, float* scores, int64_t ld,
+                        uint32_t flags, cudaStream_t stream, int* status);
+
+int launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int32_t* kv_len, int B,
+                int T, int k, int32_t* idx, cudaStream_t stream, int* status);
+
+size_t sparse_mla_workspace_size(int B, int T, int k);
+int launch_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T,
+                      int S_max, int k, float softmax_scale, uint16_t* out, float* lse,
+                      void* workspace, size_t ws_bytes, cudaStream_t stream, int* status);
+
+}  // namespace dsa

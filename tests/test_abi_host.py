@@ -1,0 +1,102 @@
+"""Host-side checks of the C-ABI library that need no GPU: every symbol the header declares is
+exported, arguments are rejected before any launch, and the library's own RoPE table agrees with
+the oracle's (the two are written independently)."""
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"DSA_API\s+[\w\s\*]+?\b(dsa_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from sparse_attention_keys_b200 import build
+    build.build()
+    import sparse_attention_keys_b200 as m
+    return m.lib
+
+
+def test_header_declares_the_path():
+    names = _declared()
+    for n in ("dsa_index_keys", "dsa_index_scores", "dsa_topk", "dsa_sparse_mla", "dsa_rope_table",
+              "dsa_get_device_status", "dsa_status_string", "dsa_sparse_mla_workspace_size"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    nm = subprocess.run(["nm", "-D", "--defined-only", L._name], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(dsa_\w+)", nm))
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing
+    for n in _declared():
+        assert hasattr(L, n)
+
+
+def test_status_strings(L):
+    import sparse_attention_keys_b200 as m
+    assert m.dsa_status_string(0) == "DSA_OK"
+    assert m.dsa_status_string(1) == "DSA_ERR_INVALID_ARG"
+    assert m.dsa_status_string(5) == "DSA_ERR_DEVICE_BOUNDS"
+    assert m.dsa_status_string(99) == "DSA_ERR_UNKNOWN"
+    assert m.dsa_version().startswith("dsa-b200")
+
+
+def test_invalid_arguments_rejected_before_launch(L):
+    """These calls fail validation on the host; no device is touched (none exists here)."""
+    p = ctypes.c_void_p(16)          # non-null, aligned dummy; never dereferenced
+    bad = ctypes.c_void_p(17)        # misaligned
+    n = None
+    assert L.dsa_index_keys(p, 4, 0, p, p, 10, 1, p, p, n, n) == 1              # heads < 1
+    assert L.dsa_index_keys(p, 4, 1, p, p, 10, 8, p, p, n, n) == 1              # unknown flag
+    assert L.dsa_index_keys(bad, 4, 1, p, p, 10, 1, p, p, n, n) == 1            # misaligned x
+    assert L.dsa_index_keys(n, 4, 1, p, p, 10, 1, p, p, n, n) == 1              # null x
+    assert L.dsa_index_keys(p, 0, 1, p, p, 10, 1, p, p, n, n) == 0              # empty: nothing to do
+    f = ctypes.c_float
+    args = [p, p, p, p, p, p, p, 1, 1, 128, f(0.088), p, 128, 0, n]
+    a = list(args); a[12] = 126; assert L.dsa_index_scores(*a) == 1          # ld not a multiple of 4
+    a = list(args); a[12] = 64; assert L.dsa_index_scores(*a) == 1           # ld < S_max
+    a = list(args); a[10] = f(0.0); assert L.dsa_index_scores(*a) == 1       # scale <= 0
+    a = list(args); a[13] = 4; assert L.dsa_index_scores(*a) == 1            # unknown flag
+    a = list(args); a[3] = bad; assert L.dsa_index_scores(*a) == 1          # misaligned k8
+    assert L.dsa_topk(p, 130, p, p, 1, 1, 8, p, n) == 1                      # ld % 4
+    assert L.dsa_topk(p, 128, p, p, 1, 1, 0, p, n) == 1                      # k < 1
+    assert L.dsa_topk(p, 128, p, p, 0, 1, 8, p, n) == 1                      # B < 1
+    assert L.dsa_sparse_mla(p, p, p, 1, 1, 16, 0, f(0.1), p, n, n, 0, n) == 1  # k < 1
+    assert L.dsa_sparse_mla(p, p, p, 1, 1, 16, 4, f(-1.0), p, n, n, 0, n) == 1
+    assert L.dsa_sparse_mla(p, bad, p, 1, 1, 16, 4, f(0.1), p, n, n, 0, n) == 1
+    assert L.dsa_rope_table(n, 10) == 1
+    assert L.dsa_rope_table(p, 0) == 1
+
+
+def test_library_rope_table_matches_oracle(L):
+    from oracle import dsa_oracle as O
+    import sparse_attention_keys_b200 as m
+    mine = m.dsa_rope_table(16384).numpy()
+    ref = O.rope_table(16384)
+    assert mine.shape == ref.shape
+    diff = np.abs(mine.view(np.int32).astype(np.int64) - ref.view(np.int32).astype(np.int64))
+    # both round cos/sin of the same fp32 angle from double; libm and numpy may differ by an ulp
+    assert diff.max() <= 1
+    assert (diff > 0).mean() < 1e-3
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    """Importing the binding with no built library raises; there is no fallback path."""
+    pkg = tmp_path / "sparse_attention_keys_b200"
+    pkg.mkdir()
+    src = open(os.path.join(ROOT, "sparse_attention_keys_b200", "__init__.py")).read()
+    (pkg / "__init__.py").write_text(src)
+    r = subprocess.run([sys.executable, "-c", "import sparse_attention_keys_b200"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "libdsa.so not built" in r.stderr
