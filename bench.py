@@ -75,6 +75,23 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+# ------------------------------------------------------------------------------ multi-rank plumbing
+def max_over_ranks(values, world, device=None):
+    """Element-wise max of per-rank timings (every rank gets the result)."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as tdist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def weak_scaling_value(units_per_rank_step, steps, world, t_max_seconds):
+    """Whole-job throughput: every rank processes its own replica, so the units add up."""
+    return units_per_rank_step * steps * world / t_max_seconds
+
+
 # ------------------------------------------------------------------------------ clocks sampling
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -91,7 +108,7 @@ class ClockSampler:
         os.close(fd)
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -270,6 +287,13 @@ def run_ours(args, rank, world, local_rank):
     kev = {}
     steps = []
     with ClockSampler(local_rank) as clk:
+        # the sampler polls every 20 ms: keep the GPU under the same load for ~0.5 s before the
+        # timed steps so that the samples taken while they run see steady-state clocks
+        t_end = time.perf_counter() + 0.5
+        while time.perf_counter() < t_end:
+            st.l2_flush()
+            st.run()
+            torch.cuda.synchronize()
         barrier()
         for _ in range(args.steps):
             st.l2_flush()
@@ -307,17 +331,13 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device status after timing: {dsa.dsa_status_string(status)}")
 
     # ---- max over ranks
-    if world > 1:
-        tt = torch.tensor([t_dev, t_e2e], dtype=torch.float64, device=dev)
-        tdist.all_reduce(tt, op=tdist.ReduceOp.MAX)
-        t_dev, t_e2e = tt.tolist()
+    t_dev, t_e2e = max_over_ranks([t_dev, t_e2e], world, dev)
     if rank != 0:
         return None
 
     peaks = load_peaks()
-    total_pairs = units["pairs"] * args.steps * world
-    value = total_pairs / t_dev
-    tok_s = units["queries"] * args.steps * world / t_dev
+    value = weak_scaling_value(units["pairs"], args.steps, world, t_dev)
+    tok_s = weak_scaling_value(units["queries"], args.steps, world, t_dev)
     # dominant kernel and its roofline
     dom = max(per_kernel, key=per_kernel.get)
     roof = roofline_entry(dom, per_kernel[dom], units, peaks, args)
@@ -342,7 +362,7 @@ def run_ours(args, rank, world, local_rank):
         "mla_decode_tok_s": tok_s if wl.decode else None,
         "kernel_ms": {n: v * 1e3 for n, v in per_kernel.items()},
         "roofline": roof,
-        "e2e": {"value": total_pairs / t_e2e, "unit": UNIT, "h2d_bytes_per_step": st.bytes_h2d(),
+        "e2e": {"value": weak_scaling_value(units["pairs"], args.steps, world, t_e2e), "unit": UNIT, "h2d_bytes_per_step": st.bytes_h2d(),
                 "d2h_bytes_per_step": st.bytes_d2h(), "ms_per_step": t_e2e / args.steps * 1e3},
         "gpu_launches": st.launches_per_step * args.steps,
         "clocks": clocks,
@@ -369,14 +389,18 @@ def roofline_entry(name, seconds, units, peaks, args):
 
 
 def load_traffic(kernel, workload):
-    """DRAM bytes per launch from the committed ncu summary for this kernel and workload, if one
-    exists and matches the current build (else null)."""
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the committed ncu
+    summary for this kernel and workload; null when none exists or the kernel's source changed
+    since the counters were taken."""
+    import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
-    e = d.get(f"{kernel}/{workload}")
+    e = json.load(open(p)).get(f"{kernel}/{workload}")
     if not e:
+        return None
+    src = os.path.join(ROOT, e["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != e["source_sha256_16"]:
         return None
     return e.get("dram_bytes_per_launch")
 
