@@ -167,6 +167,31 @@ DSA_API int dsa_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t*
                    uint16_t* out, float* lse, void* workspace, size_t ws_bytes,
                    dsa_stream_t stream);
 
+/*
+ * dsa_sparse_mla_noalloc - the same computation and arguments as dsa_sparse_mla, minus the
+ * workspace, for callers that cannot allocate device memory themselves (for example code inside
+ * a host framework whose memory manager owns every device allocation, or a serving loop that
+ * must not call cudaMalloc/cudaFree because they can synchronise the device). The pages have no
+ * counterpart to this call; it exists only for such callers.
+ *   - Allocates nothing. The split-KV scratch comes from one fixed device array inside the
+ *     library, dsa_sparse_mla_noalloc_scratch_bytes() = 32 MiB, which every GPU that loads the
+ *     library keeps until the process exits.
+ *   - A shape whose scratch need (dsa_sparse_mla_workspace_size) exceeds that array is rejected
+ *     with DSA_ERR_WORKSPACE before any launch.
+ *   - The first call on each device looks up the array's device address (a one-time set-up with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents (nothing in it needs
+ *     to start at zero: each call overwrites all the scratch it reads). Calls whose work overlaps
+ *     on the GPU (different streams, or different host threads on one device) race on it:
+ *     serialise them.
+ */
+DSA_API int dsa_sparse_mla_noalloc(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
+                                   int B, int T, int S_max, int k, float softmax_scale,
+                                   uint16_t* out, float* lse, dsa_stream_t stream);
+
+/* Size in bytes of the fixed scratch array dsa_sparse_mla_noalloc uses (32 MiB). */
+DSA_API size_t dsa_sparse_mla_noalloc_scratch_bytes(void);
+
 /* Bytes of device scratch dsa_sparse_mla needs for this shape (0 when it needs none). */
 DSA_API size_t dsa_sparse_mla_workspace_size(int B, int T, int k);
 

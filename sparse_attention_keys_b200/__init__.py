@@ -15,7 +15,8 @@ import torch
 __all__ = [
     "DsaError", "lib", "lib_path", "DSA_HADAMARD", "DSA_FILL_MASKED", "INDEXER_SOFTMAX_SCALE",
     "MLA_SOFTMAX_SCALE", "dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk",
-    "dsa_sparse_mla", "dsa_sparse_mla_workspace_size", "dsa_get_device_status", "dsa_status_string",
+    "dsa_sparse_mla", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_noalloc",
+    "dsa_sparse_mla_noalloc_scratch_bytes", "dsa_get_device_status", "dsa_status_string",
     "dsa_device_supported", "dsa_version",
 ]
 
@@ -49,13 +50,16 @@ def _load():
     L.dsa_sparse_mla.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
     L.dsa_sparse_mla_workspace_size.argtypes = [i32, i32, i32]
     L.dsa_sparse_mla_workspace_size.restype = sz
+    L.dsa_sparse_mla_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp]
+    L.dsa_sparse_mla_noalloc_scratch_bytes.argtypes = []
+    L.dsa_sparse_mla_noalloc_scratch_bytes.restype = sz
     L.dsa_get_device_status.argtypes = [vp]
     L.dsa_status_string.argtypes = [i32]
     L.dsa_status_string.restype = ctypes.c_char_p
     L.dsa_device_supported.argtypes = []
     L.dsa_version.restype = ctypes.c_char_p
     for f in ("dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk", "dsa_sparse_mla",
-              "dsa_get_device_status", "dsa_device_supported"):
+              "dsa_sparse_mla_noalloc", "dsa_get_device_status", "dsa_device_supported"):
         getattr(L, f).restype = ctypes.c_int
     return L
 
@@ -201,6 +205,28 @@ def dsa_sparse_mla(q, kv, idx, softmax_scale: float = MLA_SOFTMAX_SCALE, out=Non
                              _ptr(lse), _ptr(workspace), 0 if workspace is None else workspace.numel(),
                              _stream(stream))
     _check(rc, "dsa_sparse_mla")
+    return out, lse
+
+
+def dsa_sparse_mla_noalloc_scratch_bytes() -> int:
+    return int(_lib.dsa_sparse_mla_noalloc_scratch_bytes())
+
+
+def dsa_sparse_mla_noalloc(q, kv, idx, out, lse=None, softmax_scale: float = MLA_SOFTMAX_SCALE, stream=None):
+    """dsa_sparse_mla for callers that cannot allocate device memory: the caller passes the
+    output buffers (out bf16 [B,T,128,512], optional lse fp32 [B,T,128]) and the library takes
+    its scratch from a fixed array of dsa_sparse_mla_noalloc_scratch_bytes(). Nothing is
+    allocated here either. Calls that overlap on the GPU share that array: serialise them."""
+    _need(q, torch.bfloat16, "q")
+    _need(kv, torch.bfloat16, "kv")
+    _need(idx, torch.int32, "idx")
+    _need(out, torch.bfloat16, "out")
+    if lse is not None:
+        _need(lse, torch.float32, "lse")
+    B, T = q.shape[0], q.shape[1]
+    rc = _lib.dsa_sparse_mla_noalloc(_ptr(q), _ptr(kv), _ptr(idx), B, T, kv.shape[1], int(idx.shape[-1]),
+                                     float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream))
+    _check(rc, "dsa_sparse_mla_noalloc")
     return out, lse
 
 

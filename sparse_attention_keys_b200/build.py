@@ -1,6 +1,8 @@
 """Build libdsa.so (the C-ABI CUDA library) in-tree for sm_100a with nvcc.
 
-    python -m sparse_attention_keys_b200.build [--force] [--verbose]
+    python sparse_attention_keys_b200/build.py [--force] [--verbose]
+
+(Run it as a script: importing the package loads the library being built.)
 
 The library lands next to this file so that it travels with the source tree.
 """
@@ -19,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libdsa.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["dsa_abi.cu", "index_keys.cu", "index_scores.cu", "topk.cu", "sparse_mla.cu"]
+SOURCES = ["dsa_abi.cu", "index_keys.cu", "index_scores.cu", "topk.cu", "sparse_mla.cu", "sparse_mla_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
               "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

@@ -21,8 +21,8 @@ def _declared():
 
 @pytest.fixture(scope="module")
 def L():
-    from sparse_attention_keys_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__._build_module().build()
     import sparse_attention_keys_b200 as m
     return m.lib
 
