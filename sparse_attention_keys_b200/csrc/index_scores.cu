@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row_in_tile = warp * 32 + lane;                 // TMEM lane = key within the tile
     for (int i = 0; i < my_tiles; ++i) {
       const int a = i & 1;
-      if (!mbar_wait(&acc_full[a], (i >> 1) & 1, &abort_flag, p.status)) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[a], (i >> 1) & 1, &abort_flag, p.status))) break;
       tc_fence_after();
       const int key = (kt_begin + i) * kKeysPerTile + row_in_tile;
       const float ks = key < p.S_max ? p.k_scale[(int64_t)b * p.S_max + key] : 0.f;

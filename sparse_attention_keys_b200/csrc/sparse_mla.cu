@@ -7,13 +7,29 @@
 // gather of the selected rows, and the sparse-attention steps of the dense-block page
 // (S' = S m^2/sqrt 192, A = softmax, O = AV).
 //
-// CTA = (query, key split, half of the 128 heads): eight warps; warps 0-3 own 16 heads each and
-// output features 0..255, warps 4-7 the same heads and features 256..511. Selected latent rows
-// are gathered with 16-byte cp.async into a 3-stage shared-memory ring (32 rows per stage), the
-// scores and P.V run on bf16 tensor-core tiles (m16n8k16) with an fp32 online softmax in
-// registers. With several key splits per query, fp32 partials (O, running max, running sum) go to
-// the caller's workspace and a second kernel merges them.
+// Tensor cores (tcgen05, kind::f16, bf16 in / fp32 accumulate in TMEM). A 128-head x 512 fp32
+// output accumulator alone would fill all 512 TMEM columns, so each (query, key split) runs on two
+// CTAs that split the OUTPUT features: CTA c accumulates out[:, 256c:256c+256) (256 TMEM columns).
+// Each CTA computes the full 576-feature score itself (Q for all 128 heads resident on chip: features
+// 0..319 in TMEM as bf16 pairs, 320..575 in shared memory via TMA), so the pair never exchanges data: this costs 1.5x the Q K^T work
+// of a single pass, but exchanging 128 x 64 fp32 partial scores per tile between CTAs runs into
+// the limited bandwidth of distributed shared memory.
+//
+// Selected 1152-byte latent rows are gathered by four warps with 16-byte cp.async, one warp-wide
+// coalesced 512-byte request per instruction, written straight into the 128B-swizzled operand
+// layout (unselected slots are zero-filled) into a double-buffered ring of 64-key tiles. (Measured
+// on B200 with one CTA per SM: this moves ~2.5x more bytes per SM than TMA tile::gather4 with
+// 128-byte boxes.) One shared-memory tile is both the
+// K-major B operand of Q K^T (N = keys) and the MN-major B operand of P V (N = features).
+// TMEM: O [0,256), S [256,320), P as bf16 pairs [320,352) (the A operand of P V straight from
+// TMEM), Q features 0..319 as bf16 pairs [352,512) (the A operand of the first
+// 20 K-steps of Q K^T; the last 16 K-steps read Q from shared memory).
+// Per CTA: 4 softmax warps (thread = head = TMEM lane), 1 MMA-issuing thread that issues Q K^T and
+// P V in whichever order their inputs become ready, 4 gather warps (the first also loads Q by TMA). The running max is only moved
+// (and O rescaled in TMEM) when it grows by more than 2^8. With several key splits per query, fp32
+// partials (O, max, sum) go to the caller's workspace and a second kernel merges them.
 #include <cuda_bf16.h>
+#include <math.h>
 
 #include <algorithm>
 
@@ -27,55 +43,58 @@ namespace {
 constexpr int kHeads = 128;
 constexpr int kDqk = 576;
 constexpr int kDv = 512;
-constexpr int kHeadsPerCta = 64;
-constexpr int kKeysPerStage = 32;
-constexpr int kStages = 3;
-constexpr int kRowBytes = kDqk * 2 + 16;                  // padded: conflict-free ldmatrix
-constexpr int kQBytes = kHeadsPerCta * kRowBytes;
-constexpr int kStageBytes = kKeysPerStage * kRowBytes;
-constexpr int kMlaThreads = 256;
-constexpr int kSmemBytes = kQBytes + kStages * kStageBytes + kStages * kKeysPerStage * 4;
+constexpr int kKeys = 64;                          // selected keys per tile (N of Q K^T)
+constexpr int kRegions = 9;                        // 576 features = 9 blocks of 64 (128 B), 128B swizzle
+constexpr int kQTmemRegions = 5;                   // features 0..319 live in TMEM
+constexpr int kQRegion = kHeads * 128;             // 16 KB
+constexpr int kQBytes = (kRegions - kQTmemRegions) * kQRegion;   // 64 KB: features 320..575
+constexpr int kKvRegion = kKeys * 128;             // 8 KB
+constexpr int kStageBytes = kRegions * kKvRegion;  // 72 KB
+constexpr int kStages = 2;
+constexpr int kOffQ = 0;
+constexpr int kOffKV = kOffQ + kQBytes;
+constexpr int kOffBar = kOffKV + kStages * kStageBytes;
+constexpr int kSmemBytes = 1024 + kOffBar + 256;
+constexpr int kSoftmaxWarps = 4, kMmaWarp = 4, kGatherWarp = 5, kGatherWarps = 4;
+constexpr int kMlaThreads = (kSoftmaxWarps + 1 + kGatherWarps) * 32;
+constexpr int kMaxSlots = 2048;                    // selected slots per CTA (split chunk cap)
+constexpr int kTmemCols = 512;
+constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 320, kTmemQ = 352;   // 64 + 32 + 160 columns
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;          // log2 units
 
 struct MlaSplit {
   int nsplit;
-  int chunk;     // selected slots per split (multiple of kKeysPerStage)
+  int chunk;     // selected slots per split (multiple of kKeys, at most kMaxSlots)
 };
 
 MlaSplit choose_split(int64_t BT, int k, int sms) {
   MlaSplit s;
-  const int64_t ctas_per_split = BT * (kHeads / kHeadsPerCta);
+  const int64_t ctas_per_split = BT * 2;
   int n = (int)std::max<int64_t>(1, (sms + ctas_per_split - 1) / ctas_per_split);
   const int max_split = std::max(1, (k + 63) / 64);
   n = std::min(n, max_split);
   int chunk = (k + n - 1) / n;
-  chunk = (chunk + kKeysPerStage - 1) / kKeysPerStage * kKeysPerStage;
+  chunk = (chunk + 63) / 64 * 64;
+  chunk = std::min(chunk, kMaxSlots);
   s.chunk = chunk;
   s.nsplit = (k + chunk - 1) / chunk;
   return s;
 }
 
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                               uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// byte offset of 16-byte chunk `c` of row `r` in a 128B-swizzled tile of 128-byte rows
+__device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+// 2^x with the MUFU approximation (relative error ~2^-22; softmax weights only need bf16 accuracy)
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 }  // namespace
@@ -84,7 +103,7 @@ struct MlaParams {
   const uint16_t* q;
   const uint16_t* kv;
   const int32_t* idx;
-  int T, S_max, k;
+  int B, T, S_max, k;
   int nsplit, chunk;
   float scale_log2;          // softmax_scale * log2(e)
   uint16_t* out;
@@ -94,191 +113,298 @@ struct MlaParams {
   int* status;
 };
 
-__global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(const MlaParams p) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t* q_sm = smem;
-  uint8_t* kv_sm = smem + kQBytes;
-  int32_t* slot_idx = reinterpret_cast<int32_t*>(smem + kQBytes + kStages * kStageBytes);  // [stage][32]
+__global__ void __launch_bounds__(kMlaThreads, 1)
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap kv_map,
+                      const MlaParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_sm = smem + kOffQ;
+  uint8_t* kv_sm = smem + kOffKV;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* kv_full = bars;                    // [kStages] gather (cp.async) -> MMA
+  uint64_t* kv_empty = bars + kStages;         // [kStages] MMA (after P V) -> gather
+  uint64_t* s_full = bars + 2 * kStages;       // MMA -> softmax
+  uint64_t* s_empty = s_full + 1;              // softmax (S read) -> MMA
+  uint64_t* q_full = s_full + 2;               // TMA (Q in smem) + softmax (Q in TMEM) -> MMA
+  uint64_t* p_full = s_full + 3;               // softmax (P in TMEM) -> MMA
+  uint64_t* p_empty = s_full + 4;              // MMA (P V done) -> softmax
+  uint64_t* o_full = s_full + 5;               // MMA -> softmax (all P V done)
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int hh = blockIdx.x & 1;                      // head half
-  const int split = (blockIdx.x >> 1) % p.nsplit;
-  const int64_t bt = (blockIdx.x >> 1) / p.nsplit;
+  const int half = blockIdx.x & 1;             // output features [256*half, 256*half + 256)
+  const int unit = blockIdx.x >> 1;
+  const int split = unit % p.nsplit;
+  const int64_t bt = unit / p.nsplit;
   const int b = (int)(bt / p.T);
   const int slot0 = split * p.chunk;
   const int nslots = max(0, min(p.k, slot0 + p.chunk) - slot0);
-  const int nstages_total = (nslots + kKeysPerStage - 1) / kKeysPerStage;
+  const int ntiles = (nslots + kKeys - 1) / kKeys;
   const int32_t* idx_row = p.idx + bt * p.k + slot0;
-  const uint16_t* kv_b = p.kv + (int64_t)b * p.S_max * kDqk;
 
-  // Q: 64 heads x 576 bf16 into padded rows (72 chunks of 16 B per row)
-  {
-    const uint16_t* qsrc = p.q + (bt * kHeads + hh * kHeadsPerCta) * kDqk;
-    for (int c = tid; c < kHeadsPerCta * 72; c += kMlaThreads) {
-      const int r = c / 72, ch = c - r * 72;
-      cp_async_16(smem_u32(q_sm + r * kRowBytes + ch * 16), qsrc + r * kDqk + ch * 8);
+  if (tid == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&kv_full[s], kGatherWarps * 32);
+      mbar_init(&kv_empty[s], 1);
     }
+    mbar_init(s_full, 1);
+    mbar_init(s_empty, kSoftmaxWarps * 32);
+    mbar_init(q_full, 1 + kSoftmaxWarps * 32);
+    mbar_init(p_full, kSoftmaxWarps * 32);
+    mbar_init(p_empty, 1);
+    mbar_init(o_full, 1);
+    fence_barrier_init();
   }
-  auto load_stage = [&](int st, int buf) {
-    const int base = st * kKeysPerStage;
-    if (tid < kKeysPerStage) {
-      int v = -1;
-      if (base + tid < nslots) {
-        v = idx_row[base + tid];
-        if (v >= p.S_max) { set_status(p.status, DSA_ERR_DEVICE_BOUNDS); v = -1; }
-        if (v < -1) v = -1;
-      }
-      slot_idx[buf * kKeysPerStage + tid] = v;
-    }
-    // each of the 32 rows is 72 chunks; rows with idx -1 are zero-filled
-    uint8_t* dst = kv_sm + buf * kStageBytes;
-    for (int c = tid; c < kKeysPerStage * 72; c += kMlaThreads) {
-      const int r = c / 72, ch = c - r * 72;
-      const int slot = base + r;
-      int v = slot < nslots ? idx_row[slot] : -1;
-      const bool ok = v >= 0 && v < p.S_max;
-      cp_async_16_zfill(smem_u32(dst + r * kRowBytes + ch * 16), kv_b + (int64_t)(ok ? v : 0) * kDqk + ch * 8, ok);
-    }
-  };
-
-  for (int s = 0; s < kStages - 1; ++s) {
-    if (s < nstages_total) load_stage(s, s);
-    cp_async_commit();
+  if (warp == kMmaWarp) {
+    tmem_alloc(&tmem_base_sh, kTmemCols);
+    tmem_relinquish();
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
 
-  const int wq = warp & 3;            // head group of 16 within the CTA's 64
-  const int vhalf = warp >> 2;        // output features [vhalf*256, +256)
-  float o[32][4];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-  float m_r[2] = {-INFINITY, -INFINITY};   // rows lane/4 and lane/4+8, log2 domain
-  float l_r[2] = {0.f, 0.f};
-
-  const uint32_t q_base = smem_u32(q_sm) + (wq * 16) * kRowBytes;
-  // ldmatrix lane addressing
-  const int a_row = (lane & 7) + ((lane >> 3) & 1) * 8, a_col = (lane >> 4) * 8;
-  const int b_key = (lane & 7) + (lane >> 4) * 8, b_col = ((lane >> 3) & 1) * 8;
-  const int v_key = (lane & 7) + ((lane >> 3) & 1) * 8, v_col = (lane >> 4) * 8;
-
-  for (int st = 0; st < nstages_total; ++st) {
-    const int buf = st % kStages;
-    if (st + kStages - 1 < nstages_total) load_stage(st + kStages - 1, (st + kStages - 1) % kStages);
-    cp_async_commit();
-    cp_async_wait<kStages - 1>();
-    __syncthreads();
-
-    const uint32_t kv_base = smem_u32(kv_sm + buf * kStageBytes);
-    // S = Q K^T: 16 heads x 32 keys
-    float s[4][4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+  if (warp >= kGatherWarp) {
+    // ------------------------------------------------------------------ gather warps
+    // gather warp w copies keys 16w..16w+15 of each tile; per key, lanes take 16-byte chunks
+    // lane, lane+32, lane+64 of the 72 in the row (contiguous 512-byte warp requests)
+    const int w = warp - kGatherWarp;
+    if (w == 0 && lane == 0 && ntiles > 0) {
+      prefetch_tensormap(&q_map);
+      mbar_arrive_expect_tx(q_full, kQBytes);
+      for (int r = kQTmemRegions; r < kRegions; ++r)
+        tma_load_2d(q_sm + (r - kQTmemRegions) * kQRegion, &q_map, q_full, 64 * r, (int32_t)(bt * kHeads));
+    }
+    const uint16_t* kv_b = p.kv + (int64_t)b * p.S_max * kDqk;
+    auto load_idx = [&](int j) -> int {
+      const int slot = j * kKeys + 16 * w + (lane & 15);
+      return (j < ntiles && slot < nslots) ? __ldg(idx_row + slot) : -1;
+    };
+    int idx_next = load_idx(0);
+    for (int j = 0; j < ntiles; ++j) {
+      const int s = j % kStages;
+      const int idx_cur = idx_next;
+      idx_next = load_idx(j + 1);                     // one tile ahead
+      if (lane < 16 && idx_cur >= p.S_max) set_status(p.status, DSA_ERR_DEVICE_BOUNDS);
+      if (j >= kStages &&
+          !__all_sync(0xffffffffu, mbar_wait(&kv_empty[s], ((j / kStages) + 1) & 1, &abort_flag, p.status)))
+        break;
+      const uint32_t base = smem_u32(kv_sm + s * kStageBytes);
 #pragma unroll 4
-    for (int kk = 0; kk < kDqk / 16; ++kk) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4(q_base + a_row * kRowBytes + (kk * 16 + a_col) * 2, a0, a1, a2, a3);
+      for (int kk = 0; kk < 16; ++kk) {
+        const int v = __shfl_sync(0xffffffffu, idx_cur, kk);
+        const bool ok = v >= 0 && v < p.S_max;
+        const int key = 16 * w + kk;
+        const uint16_t* src = kv_b + (int64_t)(ok ? v : 0) * kDqk;
 #pragma unroll
-      for (int jp = 0; jp < 2; ++jp) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(kv_base + (jp * 16 + b_key) * kRowBytes + (kk * 16 + b_col) * 2, b0, b1, b2, b3);
-        mma_bf16_16816(s[2 * jp], a0, a1, a2, a3, b0, b1);
-        mma_bf16_16816(s[2 * jp + 1], a0, a1, a2, a3, b2, b3);
+        for (int i = 0; i < 3; ++i) {
+          const int c = lane + 32 * i;
+          if (c < 72)
+            cp_async_16_zfill(base + (c >> 3) * kKvRegion + sw128(key, c & 7), src + c * 8, ok);
+        }
       }
+      cp_async_mbar_arrive(&kv_full[s]);
     }
-    // mask, online softmax (base 2)
-    const int32_t* sidx = slot_idx + buf * kKeysPerStage;
-    float mx[2] = {-INFINITY, -INFINITY};
+    cp_async_wait_all();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && ntiles > 0) {
+      constexpr uint32_t idesc_s = idesc_f32acc(1 /*BF16*/, 1, 128, kKeys, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_f32acc(1, 1, 128, 256, 0, 1 /*B MN-major*/);
+      const uint32_t q_base = smem_u32(q_sm);
+      bool ok = mbar_wait(q_full, 0, &abort_flag, p.status);
+      int ns = 0, npv = 0;           // tiles whose Q K^T / P V have been issued
+      uint32_t idle = 0;
+      while (ok && npv < ntiles) {
+        bool progress = false;
+        // Q K^T of tile ns: its keys landed and its score buffer has been read by the softmax
+        if (ns < ntiles && mbar_test_wait(&kv_full[ns % kStages], (ns / kStages) & 1) &&
+            (ns == 0 || mbar_test_wait(s_empty, (ns - 1) & 1))) {
+          fence_proxy_async_smem();      // cp.async (generic proxy) writes -> MMA (async proxy) reads
+          tc_fence_after();
+          const uint32_t kv_base = smem_u32(kv_sm + (ns % kStages) * kStageBytes);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+          for (int ks = 0; ks < 4 * kQTmemRegions; ++ks)          // Q from TMEM
+            mma_f16_ts(tmem + kTmemS, tmem + kTmemQ + ks * 8,
+                       sdesc_kmajor_sw128(kv_base + (ks >> 2) * kKvRegion + (ks & 3) * 32), idesc_s,
+                       ks > 0 ? 1u : 0u);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = j * 8 + (lane & 3) * 2 + (e & 1);
-        const float z = sidx[key] >= 0 ? s[j][e] * p.scale_log2 : -INFINITY;
-        s[j][e] = z;
-        mx[e >> 1] = fmaxf(mx[e >> 1], z);
+          for (int ks = 4 * kQTmemRegions; ks < kDqk / 16; ++ks)  // Q from shared memory
+            mma_f16_ss(tmem + kTmemS,
+                       sdesc_kmajor_sw128(q_base + ((ks >> 2) - kQTmemRegions) * kQRegion + (ks & 3) * 32),
+                       sdesc_kmajor_sw128(kv_base + (ks >> 2) * kKvRegion + (ks & 3) * 32), idesc_s, 1u);
+          mma_commit(s_full);
+          ++ns;
+          progress = true;
+        }
+        // P V of tile npv: its probabilities are in TMEM
+        if (npv < ns && mbar_test_wait(p_full, npv & 1)) {
+          tc_fence_after();
+          const uint32_t v_base = smem_u32(kv_sm + (npv % kStages) * kStageBytes) + 4 * half * kKvRegion;
+#pragma unroll
+          for (int kk = 0; kk < kKeys / 16; ++kk)
+            mma_f16_ts(tmem + kTmemO, tmem + kTmemP + kk * 8,
+                       sdesc_mnmajor_sw128(v_base + kk * 2048, kKvRegion, 1024), idesc_pv,
+                       (npv > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(p_empty);
+          mma_commit(&kv_empty[npv % kStages]);
+          ++npv;
+          progress = true;
+        }
+        if (progress) {
+          idle = 0;
+        } else if (++idle > kSpinLimit || abort_flag) {
+          if (!abort_flag) set_status(p.status, DSA_ERR_TIMEOUT);
+          abort_flag = 1;
+          ok = false;
+        }
       }
-    }
-    float alpha[2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-      const float m_new = fmaxf(m_r[r], mx[r]);
-      alpha[r] = (m_new == -INFINITY) ? 1.f : exp2f(m_r[r] - m_new);
-      m_r[r] = m_new;
-    }
-    float rs[2] = {0.f, 0.f};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float m = m_r[e >> 1];
-        const float pv = (m == -INFINITY) ? 0.f : exp2f(s[j][e] - m);
-        s[j][e] = pv;
-        rs[e >> 1] += pv;
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) l_r[r] = l_r[r] * alpha[r] + rs[r];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      o[j][0] *= alpha[0]; o[j][1] *= alpha[0];
-      o[j][2] *= alpha[1]; o[j][3] *= alpha[1];
-    }
-    // O += P V over this stage's 32 keys (two k16 steps)
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      const uint32_t a0 = pack_bf16(s[2 * ks][0], s[2 * ks][1]);
-      const uint32_t a1 = pack_bf16(s[2 * ks][2], s[2 * ks][3]);
-      const uint32_t a2 = pack_bf16(s[2 * ks + 1][0], s[2 * ks + 1][1]);
-      const uint32_t a3 = pack_bf16(s[2 * ks + 1][2], s[2 * ks + 1][3]);
-#pragma unroll
-      for (int jp = 0; jp < 16; ++jp) {
-        uint32_t b0, b1, b2, b3;
-        const int col = vhalf * 256 + jp * 16 + v_col;
-        ldsm_x4_t(kv_base + (ks * 16 + v_key) * kRowBytes + col * 2, b0, b1, b2, b3);
-        mma_bf16_16816(o[2 * jp], a0, a1, a2, a3, b0, b1);
-        mma_bf16_16816(o[2 * jp + 1], a0, a1, a2, a3, b2, b3);
-      }
-    }
-    __syncthreads();     // this buffer is refilled by the next iteration's prefetch
-  }
-  cp_async_wait<0>();
-
-  // finish: full row sums across the quad
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    l_r[r] += __shfl_xor_sync(0xffffffffu, l_r[r], 1);
-    l_r[r] += __shfl_xor_sync(0xffffffffu, l_r[r], 2);
-  }
-  const int head0 = hh * kHeadsPerCta + wq * 16 + (lane >> 2);
-  if (p.nsplit == 1) {
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int head = head0 + r * 8;
-      const float inv = l_r[r] > 0.f ? 1.f / l_r[r] : 0.f;
-      uint16_t* dst = p.out + (bt * kHeads + head) * kDv + vhalf * 256;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int col = j * 8 + (lane & 3) * 2;
-        *reinterpret_cast<uint32_t*>(dst + col) = pack_bf16(o[j][2 * r] * inv, o[j][2 * r + 1] * inv);
-      }
-      if (p.lse && vhalf == 0 && (lane & 3) == 0)
-        p.lse[bt * kHeads + head] = l_r[r] > 0.f ? (m_r[r] + log2f(l_r[r])) * 0.6931471805599453f : -INFINITY;
+      mma_commit(o_full);
     }
   } else {
+    // ------------------------------------------------------------------ softmax warps (thread = head)
+    const int h = tid;
+    const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
+    // Q features 0..319 of head h -> TMEM as bf16 pairs (feature f in column f/2)
+    if (ntiles > 0) {
+      const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (bt * kHeads + h) * kDqk);
+      uint32_t buf[160];
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int head = head0 + r * 8;
-      const int64_t prow = (bt * p.nsplit + split) * kHeads + head;
-      float* dst = p.part_o + prow * kDv + vhalf * 256;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int col = j * 8 + (lane & 3) * 2;
-        *reinterpret_cast<float2*>(dst + col) = make_float2(o[j][2 * r], o[j][2 * r + 1]);
+      for (int i = 0; i < 40; ++i) {
+        const uint4 v = __ldg(qrow + i);
+        buf[4 * i] = v.x; buf[4 * i + 1] = v.y; buf[4 * i + 2] = v.z; buf[4 * i + 3] = v.w;
       }
-      if (vhalf == 0 && (lane & 3) == 0)
-        *reinterpret_cast<float2*>(p.part_ml + prow * 2) = make_float2(m_r[r], l_r[r]);
+#pragma unroll
+      for (int c = 0; c < 5; ++c) tmem_st32(t_row + kTmemQ + c * 32, *reinterpret_cast<uint32_t(*)[32]>(buf + 32 * c));
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(q_full);
     }
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+#pragma unroll 1
+    for (int j = 0; ok && j < ntiles; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full, j & 1, &abort_flag, p.status))) { ok = false; break; }
+      tc_fence_after();
+      uint32_t r0[32], r1[32];
+      tmem_ld32(t_row + kTmemS, r0);
+      tmem_ld32(t_row + kTmemS + 32, r1);
+      const int sa = j * kKeys + lane, sb = sa + 32;
+      const int va = sa < nslots ? __ldg(idx_row + sa) : -1;
+      const int vb = sb < nslots ? __ldg(idx_row + sb) : -1;
+      const uint32_t vlo = __ballot_sync(0xffffffffu, va >= 0 && va < p.S_max);
+      const uint32_t vhi = __ballot_sync(0xffffffffu, vb >= 0 && vb < p.S_max);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(s_empty);
+      float z[kKeys];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        z[i] = ((vlo >> i) & 1u) ? __uint_as_float(r0[i]) * p.scale_log2 : -INFINITY;
+        z[32 + i] = ((vhi >> i) & 1u) ? __uint_as_float(r1[i]) * p.scale_log2 : -INFINITY;
+      }
+      float t8[8];
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        t8[g] = fmaxf(fmaxf(fmaxf(z[8 * g], z[8 * g + 1]), fmaxf(z[8 * g + 2], z[8 * g + 3])),
+                      fmaxf(fmaxf(z[8 * g + 4], z[8 * g + 5]), fmaxf(z[8 * g + 6], z[8 * g + 7])));
+      const float mx = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])), fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
+      float m_new = m, alpha = 1.f;
+      if (mx > m + kRescaleThreshold) {
+        m_new = mx;
+        alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - m_new);
+      }
+      uint32_t pk[kKeys / 2];
+      float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < kKeys; i += 2) {
+        const float e0 = (m_new == -INFINITY) ? 0.f : fast_exp2(z[i] - m_new);
+        const float e1 = (m_new == -INFINITY) ? 0.f : fast_exp2(z[i + 1] - m_new);
+        rs8[(i >> 1) & 7] += e0 + e1;
+        pk[i / 2] = pack_bf16(e0, e1);
+      }
+      l = l * alpha + (((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7])));
+      // P V of the previous tile must be done: P's columns are reused and O may be rescaled
+      if (j >= 1) {
+        if (!__all_sync(0xffffffffu, mbar_wait(p_empty, (j - 1) & 1, &abort_flag, p.status))) { ok = false; break; }
+        tc_fence_after();
+        const bool rescale = (m != -INFINITY) && (m_new != m);
+        if (__any_sync(0xffffffffu, rescale)) {
+          const float a = rescale ? alpha : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_row + kTmemO + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * a);
+            tmem_st32(t_row + kTmemO + c * 32, o);
+          }
+        }
+      }
+      m = m_new;
+      tmem_st32(t_row + kTmemP, pk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    // ---- epilogue: O row (this CTA's 256 output features) / l
+    const bool have_o = ntiles > 0 && ok &&
+                        __all_sync(0xffffffffu, mbar_wait(o_full, 0, &abort_flag, p.status));
+    if (have_o) tc_fence_after();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    if (p.nsplit == 1) {
+      uint16_t* dst = p.out + (bt * kHeads + h) * kDv + 256 * half;
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t o[32];
+        if (have_o) {
+          tmem_ld32(t_row + kTmemO + c * 32, o);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          d4[i] = make_uint4(pack_bf16(__uint_as_float(o[8 * i]) * inv, __uint_as_float(o[8 * i + 1]) * inv),
+                             pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv),
+                             pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv),
+                             pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv));
+      }
+      if (p.lse && half == 0)
+        p.lse[bt * kHeads + h] = l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+    } else {
+      const int64_t prow = (bt * p.nsplit + split) * kHeads + h;
+      float* dst = p.part_o + prow * kDv + 256 * half;
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t o[32];
+        if (have_o) {
+          tmem_ld32(t_row + kTmemO + c * 32, o);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          d4[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                              __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+      }
+      if (half == 0) *reinterpret_cast<float2*>(p.part_ml + prow * 2) = make_float2(m, l);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -337,7 +463,7 @@ int launch_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
   if (BT == 0) return DSA_OK;
   const MlaSplit s = choose_split(BT, k, dsa_host::device_sm_count());
   MlaParams p{};
-  p.q = q; p.kv = kv; p.idx = idx; p.T = T; p.S_max = S_max; p.k = k;
+  p.q = q; p.kv = kv; p.idx = idx; p.B = B; p.T = T; p.S_max = S_max; p.k = k;
   p.nsplit = s.nsplit; p.chunk = s.chunk;
   p.scale_log2 = softmax_scale * kLog2e;
   p.out = out; p.lse = lse; p.status = status;
@@ -356,9 +482,15 @@ int launch_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
       return DSA_ERR_CUDA;
     configured[dev] = true;
   }
-  const int64_t grid = BT * s.nsplit * (kHeads / kHeadsPerCta);
+  const int64_t grid = BT * s.nsplit * 2;          // two CTAs (output-feature halves) per (query, split)
   if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;
-  sparse_mla_kernel<<<(unsigned)grid, kMlaThreads, kSmemBytes, stream>>>(p);
+  CUtensorMap q_map, kv_map;
+  if (!dsa_host::encode_tensor_map_2d(&q_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (void*)q, kDqk,
+                                      (uint64_t)BT * kHeads, kDqk * 2, 64, kHeads, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !dsa_host::encode_tensor_map_2d(&kv_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (void*)kv, kDqk,
+                                      (uint64_t)B * S_max, kDqk * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  sparse_mla_kernel<<<(unsigned)grid, kMlaThreads, kSmemBytes, stream>>>(q_map, kv_map, p);
   int rc = dsa_host::check_launch();
   if (rc != DSA_OK || s.nsplit == 1) return rc;
   const int64_t rows = BT * kHeads;
