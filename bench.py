@@ -236,8 +236,9 @@ class Step:
             if ev is None:
                 fn()
                 return
-            s = self.torch.cuda.Event(enable_timing=True)
-            e = self.torch.cuda.Event(enable_timing=True)
+            # external: inside a graph capture the records become event nodes of the graph
+            s = self.torch.cuda.Event(enable_timing=True, external=True)
+            e = self.torch.cuda.Event(enable_timing=True, external=True)
             s.record()
             fn()
             e.record()
@@ -283,8 +284,19 @@ def run_ours(args, rank, world, local_rank):
             tdist.barrier()
         torch.cuda.synchronize()
 
-    # ---- device-timed region (inputs resident in HBM)
+    # ---- device-timed region (inputs resident in HBM): the step is captured once as a CUDA graph
+    # (with an event node around each ABI call) and replayed, so no host launch gaps are timed
     kev = {}
+    graph = torch.cuda.CUDAGraph()
+    cap_stream = torch.cuda.Stream()
+    cap_stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap_stream):
+        st.run()                                  # warm the capture stream
+    torch.cuda.current_stream().wait_stream(cap_stream)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph, stream=cap_stream):
+        st.run(kev)
+    torch.cuda.synchronize()
     steps = []
     with ClockSampler(local_rank) as clk:
         # the sampler polls every 20 ms: keep the GPU under the same load for ~0.5 s before the
@@ -292,21 +304,26 @@ def run_ours(args, rank, world, local_rank):
         t_end = time.perf_counter() + 0.5
         while time.perf_counter() < t_end:
             st.l2_flush()
-            st.run()
+            graph.replay()
             torch.cuda.synchronize()
         barrier()
+        per_kernel_sum = {n: 0.0 for n in kev}
         for _ in range(args.steps):
             st.l2_flush()
             s = torch.cuda.Event(enable_timing=True)
             e = torch.cuda.Event(enable_timing=True)
             s.record()
-            st.run(kev)
+            graph.replay()
             e.record()
             steps.append((s, e))
+            torch.cuda.synchronize()               # read this replay's kernel events before the next
+            for n, v in kev.items():
+                per_kernel_sum[n] += sum(a.elapsed_time(b) for a, b in v)
         barrier()
     clocks = clk.summary()
     t_dev = sum(s.elapsed_time(e) for s, e in steps) / 1e3          # seconds
-    per_kernel = {n: sum(a.elapsed_time(b) for a, b in v) / len(v) / 1e3 for n, v in kev.items()}
+    per_kernel = {n: v / args.steps / 1e3 for n, v in per_kernel_sum.items()}
+    del graph
 
     # ---- end to end through host buffers (pinned H2D of the step inputs, D2H of the results)
     for _ in range(max(1, args.warmup)):
@@ -365,6 +382,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": weak_scaling_value(units["pairs"], args.steps, world, t_e2e), "unit": UNIT, "h2d_bytes_per_step": st.bytes_h2d(),
                 "d2h_bytes_per_step": st.bytes_d2h(), "ms_per_step": t_e2e / args.steps * 1e3},
         "gpu_launches": st.launches_per_step * args.steps,
+        "timing": "device: CUDA-graph replay of the step, CUDA events around each replay; e2e: plain API calls",
         "clocks": clocks,
     }
     if not args.no_cpu_baseline and world == 1:

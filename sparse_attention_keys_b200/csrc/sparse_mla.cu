@@ -11,7 +11,7 @@
 // output accumulator alone would fill all 512 TMEM columns, so each (query, key split) runs on two
 // CTAs that split the OUTPUT features: CTA c accumulates out[:, 256c:256c+256) (256 TMEM columns).
 // Each CTA computes the full 576-feature score itself (Q for all 128 heads resident on chip: features
-// 0..319 in TMEM as bf16 pairs, 320..575 in shared memory via TMA), so the pair never exchanges data: this costs 1.5x the Q K^T work
+// 0..255 in TMEM as bf16 pairs, 256..575 in shared memory via TMA), so the pair never exchanges data: this costs 1.5x the Q K^T work
 // of a single pass, but exchanging 128 x 64 fp32 partial scores per tile between CTAs runs into
 // the limited bandwidth of distributed shared memory.
 //
@@ -21,9 +21,12 @@
 // on B200 with one CTA per SM: this moves ~2.5x more bytes per SM than TMA tile::gather4 with
 // 128-byte boxes.) One shared-memory tile is both the
 // K-major B operand of Q K^T (N = keys) and the MN-major B operand of P V (N = features).
-// TMEM: O [0,256), S [256,320), P as bf16 pairs [320,352) (the A operand of P V straight from
-// TMEM), Q features 0..319 as bf16 pairs [352,512) (the A operand of the first
-// 20 K-steps of Q K^T; the last 16 K-steps read Q from shared memory).
+// TMEM: O [0,256), two score buffers S0 [256,320) and S1 [320,384), Q features 0..255 as bf16
+// pairs [384,512) (the A operand of the first 16 K-steps of Q K^T; the last 20 read Q from shared
+// memory). The probabilities of tile j overwrite the first 32 columns of the score buffer they came
+// from (bf16 pairs, the A operand of P V), so the MMA thread can run a fixed order
+// S0, S1, PV0, S2, PV1, S3, ...: Q K^T of tile j+2 is issued after P V of tile j, which the tensor
+// pipe executes in order, and it never waits for the softmax to free a buffer.
 // Per CTA: 4 softmax warps (thread = head = TMEM lane), 1 MMA-issuing thread that issues Q K^T and
 // P V in whichever order their inputs become ready, 4 gather warps (the first also loads Q by TMA). The running max is only moved
 // (and O rescaled in TMEM) when it grows by more than 2^8. With several key splits per query, fp32
@@ -45,9 +48,9 @@ constexpr int kDqk = 576;
 constexpr int kDv = 512;
 constexpr int kKeys = 64;                          // selected keys per tile (N of Q K^T)
 constexpr int kRegions = 9;                        // 576 features = 9 blocks of 64 (128 B), 128B swizzle
-constexpr int kQTmemRegions = 5;                   // features 0..319 live in TMEM
+constexpr int kQTmemRegions = 4;                   // features 0..255 live in TMEM
 constexpr int kQRegion = kHeads * 128;             // 16 KB
-constexpr int kQBytes = (kRegions - kQTmemRegions) * kQRegion;   // 64 KB: features 320..575
+constexpr int kQBytes = (kRegions - kQTmemRegions) * kQRegion;   // 80 KB: features 256..575
 constexpr int kKvRegion = kKeys * 128;             // 8 KB
 constexpr int kStageBytes = kRegions * kKvRegion;  // 72 KB
 constexpr int kStages = 2;
@@ -59,7 +62,7 @@ constexpr int kSoftmaxWarps = 4, kMmaWarp = 4, kGatherWarp = 5, kGatherWarps = 4
 constexpr int kMlaThreads = (kSoftmaxWarps + 1 + kGatherWarps) * 32;
 constexpr int kMaxSlots = 2048;                    // selected slots per CTA (split chunk cap)
 constexpr int kTmemCols = 512;
-constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 320, kTmemQ = 352;   // 64 + 32 + 160 columns
+constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 384;   // S: two 64-column buffers
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
 
@@ -123,11 +126,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* kv_full = bars;                    // [kStages] gather (cp.async) -> MMA
   uint64_t* kv_empty = bars + kStages;         // [kStages] MMA (after P V) -> gather
-  uint64_t* s_full = bars + 2 * kStages;       // MMA -> softmax
-  uint64_t* s_empty = s_full + 1;              // softmax (S read) -> MMA
+  uint64_t* s_full = bars + 2 * kStages;       // [2] MMA -> softmax (per score buffer)
   uint64_t* q_full = s_full + 2;               // TMA (Q in smem) + softmax (Q in TMEM) -> MMA
   uint64_t* p_full = s_full + 3;               // softmax (P in TMEM) -> MMA
-  uint64_t* p_empty = s_full + 4;              // MMA (P V done) -> softmax
+  uint64_t* p_empty = s_full + 4;              // MMA (P V done) -> softmax (O rescale only)
   uint64_t* o_full = s_full + 5;               // MMA -> softmax (all P V done)
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -149,8 +151,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       mbar_init(&kv_full[s], kGatherWarps * 32);
       mbar_init(&kv_empty[s], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_empty, kSoftmaxWarps * 32);
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
     mbar_init(q_full, 1 + kSoftmaxWarps * 32);
     mbar_init(p_full, kSoftmaxWarps * 32);
     mbar_init(p_empty, 1);
@@ -215,51 +217,41 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       constexpr uint32_t idesc_pv = idesc_f32acc(1, 1, 128, 256, 0, 1 /*B MN-major*/);
       const uint32_t q_base = smem_u32(q_sm);
       bool ok = mbar_wait(q_full, 0, &abort_flag, p.status);
-      int ns = 0, npv = 0;           // tiles whose Q K^T / P V have been issued
-      uint32_t idle = 0;
-      while (ok && npv < ntiles) {
-        bool progress = false;
-        // Q K^T of tile ns: its keys landed and its score buffer has been read by the softmax
-        if (ns < ntiles && mbar_test_wait(&kv_full[ns % kStages], (ns / kStages) & 1) &&
-            (ns == 0 || mbar_test_wait(s_empty, (ns - 1) & 1))) {
-          fence_proxy_async_smem();      // cp.async (generic proxy) writes -> MMA (async proxy) reads
-          tc_fence_after();
-          const uint32_t kv_base = smem_u32(kv_sm + (ns % kStages) * kStageBytes);
+      auto issue_s = [&](int j) -> bool {     // Q K^T of tile j into score buffer j & 1
+        if (!mbar_wait(&kv_full[j % kStages], (j / kStages) & 1, &abort_flag, p.status)) return false;
+        fence_proxy_async_smem();        // cp.async (generic proxy) writes -> MMA (async proxy) reads
+        tc_fence_after();
+        const uint32_t kv_base = smem_u32(kv_sm + (j % kStages) * kStageBytes);
+        const uint32_t d = tmem + kTmemS + (j & 1) * kKeys;
 #pragma unroll
-          for (int ks = 0; ks < 4 * kQTmemRegions; ++ks)          // Q from TMEM
-            mma_f16_ts(tmem + kTmemS, tmem + kTmemQ + ks * 8,
-                       sdesc_kmajor_sw128(kv_base + (ks >> 2) * kKvRegion + (ks & 3) * 32), idesc_s,
-                       ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < 4 * kQTmemRegions; ++ks)          // Q from TMEM
+          mma_f16_ts(d, tmem + kTmemQ + ks * 8,
+                     sdesc_kmajor_sw128(kv_base + (ks >> 2) * kKvRegion + (ks & 3) * 32), idesc_s, ks > 0 ? 1u : 0u);
 #pragma unroll
-          for (int ks = 4 * kQTmemRegions; ks < kDqk / 16; ++ks)  // Q from shared memory
-            mma_f16_ss(tmem + kTmemS,
-                       sdesc_kmajor_sw128(q_base + ((ks >> 2) - kQTmemRegions) * kQRegion + (ks & 3) * 32),
-                       sdesc_kmajor_sw128(kv_base + (ks >> 2) * kKvRegion + (ks & 3) * 32), idesc_s, 1u);
-          mma_commit(s_full);
-          ++ns;
-          progress = true;
-        }
-        // P V of tile npv: its probabilities are in TMEM
-        if (npv < ns && mbar_test_wait(p_full, npv & 1)) {
-          tc_fence_after();
-          const uint32_t v_base = smem_u32(kv_sm + (npv % kStages) * kStageBytes) + 4 * half * kKvRegion;
+        for (int ks = 4 * kQTmemRegions; ks < kDqk / 16; ++ks)  // Q from shared memory
+          mma_f16_ss(d, sdesc_kmajor_sw128(q_base + ((ks >> 2) - kQTmemRegions) * kQRegion + (ks & 3) * 32),
+                     sdesc_kmajor_sw128(kv_base + (ks >> 2) * kKvRegion + (ks & 3) * 32), idesc_s, 1u);
+        mma_commit(&s_full[j & 1]);
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {    // P V of tile j (P in score buffer j & 1)
+        if (!mbar_wait(p_full, j & 1, &abort_flag, p.status)) return false;
+        tc_fence_after();
+        const uint32_t v_base = smem_u32(kv_sm + (j % kStages) * kStageBytes) + 4 * half * kKvRegion;
 #pragma unroll
-          for (int kk = 0; kk < kKeys / 16; ++kk)
-            mma_f16_ts(tmem + kTmemO, tmem + kTmemP + kk * 8,
-                       sdesc_mnmajor_sw128(v_base + kk * 2048, kKvRegion, 1024), idesc_pv,
-                       (npv > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(p_empty);
-          mma_commit(&kv_empty[npv % kStages]);
-          ++npv;
-          progress = true;
-        }
-        if (progress) {
-          idle = 0;
-        } else if (++idle > kSpinLimit || abort_flag) {
-          if (!abort_flag) set_status(p.status, DSA_ERR_TIMEOUT);
-          abort_flag = 1;
-          ok = false;
-        }
+        for (int kk = 0; kk < kKeys / 16; ++kk)
+          mma_f16_ts(tmem + kTmemO, tmem + kTmemS + (j & 1) * kKeys + kk * 8,
+                     sdesc_mnmajor_sw128(v_base + kk * 2048, kKvRegion, 1024), idesc_pv,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(p_empty);
+        mma_commit(&kv_empty[j % kStages]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      if (ok && ntiles > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < ntiles; ++j) {
+        ok = issue_pv(j);
+        if (ok && j + 2 < ntiles) ok = issue_s(j + 2);
       }
       mma_commit(o_full);
     }
@@ -267,17 +259,17 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // ------------------------------------------------------------------ softmax warps (thread = head)
     const int h = tid;
     const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
-    // Q features 0..319 of head h -> TMEM as bf16 pairs (feature f in column f/2)
+    // Q features 0..255 of head h -> TMEM as bf16 pairs (feature f in column f/2)
     if (ntiles > 0) {
       const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (bt * kHeads + h) * kDqk);
-      uint32_t buf[160];
+      uint32_t buf[128];
 #pragma unroll
-      for (int i = 0; i < 40; ++i) {
+      for (int i = 0; i < 32; ++i) {
         const uint4 v = __ldg(qrow + i);
         buf[4 * i] = v.x; buf[4 * i + 1] = v.y; buf[4 * i + 2] = v.z; buf[4 * i + 3] = v.w;
       }
 #pragma unroll
-      for (int c = 0; c < 5; ++c) tmem_st32(t_row + kTmemQ + c * 32, *reinterpret_cast<uint32_t(*)[32]>(buf + 32 * c));
+      for (int c = 0; c < 4; ++c) tmem_st32(t_row + kTmemQ + c * 32, *reinterpret_cast<uint32_t(*)[32]>(buf + 32 * c));
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(q_full);
@@ -286,19 +278,18 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     bool ok = true;
 #pragma unroll 1
     for (int j = 0; ok && j < ntiles; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full, j & 1, &abort_flag, p.status))) { ok = false; break; }
+      const uint32_t s_col = kTmemS + (j & 1) * kKeys;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, &abort_flag, p.status))) { ok = false; break; }
       tc_fence_after();
       uint32_t r0[32], r1[32];
-      tmem_ld32(t_row + kTmemS, r0);
-      tmem_ld32(t_row + kTmemS + 32, r1);
+      tmem_ld32(t_row + s_col, r0);
+      tmem_ld32(t_row + s_col + 32, r1);
       const int sa = j * kKeys + lane, sb = sa + 32;
       const int va = sa < nslots ? __ldg(idx_row + sa) : -1;
       const int vb = sb < nslots ? __ldg(idx_row + sb) : -1;
       const uint32_t vlo = __ballot_sync(0xffffffffu, va >= 0 && va < p.S_max);
       const uint32_t vhi = __ballot_sync(0xffffffffu, vb >= 0 && vb < p.S_max);
       tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(s_empty);
       float z[kKeys];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -326,26 +317,27 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         pk[i / 2] = pack_bf16(e0, e1);
       }
       l = l * alpha + (((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7])));
-      // P V of the previous tile must be done: P's columns are reused and O may be rescaled
-      if (j >= 1) {
-        if (!__all_sync(0xffffffffu, mbar_wait(p_empty, (j - 1) & 1, &abort_flag, p.status))) { ok = false; break; }
+      // O rescale: every P V issued so far (tiles < j) must be done first
+      const bool rescale = (m != -INFINITY) && (m_new != m);
+      if (__any_sync(0xffffffffu, rescale)) {
+        if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(p_empty, (j - 1) & 1, &abort_flag, p.status))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const bool rescale = (m != -INFINITY) && (m_new != m);
-        if (__any_sync(0xffffffffu, rescale)) {
-          const float a = rescale ? alpha : 1.f;
+        const float a = rescale ? alpha : 1.f;
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            uint32_t o[32];
-            tmem_ld32(t_row + kTmemO + c * 32, o);
-            tmem_ld_wait();
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_row + kTmemO + c * 32, o);
+          tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * a);
-            tmem_st32(t_row + kTmemO + c * 32, o);
-          }
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * a);
+          tmem_st32(t_row + kTmemO + c * 32, o);
         }
       }
       m = m_new;
-      tmem_st32(t_row + kTmemP, pk);
+      tmem_st32(t_row + s_col, pk);              // P over the scores it came from
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
