@@ -11,7 +11,9 @@
 // weighted head-sum are an in-thread reduction over TMEM columns and the [T, 64, S] tensor of
 // per-head products never leaves the SM. The CTA keeps its NQ queries resident and streams
 // 16 KB key tiles through a TMA ring (one warp), one thread issues the MMAs into two TMEM
-// accumulators (ping-pong), and four epilogue warps drain TMEM while the next tile multiplies.
+// accumulators (ping-pong), and sixteen epilogue warps (four per TMEM lane quadrant, one query each)
+// drain TMEM while the next tile multiplies; each thread keeps eight independent partial sums so the
+// head-sum is not one serial FMA chain.
 // Key tiles above the causal diagonal of the CTA's queries are never loaded.
 #include "common.cuh"
 #include "kernels.h"
@@ -22,8 +24,9 @@ namespace {
 
 constexpr int kKeysPerTile = 128;
 constexpr int kTileBytes = kKeysPerTile * 128;      // 16 KB of e4m3 keys
-constexpr int kEpiWarps = 4;
-constexpr int kThreads = (kEpiWarps + 2) * 32;      // + TMA warp + MMA warp
+// epilogue warps: 4 per TMEM lane quadrant with 4 queries per CTA (one query each), 1 with one query
+constexpr int epi_warps(int nq) { return nq >= 4 ? 16 : 4; }
+constexpr int threads_for(int nq) { return (epi_warps(nq) + 2) * 32; }   // + TMA warp + MMA warp
 
 template <int NQ>
 struct ScoresCfg {
@@ -54,12 +57,14 @@ struct ScoresParams {
 }  // namespace
 
 template <int NQ>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_for(NQ), 1)
     index_scores_kernel(const __grid_constant__ CUtensorMap qmap,
                         const __grid_constant__ CUtensorMap kmap, const ScoresParams p) {
   using Cfg = ScoresCfg<NQ>;
   constexpr int N = Cfg::N;
   constexpr int STAGES = Cfg::kStages;
+  constexpr int kEpiWarps = epi_warps(NQ);
+  constexpr int kThreads = threads_for(NQ);
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -73,7 +78,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_full = bars + 2 * STAGES + 4;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
-  __shared__ float wq[NQ][64];
+  __shared__ __align__(16) float wq[NQ][64];
   __shared__ int nvalid[NQ];
   __shared__ int ntiles_sh;
 
@@ -164,37 +169,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------------ epilogue (warps 0-3)
-    const int row_in_tile = warp * 32 + lane;                 // TMEM lane = key within the tile
+    // ------------------------------------------------------------------ epilogue (warps 0-15)
+    // warp w reads TMEM lane quadrant w % 4 (one key per thread) for query w / 4
+    const int quad = warp & 3;
+    constexpr int QPW = 1;                             // queries per epilogue warp
+    const int q_lo = warp >> 2;
+    const bool active = q_lo < NQ;                     // NQ = 1: one warp per quadrant
+    const int row_in_tile = quad * 32 + lane;          // TMEM lane = key within the tile
     for (int i = 0; i < my_tiles; ++i) {
       const int a = i & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[a], (i >> 1) & 1, &abort_flag, p.status))) break;
       tc_fence_after();
-      const int key = (kt_begin + i) * kKeysPerTile + row_in_tile;
-      const float ks = key < p.S_max ? p.k_scale[(int64_t)b * p.S_max + key] : 0.f;
+      if (active) {
+        const int key = (kt_begin + i) * kKeysPerTile + row_in_tile;
+        const float ks = key < p.S_max ? p.k_scale[(int64_t)b * p.S_max + key] : 0.f;
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        uint32_t r0[32], r1[32];
-        const uint32_t taddr = tmem_base + ((uint32_t)(warp * 32) << 16) + a * N + q * 64;
-        tmem_ld32(taddr, r0);
-        tmem_ld32(taddr + 32, r1);
-        tmem_ld_wait();
-        float acc = 0.f;
+        for (int qq = 0; qq < QPW; ++qq) {
+          const int q = q_lo + qq;
+          uint32_t r0[32], r1[32];
+          const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + a * N + q * 64;
+          tmem_ld32(taddr, r0);
+          tmem_ld32(taddr + 32, r1);
+          tmem_ld_wait();
+          float acc[8];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) acc = fmaf(wq[q][j], fmaxf(__uint_as_float(r0[j]), 0.f), acc);
+          for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+          const float4* w4 = reinterpret_cast<const float4*>(&wq[q][0]);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) acc = fmaf(wq[q][32 + j], fmaxf(__uint_as_float(r1[j]), 0.f), acc);
-        const int t = t0 + q;
-        if (t < p.T) {
-          float* dst = p.scores + ((int64_t)b * p.T + t) * p.ld;
-          if (key < nvalid[q]) dst[key] = acc * ks;
-          else if ((p.flags & DSA_FILL_MASKED) && key < p.S_max) dst[key] = -INFINITY;
+          for (int jj = 0; jj < 8; ++jj) {
+            const float4 wa = w4[2 * jj], wb = w4[2 * jj + 1];
+            const float ww[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int j = 8 * jj + u;
+              const float v = __uint_as_float(j < 32 ? r0[j] : r1[j - 32]);
+              acc[u] = fmaf(ww[u], fmaxf(v, 0.f), acc[u]);
+            }
+          }
+          const float tot = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+          const int t = t0 + q;
+          if (t < p.T) {
+            float* dst = p.scores + ((int64_t)b * p.T + t) * p.ld;
+            if (key < nvalid[q]) dst[key] = tot * ks;
+            else if ((p.flags & DSA_FILL_MASKED) && key < p.S_max) dst[key] = -INFINITY;
+          }
         }
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[a]);
     }
-    if (p.flags & DSA_FILL_MASKED) {      // tiles of this split above the causal limit
+    if ((p.flags & DSA_FILL_MASKED) && warp < 4) {   // tiles of this split above the causal limit
       const int kt_stop = min((p.S_max + kKeysPerTile - 1) / kKeysPerTile, kt_begin + p.tiles_per_split);
       for (int kt = max(kt_begin, kt_end); kt < kt_stop; ++kt) {
         const int key = kt * kKeysPerTile + row_in_tile;
@@ -248,7 +272,7 @@ static int launch_scores_nq(const uint8_t* q8, const uint8_t* k8, const ScoresPa
       return DSA_ERR_CUDA;
     configured[dev] = true;
   }
-  index_scores_kernel<NQ><<<(unsigned)grid, kThreads, Cfg::kSmemBytes, stream>>>(qmap, kmap, p);
+  index_scores_kernel<NQ><<<(unsigned)grid, threads_for(NQ), Cfg::kSmemBytes, stream>>>(qmap, kmap, p);
   return dsa_host::check_launch();
 }
 
