@@ -261,6 +261,14 @@ class Step:
         self.flush.zero_()
 
 
+def check_status(dsa, stage):
+    """Raise if a kernel recorded an error during `stage` (with the wait site for a timeout)."""
+    status = dsa.dsa_get_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after {stage}: {dsa.dsa_status_string(status)} "
+                           f"{dsa.dsa_get_error_detail()}")
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as tdist
@@ -275,9 +283,7 @@ def run_ours(args, rank, world, local_rank):
         st.l2_flush()
         st.run()
     torch.cuda.synchronize()
-    status = dsa.dsa_get_device_status()
-    if status != 0:
-        raise RuntimeError(f"device status after warm-up: {dsa.dsa_status_string(status)}")
+    check_status(dsa, "warm-up")
 
     def barrier():
         if world > 1:
@@ -324,6 +330,7 @@ def run_ours(args, rank, world, local_rank):
     t_dev = sum(s.elapsed_time(e) for s, e in steps) / 1e3          # seconds
     per_kernel = {n: v / args.steps / 1e3 for n, v in per_kernel_sum.items()}
     del graph
+    check_status(dsa, "graph replays")
 
     # ---- end to end through host buffers (pinned H2D of the step inputs, D2H of the results)
     for _ in range(max(1, args.warmup)):
@@ -343,9 +350,7 @@ def run_ours(args, rank, world, local_rank):
         e2e.append((s, e))
     barrier()
     t_e2e = sum(s.elapsed_time(e) for s, e in e2e) / 1e3
-    status = dsa.dsa_get_device_status()
-    if status != 0:
-        raise RuntimeError(f"device status after timing: {dsa.dsa_status_string(status)}")
+    check_status(dsa, "end-to-end steps")
 
     # ---- max over ranks
     t_dev, t_e2e = max_over_ranks([t_dev, t_e2e], world, dev)

@@ -201,6 +201,44 @@ DSA_API size_t dsa_sparse_mla_workspace_size(int B, int T, int k);
  */
 DSA_API int dsa_get_device_status(dsa_stream_t stream);
 
+/*
+ * Where a DSA_ERR_TIMEOUT came from. Every wait inside a kernel is bounded (one second of device
+ * time); the first one that gives up records, next to the code, its site (one of the codes
+ * below: high nibble = kernel, low nibble = the barrier waited on), the CTA index and how long
+ * it waited.
+ */
+#define DSA_SITE_SCORES_Q 0x11          /* index scores: MMA waits for the query tile (TMA)      */
+#define DSA_SITE_SCORES_K_FULL 0x12     /* index scores: MMA waits for a key tile (TMA)          */
+#define DSA_SITE_SCORES_K_EMPTY 0x13    /* index scores: TMA waits for a free key stage          */
+#define DSA_SITE_SCORES_ACC_FULL 0x14   /* index scores: epilogue waits for an accumulator       */
+#define DSA_SITE_SCORES_ACC_EMPTY 0x15  /* index scores: MMA waits for a drained accumulator     */
+#define DSA_SITE_MLA_Q 0x21             /* sparse MLA: MMA waits for Q (TMA + TMEM copy)         */
+#define DSA_SITE_MLA_KV_FULL 0x22       /* sparse MLA: MMA waits for a gathered KV tile          */
+#define DSA_SITE_MLA_KV_EMPTY 0x23      /* sparse MLA: gather waits for a free KV stage          */
+#define DSA_SITE_MLA_S_FULL 0x24        /* sparse MLA: softmax waits for a score tile            */
+#define DSA_SITE_MLA_P_FULL 0x25        /* sparse MLA: MMA waits for probabilities               */
+#define DSA_SITE_MLA_P_EMPTY 0x26       /* sparse MLA: softmax waits for P V before rescaling O  */
+#define DSA_SITE_MLA_O_FULL 0x27        /* sparse MLA: epilogue waits for the last P V           */
+#define DSA_SITE_SELFTEST 0x31          /* dsa_selftest_wait_timeout                             */
+
+/*
+ * dsa_get_error_detail - the detail recorded with the last non-OK code that
+ * dsa_get_device_status returned on this device: *site (DSA_SITE_*, 0 if the error was not a
+ * timeout), *block (CTA index) and *wait_us (how long the wait lasted). Any pointer may be NULL.
+ * Returns DSA_OK, or DSA_ERR_CUDA if the device cannot be queried. Host only, no sync.
+ */
+DSA_API int dsa_get_error_detail(int* site, int* block, int* wait_us);
+
+/*
+ * dsa_selftest_wait_timeout - exercises the bounded-wait error path (no counterpart in the
+ * method; it exists so failure detection can be tested without hanging or faulting a GPU).
+ * Launches one CTA on `stream` that waits on a shared-memory barrier nothing arrives on; the
+ * wait gives up after its bound and records DSA_ERR_TIMEOUT with site DSA_SITE_SELFTEST, which
+ * dsa_get_device_status then returns. The CUDA context stays usable. Returns DSA_OK once
+ * launched, DSA_ERR_UNSUPPORTED / DSA_ERR_CUDA otherwise.
+ */
+DSA_API int dsa_selftest_wait_timeout(dsa_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 DSA_API const char* dsa_status_string(int code);
 

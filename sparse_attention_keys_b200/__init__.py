@@ -16,8 +16,9 @@ __all__ = [
     "DsaError", "lib", "lib_path", "DSA_HADAMARD", "DSA_FILL_MASKED", "INDEXER_SOFTMAX_SCALE",
     "MLA_SOFTMAX_SCALE", "dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk",
     "dsa_sparse_mla", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_noalloc",
-    "dsa_sparse_mla_noalloc_scratch_bytes", "dsa_get_device_status", "dsa_status_string",
-    "dsa_device_supported", "dsa_version",
+    "dsa_sparse_mla_noalloc_scratch_bytes", "dsa_get_device_status", "dsa_get_error_detail",
+    "dsa_selftest_wait_timeout", "dsa_status_string", "dsa_device_supported", "dsa_version",
+    "SITE_NAMES",
 ]
 
 DSA_OK = 0
@@ -26,6 +27,14 @@ DSA_FILL_MASKED = 0x2
 MAX_POS = 16384                 # max_seq_len of the model (ModelArgs)
 INDEXER_SOFTMAX_SCALE = 128 ** -0.5
 MLA_SOFTMAX_SCALE = 192 ** -0.5 * (1.0 + 0.1 * __import__("math").log(40.0)) ** 2
+
+# wait-site codes recorded with DSA_ERR_TIMEOUT (DSA_SITE_* in include/dsa.h)
+SITE_NAMES = {
+    0x11: "scores:q", 0x12: "scores:k_full", 0x13: "scores:k_empty", 0x14: "scores:acc_full",
+    0x15: "scores:acc_empty", 0x21: "mla:q", 0x22: "mla:kv_full", 0x23: "mla:kv_empty",
+    0x24: "mla:s_full", 0x25: "mla:p_full", 0x26: "mla:p_empty", 0x27: "mla:o_full",
+    0x31: "selftest",
+}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libdsa.so")
@@ -54,12 +63,15 @@ def _load():
     L.dsa_sparse_mla_noalloc_scratch_bytes.argtypes = []
     L.dsa_sparse_mla_noalloc_scratch_bytes.restype = sz
     L.dsa_get_device_status.argtypes = [vp]
+    L.dsa_get_error_detail.argtypes = [vp, vp, vp]
+    L.dsa_selftest_wait_timeout.argtypes = [vp]
     L.dsa_status_string.argtypes = [i32]
     L.dsa_status_string.restype = ctypes.c_char_p
     L.dsa_device_supported.argtypes = []
     L.dsa_version.restype = ctypes.c_char_p
     for f in ("dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk", "dsa_sparse_mla",
-              "dsa_sparse_mla_noalloc", "dsa_get_device_status", "dsa_device_supported"):
+              "dsa_sparse_mla_noalloc", "dsa_get_device_status", "dsa_get_error_detail",
+              "dsa_selftest_wait_timeout", "dsa_device_supported"):
         getattr(L, f).restype = ctypes.c_int
     return L
 
@@ -232,3 +244,17 @@ def dsa_sparse_mla_noalloc(q, kv, idx, out, lse=None, softmax_scale: float = MLA
 
 def dsa_get_device_status(stream=None) -> int:
     return int(_lib.dsa_get_device_status(_stream(stream)))
+
+
+def dsa_get_error_detail() -> dict:
+    """Detail of the last non-OK status read back: wait site, CTA index, wait length (us)."""
+    site, block, wait_us = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(_lib.dsa_get_error_detail(ctypes.byref(site), ctypes.byref(block), ctypes.byref(wait_us)),
+           "dsa_get_error_detail")
+    return {"site": site.value, "site_name": SITE_NAMES.get(site.value, "none"), "block": block.value,
+            "wait_us": wait_us.value}
+
+
+def dsa_selftest_wait_timeout(stream=None) -> None:
+    """Launch the bounded-wait self-test; the next dsa_get_device_status() reports the timeout."""
+    _check(_lib.dsa_selftest_wait_timeout(_stream(stream)), "dsa_selftest_wait_timeout")

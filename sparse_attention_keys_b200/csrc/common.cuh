@@ -10,13 +10,34 @@
 
 namespace dsa {
 
-// Kernels record the first error they meet in a device status word (0 = none) whose address
-// every launch receives; the host reads and clears it in dsa_get_device_status().
-__device__ __forceinline__ void set_status(int* status, int code) { atomicCAS(status, 0, code); }
+// Kernels record the first error they meet in a device status block whose address every launch
+// receives: word 0 holds the code (0 = none); for a timed-out wait, words 1-3 hold the wait's
+// site (DSA_SITE_* of dsa.h), the CTA index and how long the wait lasted in microseconds. The host
+// reads and clears the block in dsa_get_device_status().
+__device__ __forceinline__ bool set_status(int* status, int code) { return atomicCAS(status, 0, code) == 0; }
 
-// Bound on every spin wait: a wait that has not completed after this many polls records
+// Bound on every spin wait: a wait that has not completed within kWaitLimitNs of device time
+// (checked every kPollsPerCheck polls, with kSpinLimit polls as a second bound) records
 // DSA_ERR_TIMEOUT and the kernel winds down instead of hanging the GPU.
-constexpr uint32_t kSpinLimit = 1u << 26;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr uint32_t kPollsPerCheck = 256;
+constexpr uint32_t kSpinLimit = 1u << 30;
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void record_timeout(int* status, int site, uint64_t waited_ns) {
+  if (set_status(status, DSA_ERR_TIMEOUT)) {
+    volatile int* d = status;
+    d[1] = site;
+    d[2] = (int)blockIdx.x;
+    const uint64_t us = waited_ns / 1000ull;
+    d[3] = us > 0x7fffffffull ? 0x7fffffff : (int)us;
+  }
+}
 
 // ---------------------------------------------------------------------------------- addresses
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -70,78 +91,24 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t phase) {
 }
 
 // Waits for the phase with parity `phase` to complete. Returns false (and records
-// DSA_ERR_TIMEOUT) if it did not complete within kSpinLimit polls. `abort_flag` (shared) lets
-// one thread's timeout release every other waiter in the CTA.
+// DSA_ERR_TIMEOUT with `site`) if it did not complete within the wait bound. `abort_flag`
+// (shared) lets one thread's timeout release every other waiter in the CTA.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, volatile int* abort_flag,
-                                          int* status) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+                                          int* status, int site) {
+  if (mbar_try_wait(bar, phase)) return true;
+  const uint64_t t0 = global_timer_ns();
+  uint64_t waited = 0;
+  for (uint32_t i = 1; i < kSpinLimit; ++i) {
     if (mbar_try_wait(bar, phase)) return true;
     if (abort_flag && *abort_flag) return false;
+    if (i % kPollsPerCheck == 0) {
+      waited = global_timer_ns() - t0;
+      if (waited > kWaitLimitNs) break;
+    }
   }
-  set_status(status, DSA_ERR_TIMEOUT);
+  record_timeout(status, site, waited);
   if (abort_flag) *abort_flag = 1;
   return false;
-}
-
-// Cluster-scope variants: waiting on data another CTA of the cluster released into this CTA's
-// shared memory, and arriving on a barrier that lives in another CTA of the cluster.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t phase) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(phase)
-      : "memory");
-  return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t phase, volatile int* abort_flag,
-                                                  int* status) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    if (mbar_try_wait_cluster(bar, phase)) return true;
-    if (abort_flag && *abort_flag) return false;
-  }
-  set_status(status, DSA_ERR_TIMEOUT);
-  if (abort_flag) *abort_flag = 1;
-  return false;
-}
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-// Address of the same shared-memory location in CTA `rank` of this cluster.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c),
-               "f"(d)
-               : "memory");
-}
-
-// Asynchronous store into another CTA's shared memory; the 16 bytes count towards the
-// complete_tx of `cluster_mbar`, an mbarrier in that same CTA (no release fence on this side).
-__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
-                                            uint32_t cluster_mbar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                   cluster_addr),
-               "r"(a), "r"(b), "r"(c), "r"(d), "r"(cluster_mbar)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // The arrival of the executing thread on `bar` once all its prior cp.async copies have landed.
@@ -156,17 +123,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
-      : "memory");
-}
-
-// Four rows (row0..row3) x one box width starting at column x, written as 4 consecutive box rows.
-__device__ __forceinline__ void tma_gather4(uint32_t dst_smem, const CUtensorMap* map, uint64_t* bar, int32_t x,
-                                            int32_t row0, int32_t row1, int32_t row2, int32_t row3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst_smem),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(row0), "r"(row1), "r"(row2),
-      "r"(row3)
       : "memory");
 }
 

@@ -14,7 +14,21 @@
 
 namespace {
 
-__device__ int g_dsa_status = 0;
+// Status block: code, then (for a timeout) site, CTA index, wait length in microseconds.
+__device__ int g_dsa_status[4] = {0, 0, 0, 0};
+
+// A barrier nothing arrives on, waited on with the kernels' own bounded wait.
+__global__ void selftest_wait_kernel(int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    dsa::mbar_init(&bar, 1);
+    dsa::fence_barrier_init();
+  }
+  __syncthreads();
+  dsa::mbar_wait(&bar, 0, &abort_flag, status, DSA_SITE_SELFTEST);
+}
 
 constexpr int kMaxDevices = 64;
 
@@ -23,6 +37,7 @@ struct DeviceCache {
   bool supported = false;
   int sms = 0;
   int* status = nullptr;
+  int detail[3] = {0, 0, 0};   // site, block, wait_us of the last error read back
 };
 DeviceCache g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -235,13 +250,33 @@ int dsa_get_device_status(dsa_stream_t stream) {
   DeviceCache* c = device_cache();
   if (!c) return DSA_ERR_CUDA;
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return DSA_ERR_CUDA;
-  int v = 0;
-  if (cudaMemcpy(&v, c->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return DSA_ERR_CUDA;
-  if (v != 0) {
-    const int zero = 0;
-    if (cudaMemcpy(c->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return DSA_ERR_CUDA;
+  int v[4] = {0, 0, 0, 0};
+  if (cudaMemcpy(v, c->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return DSA_ERR_CUDA;
+  if (v[0] != 0) {
+    c->detail[0] = v[0] == DSA_ERR_TIMEOUT ? v[1] : 0;
+    c->detail[1] = v[0] == DSA_ERR_TIMEOUT ? v[2] : 0;
+    c->detail[2] = v[0] == DSA_ERR_TIMEOUT ? v[3] : 0;
+    const int zero[4] = {0, 0, 0, 0};
+    if (cudaMemcpy(c->status, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return DSA_ERR_CUDA;
   }
-  return v;
+  return v[0];
+}
+
+int dsa_get_error_detail(int* site, int* block, int* wait_us) {
+  DeviceCache* c = device_cache();
+  if (!c) return DSA_ERR_CUDA;
+  if (site) *site = c->detail[0];
+  if (block) *block = c->detail[1];
+  if (wait_us) *wait_us = c->detail[2];
+  return DSA_OK;
+}
+
+int dsa_selftest_wait_timeout(dsa_stream_t stream) {
+  int* status;
+  int rc = prologue(&status);
+  if (rc != DSA_OK) return rc;
+  selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(status);
+  return dsa_host::check_launch();
 }
 
 const char* dsa_status_string(int code) {

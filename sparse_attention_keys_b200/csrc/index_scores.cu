@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(threads_for(NQ), 1)
       tma_load_2d(q_smem, &qmap, q_full, 0, (b * p.T + t0) * 64);
       for (int i = 0; i < my_tiles; ++i) {
         const int s = i % STAGES;
-        if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) + 1) & 1, &abort_flag, p.status)) break;
+        if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) + 1) & 1, &abort_flag, p.status, DSA_SITE_SCORES_K_EMPTY)) break;
         mbar_arrive_expect_tx(&full[s], kTileBytes);
         tma_load_2d(k_smem + s * kTileBytes, &kmap, &full[s], 0,
                     b * p.S_max + (kt_begin + i) * kKeysPerTile);
@@ -151,11 +151,11 @@ __global__ void __launch_bounds__(threads_for(NQ), 1)
     if (lane == 0 && my_tiles > 0) {
       constexpr uint32_t idesc = idesc_f32acc(0 /*E4M3*/, 0 /*E4M3*/, 128, N, 0, 0);
       const uint32_t q_addr = smem_u32(q_smem);
-      bool ok = mbar_wait(q_full, 0, &abort_flag, p.status);
+      bool ok = mbar_wait(q_full, 0, &abort_flag, p.status, DSA_SITE_SCORES_Q);
       for (int i = 0; ok && i < my_tiles; ++i) {
         const int s = i % STAGES, a = i & 1;
-        if (i >= 2 && !mbar_wait(&acc_empty[a], ((i >> 1) + 1) & 1, &abort_flag, p.status)) break;
-        if (!mbar_wait(&full[s], (i / STAGES) & 1, &abort_flag, p.status)) break;
+        if (i >= 2 && !mbar_wait(&acc_empty[a], ((i >> 1) + 1) & 1, &abort_flag, p.status, DSA_SITE_SCORES_ACC_EMPTY)) break;
+        if (!mbar_wait(&full[s], (i / STAGES) & 1, &abort_flag, p.status, DSA_SITE_SCORES_K_FULL)) break;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(k_smem + s * kTileBytes);
         const uint32_t d_tmem = tmem_base + a * N;
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(threads_for(NQ), 1)
     const int row_in_tile = quad * 32 + lane;          // TMEM lane = key within the tile
     for (int i = 0; i < my_tiles; ++i) {
       const int a = i & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[a], (i >> 1) & 1, &abort_flag, p.status))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[a], (i >> 1) & 1, &abort_flag, p.status, DSA_SITE_SCORES_ACC_FULL))) break;
       tc_fence_after();
       if (active) {
         const int key = (kt_begin + i) * kKeysPerTile + row_in_tile;

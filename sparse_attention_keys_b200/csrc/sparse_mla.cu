@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       idx_next = load_idx(j + 1);                     // one tile ahead
       if (lane < 16 && idx_cur >= p.S_max) set_status(p.status, DSA_ERR_DEVICE_BOUNDS);
       if (j >= kStages &&
-          !__all_sync(0xffffffffu, mbar_wait(&kv_empty[s], ((j / kStages) + 1) & 1, &abort_flag, p.status)))
+          !__all_sync(0xffffffffu, mbar_wait(&kv_empty[s], ((j / kStages) + 1) & 1, &abort_flag, p.status, DSA_SITE_MLA_KV_EMPTY)))
         break;
       const uint32_t base = smem_u32(kv_sm + s * kStageBytes);
 #pragma unroll 4
@@ -216,9 +216,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       constexpr uint32_t idesc_s = idesc_f32acc(1 /*BF16*/, 1, 128, kKeys, 0, 0);
       constexpr uint32_t idesc_pv = idesc_f32acc(1, 1, 128, 256, 0, 1 /*B MN-major*/);
       const uint32_t q_base = smem_u32(q_sm);
-      bool ok = mbar_wait(q_full, 0, &abort_flag, p.status);
+      bool ok = mbar_wait(q_full, 0, &abort_flag, p.status, DSA_SITE_MLA_Q);
       auto issue_s = [&](int j) -> bool {     // Q K^T of tile j into score buffer j & 1
-        if (!mbar_wait(&kv_full[j % kStages], (j / kStages) & 1, &abort_flag, p.status)) return false;
+        if (!mbar_wait(&kv_full[j % kStages], (j / kStages) & 1, &abort_flag, p.status, DSA_SITE_MLA_KV_FULL)) return false;
         fence_proxy_async_smem();        // cp.async (generic proxy) writes -> MMA (async proxy) reads
         tc_fence_after();
         const uint32_t kv_base = smem_u32(kv_sm + (j % kStages) * kStageBytes);
@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         return true;
       };
       auto issue_pv = [&](int j) -> bool {    // P V of tile j (P in score buffer j & 1)
-        if (!mbar_wait(p_full, j & 1, &abort_flag, p.status)) return false;
+        if (!mbar_wait(p_full, j & 1, &abort_flag, p.status, DSA_SITE_MLA_P_FULL)) return false;
         tc_fence_after();
         const uint32_t v_base = smem_u32(kv_sm + (j % kStages) * kStageBytes) + 4 * half * kKvRegion;
 #pragma unroll
@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 #pragma unroll 1
     for (int j = 0; ok && j < ntiles; ++j) {
       const uint32_t s_col = kTmemS + (j & 1) * kKeys;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, &abort_flag, p.status))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, &abort_flag, p.status, DSA_SITE_MLA_S_FULL))) { ok = false; break; }
       tc_fence_after();
       uint32_t r0[32], r1[32];
       tmem_ld32(t_row + s_col, r0);
@@ -320,7 +320,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       // O rescale: every P V issued so far (tiles < j) must be done first
       const bool rescale = (m != -INFINITY) && (m_new != m);
       if (__any_sync(0xffffffffu, rescale)) {
-        if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(p_empty, (j - 1) & 1, &abort_flag, p.status))) {
+        if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(p_empty, (j - 1) & 1, &abort_flag, p.status, DSA_SITE_MLA_P_EMPTY))) {
           ok = false;
           break;
         }
@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     }
     // ---- epilogue: O row (this CTA's 256 output features) / l
     const bool have_o = ntiles > 0 && ok &&
-                        __all_sync(0xffffffffu, mbar_wait(o_full, 0, &abort_flag, p.status));
+                        __all_sync(0xffffffffu, mbar_wait(o_full, 0, &abort_flag, p.status, DSA_SITE_MLA_O_FULL));
     if (have_o) tc_fence_after();
     const float inv = l > 0.f ? 1.f / l : 0.f;
     if (p.nsplit == 1) {

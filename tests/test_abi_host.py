@@ -100,3 +100,10 @@ def test_binding_fails_loudly_without_library(tmp_path):
     r = subprocess.run([sys.executable, "-c", "import sparse_attention_keys_b200"], cwd=tmp_path,
                        capture_output=True, text=True)
     assert r.returncode != 0 and "libdsa.so not built" in r.stderr
+
+
+def test_site_names_match_header(L):
+    """The binding's wait-site table carries exactly the DSA_SITE_* codes the header defines."""
+    import sparse_attention_keys_b200 as m
+    codes = {int(v, 16) for v in re.findall(r"#define DSA_SITE_\w+ (0x[0-9a-fA-F]+)", open(HEADER).read())}
+    assert codes == set(m.SITE_NAMES)
