@@ -10,27 +10,34 @@
 // Tensor cores (tcgen05, kind::f16, bf16 in / fp32 accumulate in TMEM). A 128-head x 512 fp32
 // output accumulator alone would fill all 512 TMEM columns, so each (query, key split) runs on two
 // CTAs that split the OUTPUT features: CTA c accumulates out[:, 256c:256c+256) (256 TMEM columns).
-// Each CTA computes the full 576-feature score itself (Q for all 128 heads resident on chip: features
-// 0..255 in TMEM as bf16 pairs, 256..575 in shared memory via TMA), so the pair never exchanges data: this costs 1.5x the Q K^T work
-// of a single pass, but exchanging 128 x 64 fp32 partial scores per tile between CTAs runs into
-// the limited bandwidth of distributed shared memory.
+// Each CTA computes the full 576-feature score itself, so the pair never exchanges data (1.5x the
+// Q K^T work of a single pass; exchanging 128 x 32 fp32 partial scores per tile through distributed
+// shared memory measured slower than recomputing them).
 //
-// Selected 1152-byte latent rows are gathered by four warps with 16-byte cp.async, one warp-wide
-// coalesced 512-byte request per instruction, written straight into the 128B-swizzled operand
-// layout (unselected slots are zero-filled) into a double-buffered ring of 64-key tiles. (Measured
-// on B200 with one CTA per SM: this moves ~2.5x more bytes per SM than TMA tile::gather4 with
-// 128-byte boxes.) One shared-memory tile is both the
-// K-major B operand of Q K^T (N = keys) and the MN-major B operand of P V (N = features).
-// TMEM: O [0,256), two score buffers S0 [256,320) and S1 [320,384), Q features 0..255 as bf16
-// pairs [384,512) (the A operand of the first 16 K-steps of Q K^T; the last 20 read Q from shared
-// memory). The probabilities of tile j overwrite the first 32 columns of the score buffer they came
-// from (bf16 pairs, the A operand of P V), so the MMA thread can run a fixed order
-// S0, S1, PV0, S2, PV1, S3, ...: Q K^T of tile j+2 is issued after P V of tile j, which the tensor
-// pipe executes in order, and it never waits for the softmax to free a buffer.
-// Per CTA: 4 softmax warps (thread = head = TMEM lane), 1 MMA-issuing thread that issues Q K^T and
-// P V in whichever order their inputs become ready, 4 gather warps (the first also loads Q by TMA). The running max is only moved
-// (and O rescaled in TMEM) when it grows by more than 2^8. With several key splits per query, fp32
-// partials (O, max, sum) go to the caller's workspace and a second kernel merges them.
+// TMEM: O [0,256), three 32-column score buffers [256,352), and Q features 0..319 of all 128 heads
+// as bf16 pairs [352,512) (the A operand of the first 20 K-steps of Q K^T; the last 16 read Q
+// features 320..575 from shared memory). The probabilities of tile j overwrite the first 16
+// columns of the score buffer they came from (the A operand of P V).
+//
+// MMA issue: one thread issues a tcgen05.mma no faster than about every 30 ns (measured on B200),
+// while a 128x32x16 MMA with A in TMEM takes about 9 ns on the tensor pipe, so Q K^T (36 MMAs
+// per tile) is issued by three warps, one per score buffer (tile j uses buffer j mod 3), with every
+// descriptor a precomputed base plus a constant; a fourth warp issues P V (two 128x256x16 MMAs per
+// tile). Each buffer cycles through Q K^T, softmax and P V; three buffers keep the tensor pipe busy
+// while the softmax of another tile runs.
+//
+// Selected 1152-byte latent rows are gathered in 32-key tiles by four warps with 16-byte cp.async
+// (warp-wide 512-byte requests, unselected slots zero-filled), straight into the 128B-swizzled
+// operand layout, split over two rings: the four 64-feature blocks this CTA's P V reads ("V ring",
+// 16 KB per tile, 5 slots, freed when P V of the tile completes) and the other five blocks ("rest
+// ring", 20 KB, 4 slots, freed as soon as Q K^T of the tile completes). Freeing the rest early lets
+// the gathers run about four tiles ahead of the tensor core instead of waiting for P V.
+// One shared-memory block is both the K-major B operand of Q K^T (N = keys) and the MN-major B
+// operand of P V (N = features).
+// Per CTA: 4 softmax warps (thread = head = TMEM lane), 1 P V warp, 4 gather warps (the first also
+// loads Q features 320..575 by TMA), 3 Q K^T warps. The running max is only moved (and O rescaled in
+// TMEM) when it grows by more than 2^8. With several key splits per query, fp32 partials (O, max,
+// sum) go to the caller's workspace and a second kernel merges them.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -46,25 +53,32 @@ namespace {
 constexpr int kHeads = 128;
 constexpr int kDqk = 576;
 constexpr int kDv = 512;
-constexpr int kKeys = 64;                          // selected keys per tile (N of Q K^T)
+constexpr int kKeys = 32;                          // selected keys per tile (N of Q K^T)
 constexpr int kRegions = 9;                        // 576 features = 9 blocks of 64 (128 B), 128B swizzle
-constexpr int kQTmemRegions = 4;                   // features 0..255 live in TMEM
+constexpr int kVRegions = 4;                       // the blocks of this CTA's 256 output features
+constexpr int kRestRegions = kRegions - kVRegions; // the other half's 4 latent blocks + the rotary one
+constexpr int kQTmemRegions = 5;                   // Q features 0..319 live in TMEM
 constexpr int kQRegion = kHeads * 128;             // 16 KB
-constexpr int kQBytes = (kRegions - kQTmemRegions) * kQRegion;   // 80 KB: features 256..575
-constexpr int kKvRegion = kKeys * 128;             // 8 KB
-constexpr int kStageBytes = kRegions * kKvRegion;  // 72 KB
-constexpr int kStages = 2;
+constexpr int kQBytes = (kRegions - kQTmemRegions) * kQRegion;   // 64 KB: features 320..575
+constexpr int kKvRegion = kKeys * 128;             // 4 KB: one 64-feature block of a tile
+constexpr int kVSlotBytes = kVRegions * kKvRegion;        // 16 KB
+constexpr int kRestSlotBytes = kRestRegions * kKvRegion;  // 20 KB
+constexpr int kVSlots = 5, kRestSlots = 4, kSBufs = 3;
 constexpr int kOffQ = 0;
-constexpr int kOffKV = kOffQ + kQBytes;
-constexpr int kOffBar = kOffKV + kStages * kStageBytes;
+constexpr int kOffV = kOffQ + kQBytes;
+constexpr int kOffRest = kOffV + kVSlots * kVSlotBytes;
+constexpr int kOffBar = kOffRest + kRestSlots * kRestSlotBytes;
 constexpr int kSmemBytes = 1024 + kOffBar + 256;
-constexpr int kSoftmaxWarps = 4, kMmaWarp = 4, kGatherWarp = 5, kGatherWarps = 4;
-constexpr int kMlaThreads = (kSoftmaxWarps + 1 + kGatherWarps) * 32;
+constexpr int kSoftmaxWarps = 4, kPvWarp = 4, kGatherWarp = 5, kGatherWarps = 4, kQkWarp = 9, kQkWarps = kSBufs;
+constexpr int kMlaThreads = (kSoftmaxWarps + 1 + kGatherWarps + kQkWarps) * 32;
 constexpr int kMaxSlots = 2048;                    // selected slots per CTA (split chunk cap)
 constexpr int kTmemCols = 512;
-constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 384;   // S: two 64-column buffers
+constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = kTmemS + kSBufs * kKeys;   // S: three 32-column buffers
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+static_assert(kTmemQ + kQTmemRegions * 32 == kTmemCols, "TMEM budget");
+static_assert(kTmemQ <= kTmemCols, "TMEM budget");
 
 struct MlaSplit {
   int nsplit;
@@ -116,21 +130,46 @@ struct MlaParams {
   int* status;
 };
 
+// Q K^T of one 32-key tile: 20 K-steps with Q from TMEM, then 16 with Q from shared memory. HALF
+// fixes which ring holds each 64-feature block, so every B descriptor is a base plus a constant.
+// *_lo: low descriptor words (start address >> 4 in bits 0-13) of the shared-memory bases; hi: the
+// common high word of the K-major 128B-swizzle descriptors.
+template <int HALF>
+__device__ __forceinline__ void issue_qk_tile(uint32_t d, uint32_t tq, uint32_t q_lo, uint32_t v_lo, uint32_t r_lo,
+                                              uint32_t hi, uint32_t idesc) {
+#pragma unroll
+  for (int r = 0; r < kRegions; ++r) {
+    const bool in_v = r < 8 && (r >> 2) == HALF;
+    const uint32_t kb = in_v ? v_lo + (uint32_t)(((r & 3) * kKvRegion) >> 4)
+                             : r_lo + (uint32_t)(((r == 8 ? 4 : (r & 3)) * kKvRegion) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const int ks = 4 * r + kk;
+      if (r < kQTmemRegions) {
+        if (ks == 0) mma_f16_ts_lo<0>(d, tq, kb, hi, idesc);
+        else mma_f16_ts_lo<1>(d, tq + ks * 8, kb + kk * 2, hi, idesc);
+      } else {
+        mma_f16_ss_lo<1>(d, q_lo + (uint32_t)(((r - kQTmemRegions) * kQRegion) >> 4) + kk * 2, hi, kb + kk * 2, hi,
+                         idesc);
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kMlaThreads, 1)
-    sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap kv_map,
-                      const MlaParams p) {
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_sm = smem + kOffQ;
-  uint8_t* kv_sm = smem + kOffKV;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* kv_full = bars;                    // [kStages] gather (cp.async) -> MMA
-  uint64_t* kv_empty = bars + kStages;         // [kStages] MMA (after P V) -> gather
-  uint64_t* s_full = bars + 2 * kStages;       // [2] MMA -> softmax (per score buffer)
-  uint64_t* q_full = s_full + 2;               // TMA (Q in smem) + softmax (Q in TMEM) -> MMA
-  uint64_t* p_full = s_full + 3;               // softmax (P in TMEM) -> MMA
-  uint64_t* p_empty = s_full + 4;              // MMA (P V done) -> softmax (O rescale only)
-  uint64_t* o_full = s_full + 5;               // MMA -> softmax (all P V done)
+  uint64_t* kv_full = bars;                         // [kRestSlots] gather (cp.async) -> Q K^T issuer
+  uint64_t* rest_empty = bars + kRestSlots;         // [kRestSlots] Q K^T done -> gather
+  uint64_t* v_empty = bars + 2 * kRestSlots;        // [kVSlots]    P V done -> gather
+  uint64_t* s_full = v_empty + kVSlots;             // [kSBufs] Q K^T done -> softmax (per score buffer)
+  uint64_t* p_full = s_full + kSBufs;               // [kSBufs] softmax (P in TMEM) -> P V issuer
+  uint64_t* pv_done = p_full + kSBufs;              // [kSBufs] P V done -> Q K^T issuer, softmax (O rescale)
+  uint64_t* q_full = pv_done + kSBufs;              // TMA (Q in smem) + softmax (Q in TMEM) -> Q K^T issuers
+  uint64_t* o_full = q_full + 1;                    // last P V done -> epilogue
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -144,22 +183,25 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   const int nslots = max(0, min(p.k, slot0 + p.chunk) - slot0);
   const int ntiles = (nslots + kKeys - 1) / kKeys;
   const int32_t* idx_row = p.idx + bt * p.k + slot0;
+  const uint32_t v_ring = smem_u32(smem + kOffV), rest_ring = smem_u32(smem + kOffRest);
 
   if (tid == 0) {
     abort_flag = 0;
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kRestSlots; ++s) {
       mbar_init(&kv_full[s], kGatherWarps * 32);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&rest_empty[s], 1);
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
+    for (int s = 0; s < kVSlots; ++s) mbar_init(&v_empty[s], 1);
+    for (int i = 0; i < kSBufs; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], kSoftmaxWarps * 32);
+      mbar_init(&pv_done[i], 1);
+    }
     mbar_init(q_full, 1 + kSoftmaxWarps * 32);
-    mbar_init(p_full, kSoftmaxWarps * 32);
-    mbar_init(p_empty, 1);
     mbar_init(o_full, 1);
     fence_barrier_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == kPvWarp) {
     tmem_alloc(&tmem_base_sh, kTmemCols);
     tmem_relinquish();
   }
@@ -168,10 +210,39 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  if (warp >= kGatherWarp) {
+  if (warp >= kQkWarp) {
+    // ------------------------------------------------------------------ Q K^T issuers
+    // warp kQkWarp + e issues Q K^T of the tiles j = e (mod 3) into score buffer e: with one score
+    // buffer per issuing thread, a buffer's softmax and P V overlap the other buffers' Q K^T
+    const int e = warp - kQkWarp;
+    if (lane == 0 && ntiles > e) {
+      const uint32_t idesc_s = idesc_f32acc(1 /*BF16*/, 1, 128, kKeys, 0, 0);
+      const uint64_t q_desc = sdesc_kmajor_sw128(smem_u32(q_sm));
+      const uint32_t hi = (uint32_t)(q_desc >> 32), q_lo = (uint32_t)q_desc;
+      const uint32_t v_lo0 = (uint32_t)sdesc_kmajor_sw128(v_ring), r_lo0 = (uint32_t)sdesc_kmajor_sw128(rest_ring);
+      const uint32_t d = tmem + kTmemS + e * kKeys, tq = tmem + kTmemQ;
+      bool ok = mbar_wait(q_full, 0, &abort_flag, p.status, DSA_SITE_MLA_Q);
+      for (int j = e; ok && j < ntiles; j += kSBufs) {
+        // score buffer e still holds P of tile j - 3 until its P V completes
+        if (j >= kSBufs &&
+            !mbar_wait(&pv_done[e], ((j / kSBufs) + 1) & 1, &abort_flag, p.status, DSA_SITE_MLA_P_EMPTY))
+          break;
+        if (!mbar_wait(&kv_full[j % kRestSlots], (j / kRestSlots) & 1, &abort_flag, p.status, DSA_SITE_MLA_KV_FULL))
+          break;
+        fence_proxy_async_smem();        // cp.async (generic proxy) writes -> MMA (async proxy) reads
+        tc_fence_after();
+        const uint32_t v_lo = v_lo0 + (uint32_t)(((j % kVSlots) * kVSlotBytes) >> 4);
+        const uint32_t r_lo = r_lo0 + (uint32_t)(((j % kRestSlots) * kRestSlotBytes) >> 4);
+        if (half == 0) issue_qk_tile<0>(d, tq, q_lo, v_lo, r_lo, hi, idesc_s);
+        else issue_qk_tile<1>(d, tq, q_lo, v_lo, r_lo, hi, idesc_s);
+        mma_commit(&s_full[e]);
+        mma_commit(&rest_empty[j % kRestSlots]);
+      }
+    }
+  } else if (warp >= kGatherWarp) {
     // ------------------------------------------------------------------ gather warps
-    // gather warp w copies keys 16w..16w+15 of each tile; per key, lanes take 16-byte chunks
-    // lane, lane+32, lane+64 of the 72 in the row (contiguous 512-byte warp requests)
+    // gather warp w copies keys 8w..8w+7 of each tile; for every key, lane L copies the 16-byte
+    // chunks L (block L/8), L+32 (block 4+L/8) and, for L < 8, L+64 (the rotary block)
     const int w = warp - kGatherWarp;
     if (w == 0 && lane == 0 && ntiles > 0) {
       prefetch_tensormap(&q_map);
@@ -180,78 +251,58 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         tma_load_2d(q_sm + (r - kQTmemRegions) * kQRegion, &q_map, q_full, 64 * r, (int32_t)(bt * kHeads));
     }
     const uint16_t* kv_b = p.kv + (int64_t)b * p.S_max * kDqk;
+    const uint32_t blk = (uint32_t)(lane >> 3) * kKvRegion;      // block of chunks L and L+32 in its ring slot
     auto load_idx = [&](int j) -> int {
-      const int slot = j * kKeys + 16 * w + (lane & 15);
+      const int slot = j * kKeys + 8 * w + (lane & 7);
       return (j < ntiles && slot < nslots) ? __ldg(idx_row + slot) : -1;
     };
     int idx_next = load_idx(0);
     for (int j = 0; j < ntiles; ++j) {
-      const int s = j % kStages;
       const int idx_cur = idx_next;
       idx_next = load_idx(j + 1);                     // one tile ahead
-      if (lane < 16 && idx_cur >= p.S_max) set_status(p.status, DSA_ERR_DEVICE_BOUNDS);
-      if (j >= kStages &&
-          !__all_sync(0xffffffffu, mbar_wait(&kv_empty[s], ((j / kStages) + 1) & 1, &abort_flag, p.status, DSA_SITE_MLA_KV_EMPTY)))
+      if (lane < 8 && idx_cur >= p.S_max) set_status(p.status, DSA_ERR_DEVICE_BOUNDS);
+      if (j >= kRestSlots &&
+          !__all_sync(0xffffffffu, mbar_wait(&rest_empty[j % kRestSlots], ((j / kRestSlots) + 1) & 1, &abort_flag,
+                                             p.status, DSA_SITE_MLA_KV_EMPTY)))
         break;
-      const uint32_t base = smem_u32(kv_sm + s * kStageBytes);
-#pragma unroll 4
-      for (int kk = 0; kk < 16; ++kk) {
+      if (j >= kVSlots &&
+          !__all_sync(0xffffffffu, mbar_wait(&v_empty[j % kVSlots], ((j / kVSlots) + 1) & 1, &abort_flag,
+                                             p.status, DSA_SITE_MLA_KV_EMPTY)))
+        break;
+      const uint32_t v_slot = v_ring + (j % kVSlots) * kVSlotBytes;
+      const uint32_t r_slot = rest_ring + (j % kRestSlots) * kRestSlotBytes;
+      const uint32_t d0 = (half == 0 ? v_slot : r_slot) + blk;           // latent block L/8
+      const uint32_t d1 = (half == 1 ? v_slot : r_slot) + blk;           // latent block 4 + L/8
+      const uint32_t d2 = r_slot + 4 * kKvRegion;                        // rotary block
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
         const int v = __shfl_sync(0xffffffffu, idx_cur, kk);
         const bool ok = v >= 0 && v < p.S_max;
-        const int key = 16 * w + kk;
-        const uint16_t* src = kv_b + (int64_t)(ok ? v : 0) * kDqk;
-#pragma unroll
-        for (int i = 0; i < 3; ++i) {
-          const int c = lane + 32 * i;
-          if (c < 72)
-            cp_async_16_zfill(base + (c >> 3) * kKvRegion + sw128(key, c & 7), src + c * 8, ok);
-        }
+        const uint32_t off = sw128(8 * w + kk, lane & 7);
+        const uint16_t* src = kv_b + (int64_t)(ok ? v : 0) * kDqk + lane * 8;
+        cp_async_16_zfill(d0 + off, src, ok);
+        cp_async_16_zfill(d1 + off, src + 256, ok);
+        if (lane < 8) cp_async_16_zfill(d2 + off, src + 512, ok);
       }
-      cp_async_mbar_arrive(&kv_full[s]);
+      cp_async_mbar_arrive(&kv_full[j % kRestSlots]);
     }
     cp_async_wait_all();
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == kPvWarp) {
+    // ------------------------------------------------------------------ P V issuer
     if (lane == 0 && ntiles > 0) {
-      constexpr uint32_t idesc_s = idesc_f32acc(1 /*BF16*/, 1, 128, kKeys, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_f32acc(1, 1, 128, 256, 0, 1 /*B MN-major*/);
-      const uint32_t q_base = smem_u32(q_sm);
-      bool ok = mbar_wait(q_full, 0, &abort_flag, p.status, DSA_SITE_MLA_Q);
-      auto issue_s = [&](int j) -> bool {     // Q K^T of tile j into score buffer j & 1
-        if (!mbar_wait(&kv_full[j % kStages], (j / kStages) & 1, &abort_flag, p.status, DSA_SITE_MLA_KV_FULL)) return false;
-        fence_proxy_async_smem();        // cp.async (generic proxy) writes -> MMA (async proxy) reads
+      const uint32_t idesc_pv = idesc_f32acc(1, 1, 128, 256, 0, 1 /*B MN-major*/);
+      const uint64_t v_desc = sdesc_mnmajor_sw128(v_ring, kKvRegion, 1024);
+      const uint32_t hi = (uint32_t)(v_desc >> 32), v_lo0 = (uint32_t)v_desc;
+      for (int j = 0; j < ntiles; ++j) {
+        if (!mbar_wait(&p_full[j % kSBufs], (j / kSBufs) & 1, &abort_flag, p.status, DSA_SITE_MLA_P_FULL)) break;
         tc_fence_after();
-        const uint32_t kv_base = smem_u32(kv_sm + (j % kStages) * kStageBytes);
-        const uint32_t d = tmem + kTmemS + (j & 1) * kKeys;
-#pragma unroll
-        for (int ks = 0; ks < 4 * kQTmemRegions; ++ks)          // Q from TMEM
-          mma_f16_ts(d, tmem + kTmemQ + ks * 8,
-                     sdesc_kmajor_sw128(kv_base + (ks >> 2) * kKvRegion + (ks & 3) * 32), idesc_s, ks > 0 ? 1u : 0u);
-#pragma unroll
-        for (int ks = 4 * kQTmemRegions; ks < kDqk / 16; ++ks)  // Q from shared memory
-          mma_f16_ss(d, sdesc_kmajor_sw128(q_base + ((ks >> 2) - kQTmemRegions) * kQRegion + (ks & 3) * 32),
-                     sdesc_kmajor_sw128(kv_base + (ks >> 2) * kKvRegion + (ks & 3) * 32), idesc_s, 1u);
-        mma_commit(&s_full[j & 1]);
-        return true;
-      };
-      auto issue_pv = [&](int j) -> bool {    // P V of tile j (P in score buffer j & 1)
-        if (!mbar_wait(p_full, j & 1, &abort_flag, p.status, DSA_SITE_MLA_P_FULL)) return false;
-        tc_fence_after();
-        const uint32_t v_base = smem_u32(kv_sm + (j % kStages) * kStageBytes) + 4 * half * kKvRegion;
-#pragma unroll
-        for (int kk = 0; kk < kKeys / 16; ++kk)
-          mma_f16_ts(tmem + kTmemO, tmem + kTmemS + (j & 1) * kKeys + kk * 8,
-                     sdesc_mnmajor_sw128(v_base + kk * 2048, kKvRegion, 1024), idesc_pv,
-                     (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(p_empty);
-        mma_commit(&kv_empty[j % kStages]);
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      if (ok && ntiles > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < ntiles; ++j) {
-        ok = issue_pv(j);
-        if (ok && j + 2 < ntiles) ok = issue_s(j + 2);
+        const uint32_t v_lo = v_lo0 + (uint32_t)(((j % kVSlots) * kVSlotBytes) >> 4);
+        const uint32_t a = tmem + kTmemS + (j % kSBufs) * kKeys;
+        if (j == 0) mma_f16_ts_lo<0>(tmem + kTmemO, a, v_lo, hi, idesc_pv);
+        else mma_f16_ts_lo<1>(tmem + kTmemO, a, v_lo, hi, idesc_pv);
+        mma_f16_ts_lo<1>(tmem + kTmemO, a + 8, v_lo + (2048 >> 4), hi, idesc_pv);    // keys 16..31
+        mma_commit(&pv_done[j % kSBufs]);
+        mma_commit(&v_empty[j % kVSlots]);
       }
       mma_commit(o_full);
     }
@@ -259,49 +310,53 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // ------------------------------------------------------------------ softmax warps (thread = head)
     const int h = tid;
     const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
-    // Q features 0..255 of head h -> TMEM as bf16 pairs (feature f in column f/2)
+    // Q features 0..319 of head h -> TMEM as bf16 pairs (feature f in column f/2)
     if (ntiles > 0) {
       const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (bt * kHeads + h) * kDqk);
-      uint32_t buf[128];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const uint4 v = __ldg(qrow + i);
-        buf[4 * i] = v.x; buf[4 * i + 1] = v.y; buf[4 * i + 2] = v.z; buf[4 * i + 3] = v.w;
+      for (int c = 0; c < kQTmemRegions; ++c) {
+        uint32_t buf[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 v = __ldg(qrow + 8 * c + i);
+          buf[4 * i] = v.x; buf[4 * i + 1] = v.y; buf[4 * i + 2] = v.z; buf[4 * i + 3] = v.w;
+        }
+        tmem_st32(t_row + kTmemQ + c * 32, buf);
       }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_st32(t_row + kTmemQ + c * 32, *reinterpret_cast<uint32_t(*)[32]>(buf + 32 * c));
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(q_full);
     }
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+    int v_next = lane < nslots ? __ldg(idx_row + lane) : -1;     // slot j * 32 + lane of the next tile
 #pragma unroll 1
     for (int j = 0; ok && j < ntiles; ++j) {
-      const uint32_t s_col = kTmemS + (j & 1) * kKeys;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, &abort_flag, p.status, DSA_SITE_MLA_S_FULL))) { ok = false; break; }
+      const uint32_t s_col = kTmemS + (j % kSBufs) * kKeys;
+      const int v_cur = v_next;
+      {
+        const int sn = (j + 1) * kKeys + lane;
+        v_next = sn < nslots ? __ldg(idx_row + sn) : -1;
+      }
+      const uint32_t vmask = __ballot_sync(0xffffffffu, v_cur >= 0 && v_cur < p.S_max);
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j % kSBufs], (j / kSBufs) & 1, &abort_flag, p.status,
+                                             DSA_SITE_MLA_S_FULL))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
-      uint32_t r0[32], r1[32];
+      uint32_t r0[32];
       tmem_ld32(t_row + s_col, r0);
-      tmem_ld32(t_row + s_col + 32, r1);
-      const int sa = j * kKeys + lane, sb = sa + 32;
-      const int va = sa < nslots ? __ldg(idx_row + sa) : -1;
-      const int vb = sb < nslots ? __ldg(idx_row + sb) : -1;
-      const uint32_t vlo = __ballot_sync(0xffffffffu, va >= 0 && va < p.S_max);
-      const uint32_t vhi = __ballot_sync(0xffffffffu, vb >= 0 && vb < p.S_max);
       tmem_ld_wait();
       float z[kKeys];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        z[i] = ((vlo >> i) & 1u) ? __uint_as_float(r0[i]) * p.scale_log2 : -INFINITY;
-        z[32 + i] = ((vhi >> i) & 1u) ? __uint_as_float(r1[i]) * p.scale_log2 : -INFINITY;
-      }
-      float t8[8];
+      for (int i = 0; i < kKeys; ++i) z[i] = ((vmask >> i) & 1u) ? __uint_as_float(r0[i]) * p.scale_log2 : -INFINITY;
+      float t4[4];
 #pragma unroll
-      for (int g = 0; g < 8; ++g)
-        t8[g] = fmaxf(fmaxf(fmaxf(z[8 * g], z[8 * g + 1]), fmaxf(z[8 * g + 2], z[8 * g + 3])),
+      for (int g = 0; g < 4; ++g)
+        t4[g] = fmaxf(fmaxf(fmaxf(z[8 * g], z[8 * g + 1]), fmaxf(z[8 * g + 2], z[8 * g + 3])),
                       fmaxf(fmaxf(z[8 * g + 4], z[8 * g + 5]), fmaxf(z[8 * g + 6], z[8 * g + 7])));
-      const float mx = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])), fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
+      const float mx = fmaxf(fmaxf(t4[0], t4[1]), fmaxf(t4[2], t4[3]));
       float m_new = m, alpha = 1.f;
       if (mx > m + kRescaleThreshold) {
         m_new = mx;
@@ -317,10 +372,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         pk[i / 2] = pack_bf16(e0, e1);
       }
       l = l * alpha + (((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7])));
-      // O rescale: every P V issued so far (tiles < j) must be done first
+      // O rescale: P V of every earlier tile must be done first (P V of tile j - 1 completes last)
       const bool rescale = (m != -INFINITY) && (m_new != m);
       if (__any_sync(0xffffffffu, rescale)) {
-        if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(p_empty, (j - 1) & 1, &abort_flag, p.status, DSA_SITE_MLA_P_EMPTY))) {
+        if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(&pv_done[(j - 1) % kSBufs], ((j - 1) / kSBufs) & 1, &abort_flag,
+                                                         p.status, DSA_SITE_MLA_P_EMPTY))) {
           ok = false;
           break;
         }
@@ -337,10 +393,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         }
       }
       m = m_new;
-      tmem_st32(t_row + s_col, pk);              // P over the scores it came from
+      tmem_st16(t_row + s_col, pk);              // P over the scores it came from
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[j % kSBufs]);
     }
     // ---- epilogue: O row (this CTA's 256 output features) / l
     const bool have_o = ntiles > 0 && ok &&
@@ -394,7 +450,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kPvWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -476,13 +532,11 @@ int launch_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
   }
   const int64_t grid = BT * s.nsplit * 2;          // two CTAs (output-feature halves) per (query, split)
   if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;
-  CUtensorMap q_map, kv_map;
+  CUtensorMap q_map;
   if (!dsa_host::encode_tensor_map_2d(&q_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (void*)q, kDqk,
-                                      (uint64_t)BT * kHeads, kDqk * 2, 64, kHeads, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !dsa_host::encode_tensor_map_2d(&kv_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (void*)kv, kDqk,
-                                      (uint64_t)B * S_max, kDqk * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+                                      (uint64_t)BT * kHeads, kDqk * 2, 64, kHeads, CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
-  sparse_mla_kernel<<<(unsigned)grid, kMlaThreads, kSmemBytes, stream>>>(q_map, kv_map, p);
+  sparse_mla_kernel<<<(unsigned)grid, kMlaThreads, kSmemBytes, stream>>>(q_map, p);
   int rc = dsa_host::check_launch();
   if (rc != DSA_OK || s.nsplit == 1) return rc;
   const int64_t rows = BT * kHeads;
