@@ -185,6 +185,18 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   const int32_t* idx_row = p.idx + bt * p.k + slot0;
   const uint32_t v_ring = smem_u32(smem + kOffV), rest_ring = smem_u32(smem + kOffRest);
 
+  // Start the first global reads before the set-up barrier: the first tile's indices (gather warps)
+  // and, into L2, each head's Q features 0..319 (softmax warps, staged into TMEM below).
+  int idx_first = -1;
+  if (warp >= kGatherWarp && warp < kQkWarp) {
+    const int slot = 8 * (warp - kGatherWarp) + (lane & 7);
+    if (slot < nslots) idx_first = __ldg(idx_row + slot);
+  } else if (warp < kSoftmaxWarps && ntiles > 0) {
+    const char* qrow = reinterpret_cast<const char*>(p.q + (bt * kHeads + tid) * kDqk);
+#pragma unroll
+    for (int i = 0; i < kQTmemRegions; ++i) asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + 128 * i));
+  }
+
   if (tid == 0) {
     abort_flag = 0;
     for (int s = 0; s < kRestSlots; ++s) {
@@ -256,7 +268,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       const int slot = j * kKeys + 8 * w + (lane & 7);
       return (j < ntiles && slot < nslots) ? __ldg(idx_row + slot) : -1;
     };
-    int idx_next = load_idx(0);
+    int idx_next = idx_first;                        // load_idx(0), issued before the set-up barrier
     for (int j = 0; j < ntiles; ++j) {
       const int idx_cur = idx_next;
       idx_next = load_idx(j + 1);                     // one tile ahead
@@ -312,17 +324,29 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
     // Q features 0..319 of head h -> TMEM as bf16 pairs (feature f in column f/2)
     if (ntiles > 0) {
+      // two batches of loads, each fully in flight before its TMEM stores (which order memory)
       const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (bt * kHeads + h) * kDqk);
+      auto stage = [&](int c0, int nc) {
+        uint4 v[3 * 8];
 #pragma unroll
-      for (int c = 0; c < kQTmemRegions; ++c) {
-        uint32_t buf[32];
+        for (int i = 0; i < 3 * 8; ++i)
+          if (i < nc * 8) v[i] = __ldg(qrow + 8 * c0 + i);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 v = __ldg(qrow + 8 * c + i);
-          buf[4 * i] = v.x; buf[4 * i + 1] = v.y; buf[4 * i + 2] = v.z; buf[4 * i + 3] = v.w;
+        for (int c = 0; c < 3; ++c) {
+          if (c < nc) {
+            uint32_t buf[32];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              buf[4 * i] = v[8 * c + i].x; buf[4 * i + 1] = v[8 * c + i].y;
+              buf[4 * i + 2] = v[8 * c + i].z; buf[4 * i + 3] = v[8 * c + i].w;
+            }
+            tmem_st32(t_row + kTmemQ + (c0 + c) * 32, buf);
+          }
         }
-        tmem_st32(t_row + kTmemQ + c * 32, buf);
-      }
+      };
+      static_assert(kQTmemRegions == 5, "Q staging batches");
+      stage(0, 3);
+      stage(3, 2);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(q_full);
