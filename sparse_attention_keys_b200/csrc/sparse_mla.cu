@@ -85,18 +85,31 @@ struct MlaSplit {
   int chunk;     // selected slots per split (multiple of kKeys, at most kMaxSlots)
 };
 
+// Key splits per query. Each CTA pays a fixed pipeline fill (about four tiles' time: Q staging and
+// the first gather) and the splits need a merge pass, so the count minimises an estimate in tile
+// units: waves x (tiles per CTA + fill) + merge, with waves = ceil(CTAs / SMs).
 MlaSplit choose_split(int64_t BT, int k, int sms) {
-  MlaSplit s;
-  const int64_t ctas_per_split = BT * 2;
-  int n = (int)std::max<int64_t>(1, (sms + ctas_per_split - 1) / ctas_per_split);
-  const int max_split = std::max(1, (k + 63) / 64);
-  n = std::min(n, max_split);
-  int chunk = (k + n - 1) / n;
-  chunk = (chunk + 63) / 64 * 64;
-  chunk = std::min(chunk, kMaxSlots);
-  s.chunk = chunk;
-  s.nsplit = (k + chunk - 1) / chunk;
-  return s;
+  constexpr double kFillTiles = 4.0, kMergeTiles = 2.0;
+  constexpr double kMergeTilesPerMB = 0.15;          // partials written + read, ~1.2 us per tile at HBM rate
+  const int n_min = (k + kMaxSlots - 1) / kMaxSlots;  // a split holds at most kMaxSlots slots
+  const int n_max = std::min((k + kKeys - 1) / kKeys, n_min + 256);
+  MlaSplit best{0, 0};
+  double best_cost = 1e300;
+  for (int n = n_min; n <= n_max; ++n) {
+    int chunk = (k + n - 1) / n;
+    chunk = (chunk + kKeys - 1) / kKeys * kKeys;     // <= kMaxSlots, a multiple of kKeys
+    const int nsplit = (k + chunk - 1) / chunk;
+    const int64_t ctas = BT * 2 * nsplit;
+    const double waves = (double)((ctas + sms - 1) / sms);
+    double cost = waves * (chunk / kKeys + kFillTiles);
+    if (nsplit > 1) cost += kMergeTiles + kMergeTilesPerMB * (double)BT * nsplit * kHeads * kDv * 8 / 1e6;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best.nsplit = nsplit;
+      best.chunk = chunk;
+    }
+  }
+  return best;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {

@@ -56,7 +56,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
 def test_noalloc_rejects_shape_beyond_its_scratch():
     if not torch.cuda.is_available():
         pytest.skip("no GPU")
-    B, k = 73, 2048
+    B, k = 73, 16384                                           # 8+ key splits of 73 queries
     assert dsa.dsa_sparse_mla_workspace_size(B, 1, k) > dsa.dsa_sparse_mla_noalloc_scratch_bytes()
     q = torch.zeros((B, 1, 128, 576), dtype=torch.bfloat16, device="cuda")
     kv = torch.zeros((B, 64, 576), dtype=torch.bfloat16, device="cuda")
