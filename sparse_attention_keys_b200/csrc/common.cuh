@@ -333,6 +333,10 @@ int* status_word();                 // device address of this device's status wo
 int check_launch();                 // DSA_OK or DSA_ERR_CUDA after a launch
 bool aligned16(const void* p);
 int device_sm_count();
+// CTAs of `func` that fit on one SM at once: the least of the shared-memory, register, thread and
+// TMEM-column limits, from the kernel's own attributes (the runtime's occupancy query does not
+// count these kernels' residency correctly). 0 if the attributes cannot be read.
+int resident_ctas_per_sm(const void* func, int threads, int dyn_smem, int tmem_cols);
 bool encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, void* base,
                           uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
                           uint32_t box_outer, CUtensorMapSwizzle swizzle);

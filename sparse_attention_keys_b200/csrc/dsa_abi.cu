@@ -107,6 +107,26 @@ int device_sm_count() {
   return (c && c->sms > 0) ? c->sms : 148;
 }
 
+int resident_ctas_per_sm(const void* func, int threads, int dyn_smem, int tmem_cols) {
+  cudaFuncAttributes a;
+  int dev = 0, smem_sm = 0, regs_sm = 0, threads_sm = 0, blocks_sm = 0, reserved = 0;
+  if (cudaFuncGetAttributes(&a, func) != cudaSuccess || cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&threads_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&blocks_sm, cudaDevAttrMaxBlocksPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
+    return 0;
+  const int warps = (threads + 31) / 32;
+  const int regs_cta = ((a.numRegs + 7) / 8 * 8) * 32 * warps;      // registers are allocated per warp, 8 at a time
+  int n = blocks_sm;
+  n = std::min(n, smem_sm / std::max(1, dyn_smem + (int)a.sharedSizeBytes + reserved));
+  n = std::min(n, regs_sm / std::max(1, regs_cta));
+  n = std::min(n, threads_sm / std::max(1, warps * 32));
+  if (tmem_cols > 0) n = std::min(n, 512 / tmem_cols);
+  return std::max(n, 0);
+}
+
 bool encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, void* base, uint64_t inner,
                           uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                           CUtensorMapSwizzle swizzle) {

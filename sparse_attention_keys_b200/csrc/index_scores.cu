@@ -10,11 +10,14 @@
 // Each TMEM lane then holds one key and its N (query, head) dot products, so the ReLU and the
 // weighted head-sum are an in-thread reduction over TMEM columns and the [T, 64, S] tensor of
 // per-head products never leaves the SM. The CTA keeps its NQ queries resident and streams
-// 16 KB key tiles through a TMA ring (one warp), one thread issues the MMAs into two TMEM
-// accumulators (ping-pong), and sixteen epilogue warps (four per TMEM lane quadrant, one query each)
+// 16 KB key tiles through a TMA ring (one warp), one thread issues the MMAs into a ring of TMEM
+// accumulators (two of 256 columns with four queries, four of 64 with one), and the epilogue warps
+// (four per TMEM lane quadrant with four queries, one query each)
 // drain TMEM while the next tile multiplies; each thread keeps eight independent partial sums so the
 // head-sum is not one serial FMA chain.
 // Key tiles above the causal diagonal of the CTA's queries are never loaded.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -32,8 +35,9 @@ template <int NQ>
 struct ScoresCfg {
   static constexpr int N = NQ * 64;                 // MMA N: (query, head) columns
   static constexpr int kStages = NQ >= 4 ? 6 : 4;
+  static constexpr int kAcc = NQ >= 4 ? 2 : 4;      // TMEM accumulators (ring)
   static constexpr int kQBytes = N * 128;
-  static constexpr int kTmemCols = 2 * N;           // two accumulators
+  static constexpr int kTmemCols = kAcc * N;
   static constexpr int kSmemBytes = 1024 /*align slack*/ + kQBytes + kStages * kTileBytes + 1024;
 };
 
@@ -73,9 +77,10 @@ __global__ void __launch_bounds__(threads_for(NQ), 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(k_smem + STAGES * kTileBytes);
   uint64_t* full = bars;                                    // [STAGES] TMA -> MMA
   uint64_t* empty = bars + STAGES;                          // [STAGES] MMA -> TMA
-  uint64_t* acc_full = bars + 2 * STAGES;                   // [2]      MMA -> epilogue
-  uint64_t* acc_empty = bars + 2 * STAGES + 2;              // [2]      epilogue -> MMA
-  uint64_t* q_full = bars + 2 * STAGES + 4;
+  constexpr int kAcc = Cfg::kAcc;
+  uint64_t* acc_full = bars + 2 * STAGES;                   // [kAcc]   MMA -> epilogue
+  uint64_t* acc_empty = acc_full + kAcc;                    // [kAcc]   epilogue -> MMA
+  uint64_t* q_full = acc_empty + kAcc;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
   __shared__ __align__(16) float wq[NQ][64];
@@ -93,7 +98,7 @@ __global__ void __launch_bounds__(threads_for(NQ), 1)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], kEpiWarps * 32); }
+    for (int a = 0; a < kAcc; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], kEpiWarps * 32); }
     mbar_init(q_full, 1);
     fence_barrier_init();
   }
@@ -153,8 +158,8 @@ __global__ void __launch_bounds__(threads_for(NQ), 1)
       const uint32_t q_addr = smem_u32(q_smem);
       bool ok = mbar_wait(q_full, 0, &abort_flag, p.status, DSA_SITE_SCORES_Q);
       for (int i = 0; ok && i < my_tiles; ++i) {
-        const int s = i % STAGES, a = i & 1;
-        if (i >= 2 && !mbar_wait(&acc_empty[a], ((i >> 1) + 1) & 1, &abort_flag, p.status, DSA_SITE_SCORES_ACC_EMPTY)) break;
+        const int s = i % STAGES, a = i % kAcc;
+        if (i >= kAcc && !mbar_wait(&acc_empty[a], ((i / kAcc) + 1) & 1, &abort_flag, p.status, DSA_SITE_SCORES_ACC_EMPTY)) break;
         if (!mbar_wait(&full[s], (i / STAGES) & 1, &abort_flag, p.status, DSA_SITE_SCORES_K_FULL)) break;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(k_smem + s * kTileBytes);
@@ -176,13 +181,20 @@ __global__ void __launch_bounds__(threads_for(NQ), 1)
     const int q_lo = warp >> 2;
     const bool active = q_lo < NQ;                     // NQ = 1: one warp per quadrant
     const int row_in_tile = quad * 32 + lane;          // TMEM lane = key within the tile
+    const float* ks_row = p.k_scale + (int64_t)b * p.S_max;
+    auto load_ks = [&](int i) -> float {               // k_scale of this thread's key in tile i
+      const int key = (kt_begin + i) * kKeysPerTile + row_in_tile;
+      return (active && i < my_tiles && key < p.S_max) ? __ldg(ks_row + key) : 0.f;
+    };
+    float ks_next = load_ks(0);
     for (int i = 0; i < my_tiles; ++i) {
-      const int a = i & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[a], (i >> 1) & 1, &abort_flag, p.status, DSA_SITE_SCORES_ACC_FULL))) break;
+      const int a = i % kAcc;
+      const float ks = ks_next;
+      ks_next = load_ks(i + 1);                        // one tile ahead
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[a], (i / kAcc) & 1, &abort_flag, p.status, DSA_SITE_SCORES_ACC_FULL))) break;
       tc_fence_after();
       if (active) {
         const int key = (kt_begin + i) * kKeysPerTile + row_in_tile;
-        const float ks = key < p.S_max ? p.k_scale[(int64_t)b * p.S_max + key] : 0.f;
 #pragma unroll
         for (int qq = 0; qq < QPW; ++qq) {
           const int q = q_lo + qq;
@@ -255,23 +267,34 @@ static int launch_scores_nq(const uint8_t* q8, const uint8_t* k8, const ScoresPa
   p.groups = (base.T + NQ - 1) / NQ;
   const int tiles_max = (base.S_max + kKeysPerTile - 1) / kKeysPerTile;
   const int64_t units = (int64_t)base.B * p.groups;
-  const int target = 4 * dsa_host::device_sm_count();
-  int ksplit = (int)((target + units - 1) / units);
+  // one wave: as many CTAs as fit on the device at once (key splits share a query group's tiles)
+  static int occupancy[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && occupancy[dev] == 0) {
+    // all of the unified L1 / shared storage as shared memory, so that as many CTAs as the shared
+    // memory allows are resident
+    if (cudaFuncSetAttribute(index_scores_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(index_scores_kernel<NQ>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    const int per_sm = dsa_host::resident_ctas_per_sm((const void*)index_scores_kernel<NQ>, threads_for(NQ),
+                                                      Cfg::kSmemBytes, Cfg::kTmemCols);
+    if (per_sm < 1) return DSA_ERR_CUDA;
+    occupancy[dev] = per_sm;
+  }
+  const int64_t target = (int64_t)(dev < 64 ? occupancy[dev] : 1) * dsa_host::device_sm_count();
+  int ksplit = (int)std::max<int64_t>(1, target / units);
   ksplit = max(1, min(ksplit, tiles_max));
   p.ksplit = ksplit;
   p.tiles_per_split = (tiles_max + ksplit - 1) / ksplit;
   p.ksplit = (tiles_max + p.tiles_per_split - 1) / p.tiles_per_split;
   const int64_t grid = units * p.ksplit;
   if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;
-  static bool configured[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
-    if (cudaFuncSetAttribute(index_scores_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::kSmemBytes) != cudaSuccess)
-      return DSA_ERR_CUDA;
-    configured[dev] = true;
-  }
+  if (dev >= 64 && cudaFuncSetAttribute(index_scores_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        Cfg::kSmemBytes) != cudaSuccess)
+    return DSA_ERR_CUDA;
   index_scores_kernel<NQ><<<(unsigned)grid, threads_for(NQ), Cfg::kSmemBytes, stream>>>(qmap, kmap, p);
   return dsa_host::check_launch();
 }
