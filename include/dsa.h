@@ -12,9 +12,9 @@
  *   [rope]    "DeepSeek-V3.2-Exp - RoPE coefficients": YaRN precompute excerpt, ModelArgs.
  *   [dense]   "DeepSeek-V3.2-Exp - Dense transformer block, Sparse latent attention": the
  *             43-step equation list (indexer steps, sparse attention steps, m = 1 + 0.1 ln 40).
- *   [rotate]  "DeepSeek-V3.2-Exp - Rotate first features": Indexer.forward (model.py 457-487),
- *             apply_rotary_emb (model.py 405-425).
- *   [sim]     "DeepSeek-V3.2-Exp - Similarities": absorbed MQA decode (model.py 590-606).
+ *   [rotate]  "DeepSeek-V3.2-Exp - Rotate first features": Indexer.forward excerpt,
+ *             apply_rotary_emb excerpt.
+ *   [sim]     "DeepSeek-V3.2-Exp - Similarities": absorbed MQA decode excerpt.
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers unless a comment says "host". The caller owns

@@ -13,16 +13,16 @@ the fp32 block scales). Every function cites the page passage it restates:
   64 heads, ReLU instead of softmax, block-wise FP8 quantisation with 128-element
   blocks, and the non-interleaved indexer RoPE notice.
 * "DeepSeek-V3.2-Exp - RoPE coefficients" (atlas page, block-rotations): the YaRN
-  frequency code (model.py 334-402 excerpt) and the ModelArgs defaults.
+  frequency code (precompute excerpt) and the ModelArgs defaults.
 * "DeepSeek-V3.2-Exp - Dense transformer block / Sparse latent attention" (atlas
   page, dense-blocks): the lightning-indexer steps (RoPE_64, (1/sqrt 128) H_128,
   S^I = 1/(sqrt64 sqrt128) sum_h w ReLU(.), top-2048 with the causal mask) and the
   sparse-attention steps (S' = S m^2/sqrt(192), m = 1 + 0.1 ln 40, softmax, O = AV);
-  the MLA prefill excerpt (model.py 574-589).
+  the MLA prefill excerpt.
 * "DeepSeek-V3.2-Exp - Rotate first features" (atlas page, index-keys/rotate):
-  Indexer.forward (model.py 457-487) and apply_rotary_emb (model.py 405-425).
+  Indexer.forward excerpt and apply_rotary_emb excerpt.
 * "DeepSeek-V3.2-Exp - Similarities" (atlas page, attend/weights/similarities):
-  the absorbed MQA decode (model.py 590-606) and the p+1 visible keys at p=1000.
+  the absorbed MQA decode excerpt and the p+1 visible keys at p=1000.
 
 Readings where the pages are silent or garbled are marked READING.
 Pins for every function live in tests/test_oracle_pins.py.

@@ -1,7 +1,7 @@
 // dsa_index_keys: indexer query/key transform and block FP8 quantisation.
 //
 // Restates, per 128-feature head row, the steps of Indexer.forward ("DeepSeek-V3.2-Exp - Rotate
-// first features", model.py 457-487 excerpt): non-interleaved RoPE on the first 64 features
+// first features", Indexer.forward excerpt): non-interleaved RoPE on the first 64 features
 // (feature j pairs with j+32, apply_rotary_emb with interleaved=False), rotate_activation
 // ((1/sqrt 128) H_128, dense-block page indexer steps), act_quant with 128-element blocks
 // (news page), and the k_cache / k_scale_cache write.

@@ -3,7 +3,7 @@
 // Computes I[b,t,s] = k_scale[b,s] * sum_j w'[b,t,j] * ReLU(q8[b,t,j,:] . k8[b,s,:]) for every
 // visible s (s <= q_pos, s < kv_len), w' = w * 64^-0.5 * q_scale * softmax_scale: the fp8_index
 // call and weight fold of Indexer.forward ("DeepSeek-V3.2-Exp - Rotate first features",
-// model.py 457-487 excerpt) and S^I of the lightning-indexer steps (dense-block page).
+// Indexer.forward excerpt) and S^I of the lightning-indexer steps (dense-block page).
 //
 // Tile: the MMA's M = 128 keys (A = K-cache rows, K-major, 128 B each = one 128B-swizzle atom
 // row), N = NQ queries x 64 heads (B = the queries' FP8 head rows), K = 128 (4 MMAs of K=32).

@@ -2,7 +2,7 @@
 //
 // For each (b, t, head h): z_u = scale * q[h] . kv[idx_u] over the 576 features (512 latent +
 // 64 rotary), p = softmax over the selected u, out[h] = sum_u p_u kv[idx_u][0:512]. This is the
-// absorbed MQA decode of "DeepSeek-V3.2-Exp - Similarities" (model.py 590-606 excerpt: latent and
+// absorbed MQA decode of "DeepSeek-V3.2-Exp - Similarities" (absorbed MQA decode excerpt: latent and
 // rotary score terms, index mask, softmax, latent-weighted sum) with the index mask replaced by a
 // gather of the selected rows, and the sparse-attention steps of the dense-block page
 // (S' = S m^2/sqrt 192, A = softmax, O = AV).

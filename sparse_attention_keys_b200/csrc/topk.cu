@@ -1,7 +1,7 @@
 // dsa_topk: per-query top-k of the index scores over the visible (causal) positions.
 //
 // Restates index_score.topk(min(index_topk, end_pos)) after the mask add in Indexer.forward
-// ("DeepSeek-V3.2-Exp - Rotate first features", model.py 457-487 excerpt) and top_2048 of the
+// ("DeepSeek-V3.2-Exp - Rotate first features", Indexer.forward excerpt) and top_2048 of the
 // lightning-indexer steps (dense-block page). Ties go to the smaller position; the selection
 // is written in ascending position order, then -1 padding.
 //
