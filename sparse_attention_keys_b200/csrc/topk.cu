@@ -6,10 +6,10 @@
 // is written in ascending position order, then -1 padding.
 //
 // One CTA per score row. The row's visible scores are staged once into shared memory as
-// order-preserving 32-bit keys (coalesced 16-byte loads), then a 3-pass radix select (12, 10,
-// 10 bits) finds the k-th largest key with shared-memory histograms, and a warp-ballot
-// compaction writes the selected positions in order. HBM-bound: 4 B read per visible score,
-// 4 B written per selected index.
+// order-preserving 32-bit keys (coalesced 16-byte loads, four in flight per thread); a 3-pass
+// radix select (12, 10, 10 bits) finds the k-th largest key with shared-memory histograms, and a
+// compaction (four keys per lane, warp shuffle scans of the per-lane counts) writes the selected
+// positions in order. HBM-bound: 4 B read per visible score, 4 B written per selected index.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -53,9 +53,13 @@ __device__ __forceinline__ uint32_t block_inclusive_scan(uint32_t v, uint32_t* w
   return v + before;
 }
 
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
+  if (active) atomicAdd(&hist[bin], 1u);
+}
+
 }  // namespace
 
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restrict__ scores,
+__global__ void __launch_bounds__(kTopkThreads, 4) topk_kernel(const float* __restrict__ scores,
                                                             int64_t ld,
                                                             const int32_t* __restrict__ q_pos,
                                                             const int32_t* __restrict__ kv_len,
@@ -85,14 +89,30 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
     return;
   }
 
-  // Stage the visible scores as keys.
+  // Stage the visible scores as keys (zero-padded to a multiple of four).
   const float* src = scores + row * ld;
   const int n4 = n >> 2;
-  for (int i = tid; i < n4; i += kTopkThreads) {
-    const float4 f = reinterpret_cast<const float4*>(src)[i];
-    reinterpret_cast<uint4*>(keys)[i] = make_uint4(order_key(f.x), order_key(f.y), order_key(f.z), order_key(f.w));
+  constexpr int kInFlight = 4;                 // float4 loads issued before any is used
+  for (int i0 = 0; i0 < n4; i0 += kInFlight * kTopkThreads) {
+    float4 f[kInFlight];
+#pragma unroll
+    for (int u = 0; u < kInFlight; ++u) {
+      const int i = i0 + u * kTopkThreads + tid;
+      if (i < n4) f[u] = reinterpret_cast<const float4*>(src)[i];
+    }
+#pragma unroll
+    for (int u = 0; u < kInFlight; ++u) {
+      const int i = i0 + u * kTopkThreads + tid;
+      if (i < n4)
+        reinterpret_cast<uint4*>(keys)[i] =
+            make_uint4(order_key(f[u].x), order_key(f[u].y), order_key(f[u].z), order_key(f[u].w));
+    }
   }
-  for (int i = (n4 << 2) + tid; i < n; i += kTopkThreads) keys[i] = order_key(src[i]);
+  if (tid < 4 && (n4 << 2) + tid < ((n + 3) & ~3)) {   // the n % 4 tail
+    const int i = (n4 << 2) + tid;
+    keys[i] = i < n ? order_key(src[i]) : 0u;
+  }
+  __syncthreads();
 
   // Radix select of the k-th largest key: digits of 12, 10 and 10 bits from the top.
   uint32_t prefix = 0, prefix_mask = 0, remaining = (uint32_t)k;
@@ -100,11 +120,18 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
   for (int pass = 0; pass < 3; ++pass) {
     const int shift = pass == 0 ? 20 : (pass == 1 ? 10 : 0);
     const int nb = pass == 0 ? 4096 : 1024;
-    for (int i = tid; i < nb; i += kTopkThreads) hist[i] = 0;
-    __syncthreads();
-    for (int i = tid; i < n; i += kTopkThreads) {
-      const uint32_t key = keys[i];
-      if ((key & prefix_mask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+    {
+      for (int i = tid; i < nb; i += kTopkThreads) hist[i] = 0;
+      __syncthreads();
+      // four keys per thread per step (the keys array is zero-padded to a multiple of four)
+      for (int i4 = tid; 4 * i4 < n; i4 += kTopkThreads) {
+        const uint4 kk = reinterpret_cast<const uint4*>(keys)[i4];
+        const int i = 4 * i4;
+        hist_add(hist, (kk.x >> shift) & (nb - 1), (kk.x & prefix_mask) == prefix);
+        hist_add(hist, (kk.y >> shift) & (nb - 1), i + 1 < n && (kk.y & prefix_mask) == prefix);
+        hist_add(hist, (kk.z >> shift) & (nb - 1), i + 2 < n && (kk.z & prefix_mask) == prefix);
+        hist_add(hist, (kk.w >> shift) & (nb - 1), i + 3 < n && (kk.w & prefix_mask) == prefix);
+      }
     }
     __syncthreads();
     // thread t owns bins nb-1-t*c .. nb-(t+1)*c (descending); c = nb / threads
@@ -134,16 +161,37 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
   const uint32_t thr = prefix;           // the k-th largest key
   const uint32_t need_eq = remaining;    // how many keys equal to thr are selected
 
-  // Compaction in ascending position order. Warp w owns a contiguous chunk.
+  // Compaction in ascending position order. Warp w owns a contiguous chunk of whole 128-key steps;
+  // in each step lane l holds keys 4l..4l+3 (one 16-byte shared-memory load).
   const int warp = tid >> 5, lane = tid & 31;
-  const int chunk = ((n + kTopkWarps - 1) / kTopkWarps + 31) & ~31;
-  const int beg = min(n, warp * chunk), end = min(n, beg + chunk);
+  const int steps = (n + 127) / 128;
+  const int per_warp = (steps + kTopkWarps - 1) / kTopkWarps;
+  const int s_beg = min(steps, warp * per_warp), s_end = min(steps, s_beg + per_warp);
+  auto classify = [&](int st, uint32_t& gt4, uint32_t& eq4) {   // 4-bit masks of keys > thr, == thr
+    const int i = st * 128 + 4 * lane;
+    gt4 = 0; eq4 = 0;
+    if (i < n) {
+      const uint4 kk = reinterpret_cast<const uint4*>(keys)[i >> 2];
+      const uint32_t v[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const bool in = i + u < n;
+        gt4 |= (uint32_t)(in && v[u] > thr) << u;
+        eq4 |= (uint32_t)(in && v[u] == thr) << u;
+      }
+    }
+  };
   uint32_t n_gt = 0, n_eq = 0;
-  for (int base = beg; base < end; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = i < end ? keys[i] : 0;
-    n_gt += __popc(__ballot_sync(0xffffffffu, i < end && key > thr));
-    n_eq += __popc(__ballot_sync(0xffffffffu, i < end && key == thr));
+  for (int st = s_beg; st < s_end; ++st) {
+    uint32_t g4, e4;
+    classify(st, g4, e4);
+    n_gt += __popc(g4);
+    n_eq += __popc(e4);
+  }
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) {
+    n_gt += __shfl_xor_sync(0xffffffffu, n_gt, d);
+    n_eq += __shfl_xor_sync(0xffffffffu, n_eq, d);
   }
   // exclusive offsets across warps (lane 0 of each warp contributes its counts)
   __shared__ uint32_t gt_off[kTopkWarps], eq_off[kTopkWarps];
@@ -159,20 +207,31 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
   }
   __syncthreads();
   uint32_t gt_seen = gt_off[warp], eq_seen = eq_off[warp];
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int base = beg; base < end; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = i < end ? keys[i] : 0;
-    const bool gt = i < end && key > thr;
-    const bool eq = i < end && key == thr;
-    const uint32_t mg = __ballot_sync(0xffffffffu, gt);
-    const uint32_t me = __ballot_sync(0xffffffffu, eq);
-    const uint32_t g_before = gt_seen + __popc(mg & lt_mask);
-    const uint32_t e_before = eq_seen + __popc(me & lt_mask);
-    if (gt) out[g_before + min(e_before, need_eq)] = i;
-    else if (eq && e_before < need_eq) out[g_before + e_before] = i;
-    gt_seen += __popc(mg);
-    eq_seen += __popc(me);
+  for (int st = s_beg; st < s_end; ++st) {
+    uint32_t g4, e4;
+    classify(st, g4, e4);
+    // exclusive prefix of the per-lane counts (lane order = position order)
+    uint32_t gi = __popc(g4), ei = __popc(e4);
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint32_t og = __shfl_up_sync(0xffffffffu, gi, d), oe = __shfl_up_sync(0xffffffffu, ei, d);
+      if (lane >= d) { gi += og; ei += oe; }
+    }
+    const uint32_t g_tot = __shfl_sync(0xffffffffu, gi, 31), e_tot = __shfl_sync(0xffffffffu, ei, 31);
+    uint32_t g_before = gt_seen + gi - __popc(g4), e_before = eq_seen + ei - __popc(e4);
+    const int i = st * 128 + 4 * lane;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if ((g4 >> u) & 1u) {
+        out[g_before + min(e_before, need_eq)] = i + u;
+        ++g_before;
+      } else if ((e4 >> u) & 1u) {
+        if (e_before < need_eq) out[g_before + e_before] = i + u;
+        ++e_before;
+      }
+    }
+    gt_seen += g_tot;
+    eq_seen += e_tot;
   }
 }
 
