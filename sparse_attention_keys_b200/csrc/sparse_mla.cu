@@ -36,7 +36,7 @@
 // operand of P V (N = features).
 // Per CTA: 4 softmax warps (thread = head = TMEM lane), 1 P V warp, 4 gather warps (the first also
 // loads Q features 320..575 by TMA), 3 Q K^T warps. The running max is only moved (and O rescaled in
-// TMEM) when it grows by more than 2^8. With several key splits per query, fp32 partials (O, max,
+// TMEM) when it grows by more than 2^32. With several key splits per query, fp32 partials (O, max,
 // sum) go to the caller's workspace and a second kernel merges them.
 #include <cuda_bf16.h>
 #include <math.h>
@@ -75,7 +75,11 @@ constexpr int kMaxSlots = 2048;                    // selected slots per CTA (sp
 constexpr int kTmemCols = 512;
 constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = kTmemS + kSBufs * kKeys;   // S: three 32-column buffers
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleThreshold = 8.0f;          // log2 units
+// The running max moves (and O is rescaled in TMEM, 256 columns per thread) only when a tile's
+// max exceeds it by more than 2^32: P then stays below 2^32 (bf16 keeps its relative precision at
+// any magnitude), l below 2^43 and O far from the fp32 range, and a rescale, which stalls the
+// warp that does it while the other softmax warps wait at the next barrier, becomes rare.
+constexpr float kRescaleThreshold = 32.0f;         // log2 units
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 static_assert(kTmemQ + kQTmemRegions * 32 == kTmemCols, "TMEM budget");
 static_assert(kTmemQ <= kTmemCols, "TMEM budget");
