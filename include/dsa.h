@@ -65,10 +65,15 @@ typedef struct CUstream_st* dsa_stream_t; /* a cudaStream_t */
 #define DSA_MLA_QK 576          /* latent + rotary key width */
 #define DSA_MAX_POS 1048576     /* positions accepted by dsa_rope_table / dsa_index_keys */
 #define DSA_TOPK_MAX_ROW 32768  /* longest score row dsa_topk accepts (kept in shared memory) */
+#define DSA_TOPK_SORT_MAX 4096  /* largest k with DSA_SORTED                                    */
 
 /* Flags */
 #define DSA_HADAMARD 0x1u      /* dsa_index_keys: apply (1/sqrt 128) H_128 after RoPE ([dense]
                                   indexer steps; rotate_activation in Indexer.forward)         */
+#define DSA_SORTED 0x4u        /* dsa_topk: order the selection by descending score, ties by
+                                  ascending position (default: ascending position)           */
+#define DSA_F32 0              /* dsa_index_keys input element types                           */
+#define DSA_BF16 1
 #define DSA_FILL_MASKED 0x2u   /* dsa_index_scores: write -inf at masked (s > pos) entries of
                                   each row up to S_max (the mask add of Indexer.forward)       */
 
@@ -88,7 +93,8 @@ DSA_API int dsa_rope_table(float* table, int max_pos);
  * ([rotate] Indexer.forward: RoPE on q_pe/k_pe with interleaved=False, rotate_activation,
  * act_quant, k_cache / k_scale_cache write; [news] 128-element blocks).
  *
- *   x        fp32 [rows][heads][128]   rows = tokens; heads = 64 for queries, 1 for keys
+ *   x        [rows][heads][128] of x_dtype: DSA_F32 (fp32) or DSA_BF16 (bf16 bit patterns,
+ *            widened exactly to fp32); rows = tokens; heads = 64 for queries, 1 for keys
  *   pos      int32 [rows]              absolute position of each row (0 <= pos < max_pos)
  *   rope_cs  fp32 [max_pos][32][2]     table from dsa_rope_table (copied to the device)
  *   flags    DSA_HADAMARD or 0
@@ -104,7 +110,7 @@ DSA_API int dsa_rope_table(float* table, int max_pos);
  * the IEEE fp32 quotient y / scale.
  * A pos outside [0, max_pos) sets DSA_ERR_DEVICE_BOUNDS and leaves that row unwritten.
  */
-DSA_API int dsa_index_keys(const float* x, int64_t rows, int heads, const int32_t* pos,
+DSA_API int dsa_index_keys(const void* x, int x_dtype, int64_t rows, int heads, const int32_t* pos,
                    const float* rope_cs, int max_pos, uint32_t flags,
                    uint8_t* out_fp8, float* out_scale, const int64_t* dst_row,
                    dsa_stream_t stream);
@@ -138,12 +144,14 @@ DSA_API int dsa_index_scores(const uint8_t* q8, const float* q_scale, const floa
  * top_2048). n_valid = min(q_pos+1, kv_len). Only visible entries of `scores` are read.
  *
  *   scores fp32 [B][T][ld];  idx int32 [B][T][k] (output)
- * Ties go to the smaller position. The selected positions are written in ascending order,
- * then -1 up to k. NaN scores are not allowed. -0.0 and +0.0 compare equal.
+ * Ties go to the smaller position. The selected positions are written in ascending order, or
+ * with flags = DSA_SORTED by descending score (equal scores by ascending position), then -1 up
+ * to k. NaN scores are not allowed. -0.0 and +0.0 compare equal.
+ * DSA_SORTED needs k <= DSA_TOPK_SORT_MAX (it sorts the selection in shared memory).
  * Constraints: 1 <= k; every row's n_valid <= DSA_TOPK_MAX_ROW (ld may be larger).
  */
 DSA_API int dsa_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int32_t* kv_len,
-             int B, int T, int k, int32_t* idx, dsa_stream_t stream);
+             int B, int T, int k, uint32_t flags, int32_t* idx, dsa_stream_t stream);
 
 /*
  * dsa_sparse_mla - sparse MQA-style latent attention over the selected positions

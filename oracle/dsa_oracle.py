@@ -284,12 +284,13 @@ def index_score_magnitude(q8, q_scale, w, k8, k_scale, q_pos, kv_len,
     return out
 
 
-def topk_indices(scores, q_pos, kv_len, k: int) -> np.ndarray:
+def topk_indices(scores, q_pos, kv_len, k: int, sorted_by_score: bool = False) -> np.ndarray:
     """Per query, the min(k, n_valid) visible positions with the largest scores
     (index_score.topk(min(index_topk, end_pos)) after the causal mask).
 
     READING: equal scores go to the smaller position; the selected positions are written in
-    ascending order, followed by -1 padding. int32 [B, T, k].
+    ascending order (or, with sorted_by_score, in the order of the stable sort by descending
+    score), followed by -1 padding. int32 [B, T, k].
     """
     scores = np.asarray(scores)
     B, T, _ = scores.shape
@@ -302,7 +303,7 @@ def topk_indices(scores, q_pos, kv_len, k: int) -> np.ndarray:
                 continue
             row = scores[b, t, :n]
             order = np.lexsort((np.arange(n), -row))     # by score desc, then position asc
-            sel = np.sort(order[:min(k, n)])
+            sel = order[:min(k, n)] if sorted_by_score else np.sort(order[:min(k, n)])
             out[b, t, :sel.size] = sel
     return out
 

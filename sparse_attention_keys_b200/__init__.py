@@ -13,7 +13,7 @@ import os
 import torch
 
 __all__ = [
-    "DsaError", "lib", "lib_path", "DSA_HADAMARD", "DSA_FILL_MASKED", "INDEXER_SOFTMAX_SCALE",
+    "DsaError", "lib", "lib_path", "DSA_HADAMARD", "DSA_FILL_MASKED", "DSA_SORTED", "DSA_F32", "DSA_BF16", "INDEXER_SOFTMAX_SCALE",
     "MLA_SOFTMAX_SCALE", "dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk",
     "dsa_sparse_mla", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_noalloc",
     "dsa_sparse_mla_noalloc_scratch_bytes", "dsa_get_device_status", "dsa_get_error_detail",
@@ -24,6 +24,9 @@ __all__ = [
 DSA_OK = 0
 DSA_HADAMARD = 0x1
 DSA_FILL_MASKED = 0x2
+DSA_SORTED = 0x4
+DSA_F32 = 0
+DSA_BF16 = 1
 MAX_POS = 16384                 # max_seq_len of the model (ModelArgs)
 INDEXER_SOFTMAX_SCALE = 128 ** -0.5
 MLA_SOFTMAX_SCALE = 192 ** -0.5 * (1.0 + 0.1 * __import__("math").log(40.0)) ** 2
@@ -53,9 +56,9 @@ def _load():
     vp, i32, i64, u32, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint32,
                                   ctypes.c_float, ctypes.c_size_t)
     L.dsa_rope_table.argtypes = [vp, i32]
-    L.dsa_index_keys.argtypes = [vp, i64, i32, vp, vp, i32, u32, vp, vp, vp, vp]
+    L.dsa_index_keys.argtypes = [vp, i32, i64, i32, vp, vp, i32, u32, vp, vp, vp, vp]
     L.dsa_index_scores.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, f32, vp, i64, u32, vp]
-    L.dsa_topk.argtypes = [vp, i64, vp, vp, i32, i32, i32, vp, vp]
+    L.dsa_topk.argtypes = [vp, i64, vp, vp, i32, i32, i32, u32, vp, vp]
     L.dsa_sparse_mla.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
     L.dsa_sparse_mla_workspace_size.argtypes = [i32, i32, i32]
     L.dsa_sparse_mla_workspace_size.restype = sz
@@ -127,11 +130,13 @@ def dsa_rope_table(max_pos: int = MAX_POS) -> torch.Tensor:
 
 def dsa_index_keys(x, pos, rope_cs, flags: int = DSA_HADAMARD, out_fp8=None, out_scale=None,
                    dst_row=None, stream=None):
-    """x fp32 [rows, heads, 128] (or [rows, 128] for keys) -> (codes uint8, scales fp32).
+    """x fp32 or bf16 [rows, heads, 128] (or [rows, 128] for keys) -> (codes uint8, scales fp32).
 
     With dst_row (int64 [rows]) the outputs are written into the given cache tensors at those rows.
     """
-    _need(x, torch.float32, "x")
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("x must be float32 or bfloat16")
+    _need(x, x.dtype, "x")
     _need(pos, torch.int32, "pos")
     _need(rope_cs, torch.float32, "rope_cs")
     if x.shape[-1] != 128:
@@ -151,7 +156,8 @@ def dsa_index_keys(x, pos, rope_cs, flags: int = DSA_HADAMARD, out_fp8=None, out
             raise ValueError("dst_row needs the destination out_fp8 and out_scale tensors")
     _need(out_fp8, torch.uint8, "out_fp8")
     _need(out_scale, torch.float32, "out_scale")
-    rc = _lib.dsa_index_keys(_ptr(x), rows, heads, _ptr(pos), _ptr(rope_cs), rope_cs.shape[0], int(flags),
+    x_dtype = DSA_BF16 if x.dtype == torch.bfloat16 else DSA_F32
+    rc = _lib.dsa_index_keys(_ptr(x), x_dtype, rows, heads, _ptr(pos), _ptr(rope_cs), rope_cs.shape[0], int(flags),
                              _ptr(out_fp8), _ptr(out_scale), _ptr(dst_row), _stream(stream))
     _check(rc, "dsa_index_keys")
     return out_fp8, out_scale
@@ -179,8 +185,9 @@ def dsa_index_scores(q8, q_scale, w, k8, k_scale, q_pos, kv_len, softmax_scale: 
     return scores
 
 
-def dsa_topk(scores, q_pos, kv_len, k: int, idx=None, stream=None):
-    """scores fp32 [B,T,ld] -> idx int32 [B,T,k] (ascending positions, -1 padded)."""
+def dsa_topk(scores, q_pos, kv_len, k: int, idx=None, flags: int = 0, stream=None):
+    """scores fp32 [B,T,ld] -> idx int32 [B,T,k] (ascending positions, or by descending score with
+    flags=DSA_SORTED; -1 padded)."""
     _need(scores, torch.float32, "scores")
     _need(q_pos, torch.int32, "q_pos")
     _need(kv_len, torch.int32, "kv_len")
@@ -188,7 +195,8 @@ def dsa_topk(scores, q_pos, kv_len, k: int, idx=None, stream=None):
     if idx is None:
         idx = torch.empty((B, T, k), dtype=torch.int32, device=scores.device)
     _need(idx, torch.int32, "idx")
-    rc = _lib.dsa_topk(_ptr(scores), int(ld), _ptr(q_pos), _ptr(kv_len), B, T, int(k), _ptr(idx), _stream(stream))
+    rc = _lib.dsa_topk(_ptr(scores), int(ld), _ptr(q_pos), _ptr(kv_len), B, T, int(k), int(flags), _ptr(idx),
+                       _stream(stream))
     _check(rc, "dsa_topk")
     return idx
 

@@ -191,11 +191,11 @@ int dsa_rope_table(float* table, int max_pos) {
   return DSA_OK;
 }
 
-int dsa_index_keys(const float* x, int64_t rows, int heads, const int32_t* pos, const float* rope_cs,
+int dsa_index_keys(const void* x, int x_dtype, int64_t rows, int heads, const int32_t* pos, const float* rope_cs,
                    int max_pos, uint32_t flags, uint8_t* out_fp8, float* out_scale,
                    const int64_t* dst_row, dsa_stream_t stream) {
   if (rows < 0 || heads < 1 || heads > 4096 || max_pos < 1 || max_pos > DSA_MAX_POS ||
-      (flags & ~DSA_HADAMARD) != 0)
+      (flags & ~DSA_HADAMARD) != 0 || (x_dtype != DSA_F32 && x_dtype != DSA_BF16))
     return DSA_ERR_INVALID_ARG;
   if (rows == 0) return DSA_OK;
   if (!x || !pos || !rope_cs || !out_fp8 || !out_scale) return DSA_ERR_INVALID_ARG;
@@ -206,7 +206,7 @@ int dsa_index_keys(const float* x, int64_t rows, int heads, const int32_t* pos, 
   int* status;
   int rc = prologue(&status);
   if (rc != DSA_OK) return rc;
-  return dsa::launch_index_keys(x, rows, heads, pos, rope_cs, max_pos, flags, out_fp8, out_scale,
+  return dsa::launch_index_keys(x, x_dtype, rows, heads, pos, rope_cs, max_pos, flags, out_fp8, out_scale,
                                 dst_row, (cudaStream_t)stream, status);
 }
 
@@ -230,8 +230,9 @@ int dsa_index_scores(const uint8_t* q8, const float* q_scale, const float* w, co
 }
 
 int dsa_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int32_t* kv_len, int B, int T,
-             int k, int32_t* idx, dsa_stream_t stream) {
-  if (B < 1 || T < 1 || k < 1 || ld < 1 || (ld & 3) != 0) return DSA_ERR_INVALID_ARG;
+             int k, uint32_t flags, int32_t* idx, dsa_stream_t stream) {
+  if (B < 1 || T < 1 || k < 1 || ld < 1 || (ld & 3) != 0 || (flags & ~DSA_SORTED) != 0) return DSA_ERR_INVALID_ARG;
+  if ((flags & DSA_SORTED) && k > DSA_TOPK_SORT_MAX) return DSA_ERR_INVALID_ARG;
   if ((int64_t)B * T > 0x7fffffffLL) return DSA_ERR_INVALID_ARG;
   if (!scores || !q_pos || !kv_len || !idx) return DSA_ERR_INVALID_ARG;
   if (!dsa_host::aligned16(scores) || !dsa_host::aligned16(q_pos) || !dsa_host::aligned16(kv_len) ||
@@ -240,7 +241,7 @@ int dsa_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int32_
   int* status;
   int rc = prologue(&status);
   if (rc != DSA_OK) return rc;
-  return dsa::launch_topk(scores, ld, q_pos, kv_len, B, T, k, idx, (cudaStream_t)stream, status);
+  return dsa::launch_topk(scores, ld, q_pos, kv_len, B, T, k, flags, idx, (cudaStream_t)stream, status);
 }
 
 size_t dsa_sparse_mla_workspace_size(int B, int T, int k) {

@@ -17,7 +17,22 @@
 
 namespace dsa {
 
-__global__ void __launch_bounds__(256) index_keys_kernel(const float* __restrict__ x, int64_t blocks,
+// Four consecutive features of block `blk` for lane `lane`, widened to fp32 (bf16 widening is exact).
+template <typename In>
+__device__ __forceinline__ float4 load4(const In* __restrict__ x, int64_t blk, int lane);
+template <>
+__device__ __forceinline__ float4 load4<float>(const float* __restrict__ x, int64_t blk, int lane) {
+  return reinterpret_cast<const float4*>(x + blk * 128)[lane];
+}
+template <>
+__device__ __forceinline__ float4 load4<uint16_t>(const uint16_t* __restrict__ x, int64_t blk, int lane) {
+  const uint2 u = reinterpret_cast<const uint2*>(x + blk * 128)[lane];
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u), __uint_as_float(u.y << 16),
+                     __uint_as_float(u.y & 0xffff0000u));
+}
+
+template <typename In>
+__global__ void __launch_bounds__(256) index_keys_kernel(const In* __restrict__ x, int64_t blocks,
                                                           int heads, const int32_t* __restrict__ pos,
                                                           const float* __restrict__ rope_cs,
                                                           int max_pos, uint32_t flags,
@@ -36,7 +51,7 @@ __global__ void __launch_bounds__(256) index_keys_kernel(const float* __restrict
     return;
   }
 
-  float4 v4 = reinterpret_cast<const float4*>(x + blk * 128)[lane];
+  const float4 v4 = load4<In>(x, blk, lane);
   float v[4] = {v4.x, v4.y, v4.z, v4.w};
 
   // RoPE on features 0..63: lanes 0-7 hold the first halves a_j (j = 4*lane + i), lanes 8-15
@@ -99,16 +114,21 @@ __global__ void __launch_bounds__(256) index_keys_kernel(const float* __restrict
   if (lane == 0) out_scale[out_blk] = scale;
 }
 
-int launch_index_keys(const float* x, int64_t rows, int heads, const int32_t* pos,
+int launch_index_keys(const void* x, int x_dtype, int64_t rows, int heads, const int32_t* pos,
                       const float* rope_cs, int max_pos, uint32_t flags, uint8_t* out_fp8,
                       float* out_scale, const int64_t* dst_row, cudaStream_t stream, int* status) {
   const int64_t blocks = rows * heads;
   if (blocks == 0) return DSA_OK;
   const int warps = 8;
   const int64_t grid = (blocks + warps - 1) / warps;
-  index_keys_kernel<<<(unsigned)grid, warps * 32, 0, stream>>>(x, blocks, heads, pos, rope_cs, max_pos,
-                                                               flags, out_fp8, out_scale, dst_row,
-                                                               status);
+  if (x_dtype == DSA_BF16)
+    index_keys_kernel<uint16_t><<<(unsigned)grid, warps * 32, 0, stream>>>(
+        static_cast<const uint16_t*>(x), blocks, heads, pos, rope_cs, max_pos, flags, out_fp8, out_scale, dst_row,
+        status);
+  else
+    index_keys_kernel<float><<<(unsigned)grid, warps * 32, 0, stream>>>(
+        static_cast<const float*>(x), blocks, heads, pos, rope_cs, max_pos, flags, out_fp8, out_scale, dst_row,
+        status);
   return dsa_host::check_launch();
 }
 

@@ -7,7 +7,7 @@
 
 namespace dsa {
 
-int launch_index_keys(const float* x, int64_t rows, int heads, const int32_t* pos,
+int launch_index_keys(const void* x, int x_dtype, int64_t rows, int heads, const int32_t* pos,
                       const float* rope_cs, int max_pos, uint32_t flags, uint8_t* out_fp8,
                       float* out_scale, const int64_t* dst_row, cudaStream_t stream, int* status);
 
@@ -17,7 +17,7 @@ int launch_index_scores(const uint8_t* q8, const float* q_scale, const float* w,
                         uint32_t flags, cudaStream_t stream, int* status);
 
 int launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int32_t* kv_len, int B,
-                int T, int k, int32_t* idx, cudaStream_t stream, int* status);
+                int T, int k, uint32_t flags, int32_t* idx, cudaStream_t stream, int* status);
 
 size_t sparse_mla_workspace_size(int B, int T, int k);
 int launch_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T,

@@ -3,7 +3,8 @@
 // Restates index_score.topk(min(index_topk, end_pos)) after the mask add in Indexer.forward
 // ("DeepSeek-V3.2-Exp - Rotate first features", Indexer.forward excerpt) and top_2048 of the
 // lightning-indexer steps (dense-block page). Ties go to the smaller position; the selection
-// is written in ascending position order, then -1 padding.
+// is written in ascending position order (with DSA_SORTED: by descending score, equal scores by
+// ascending position, via a bitonic sort in shared memory), then -1 padding.
 //
 // One CTA per score row. The row's visible scores are staged once into shared memory as
 // order-preserving 32-bit keys (coalesced 16-byte loads, four in flight per thread); a 3-pass
@@ -57,6 +58,24 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool acti
   if (active) atomicAdd(&hist[bin], 1u);
 }
 
+// Ascending bitonic sort of buf[0, n) (n a power of two) by the CTA, then out[i] = the position in
+// the low word of buf[i] for i < count, and -1 for count <= i < k.
+__device__ void sort_and_write(uint64_t* buf, int n, int count, int k, int32_t* out) {
+  __syncthreads();
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < (n >> 1); i += kTopkThreads) {
+        const int lo = 2 * stride * (i / stride) + (i % stride), hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const uint64_t a = buf[lo], b = buf[hi];
+        if ((a > b) == up) { buf[lo] = b; buf[hi] = a; }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < k; i += kTopkThreads) out[i] = i < count ? (int32_t)(uint32_t)buf[i] : -1;
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kTopkThreads, 4) topk_kernel(const float* __restrict__ scores,
@@ -64,11 +83,15 @@ __global__ void __launch_bounds__(kTopkThreads, 4) topk_kernel(const float* __re
                                                             const int32_t* __restrict__ q_pos,
                                                             const int32_t* __restrict__ kv_len,
                                                             int T, int k, int max_row,
+                                                            uint32_t flags, int sort_n,
                                                             int32_t* __restrict__ idx,
                                                             int* status) {
   extern __shared__ __align__(16) uint32_t smem[];
   uint32_t* hist = smem;                       // kHistBins
-  uint32_t* keys = smem + kHistBins;           // max_row
+  uint32_t* keys = smem + kHistBins;           // max_row (rounded up to 4)
+  // DSA_SORTED: sort_n (a power of two >= k) 64-bit keys, (~score key) << 32 | position
+  uint64_t* sbuf = reinterpret_cast<uint64_t*>(smem + kHistBins + ((max_row + 3) & ~3));
+  const bool sorted = (flags & DSA_SORTED) != 0;
   __shared__ uint32_t warp_tot[kTopkWarps];
   __shared__ uint32_t sel_digit, sel_remaining;
 
@@ -79,7 +102,7 @@ __global__ void __launch_bounds__(kTopkThreads, 4) topk_kernel(const float* __re
   int n = min(q_pos[row] + 1, kv_len[b]);
   if (n < 0) n = 0;
 
-  if (n <= k) {   // everything visible is selected
+  if (n <= k && !sorted) {   // everything visible is selected
     for (int i = tid; i < k; i += kTopkThreads) out[i] = i < n ? i : -1;
     return;
   }
@@ -113,6 +136,13 @@ __global__ void __launch_bounds__(kTopkThreads, 4) topk_kernel(const float* __re
     keys[i] = i < n ? order_key(src[i]) : 0u;
   }
   __syncthreads();
+
+  if (n <= k) {                               // DSA_SORTED with everything selected
+    for (int i = tid; i < sort_n; i += kTopkThreads)
+      sbuf[i] = i < n ? ((uint64_t)(~keys[i]) << 32) | (uint32_t)i : ~0ull;
+    sort_and_write(sbuf, sort_n, n, k, out);
+    return;
+  }
 
   // Radix select of the k-th largest key: digits of 12, 10 and 10 bits from the top.
   uint32_t prefix = 0, prefix_mask = 0, remaining = (uint32_t)k;
@@ -222,25 +252,38 @@ __global__ void __launch_bounds__(kTopkThreads, 4) topk_kernel(const float* __re
     const int i = st * 128 + 4 * lane;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
+      int slot = -1;
       if ((g4 >> u) & 1u) {
-        out[g_before + min(e_before, need_eq)] = i + u;
+        slot = (int)(g_before + min(e_before, need_eq));
         ++g_before;
       } else if ((e4 >> u) & 1u) {
-        if (e_before < need_eq) out[g_before + e_before] = i + u;
+        if (e_before < need_eq) slot = (int)(g_before + e_before);
         ++e_before;
+      }
+      if (slot >= 0) {
+        if (sorted) sbuf[slot] = ((uint64_t)(~keys[i + u]) << 32) | (uint32_t)(i + u);
+        else out[slot] = i + u;
       }
     }
     gt_seen += g_tot;
     eq_seen += e_tot;
   }
+  if (sorted) {                                 // the k selected entries, by descending score
+    for (int i = k + tid; i < sort_n; i += kTopkThreads) sbuf[i] = ~0ull;
+    sort_and_write(sbuf, sort_n, k, k, out);
+  }
 }
 
 int launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int32_t* kv_len, int B,
-                int T, int k, int32_t* idx, cudaStream_t stream, int* status) {
+                int T, int k, uint32_t flags, int32_t* idx, cudaStream_t stream, int* status) {
   const int64_t rows = (int64_t)B * T;
   if (rows == 0) return DSA_OK;
   const int max_row = (int)(ld < DSA_TOPK_MAX_ROW ? ld : DSA_TOPK_MAX_ROW);
-  const size_t smem = (size_t)(kHistBins + ((max_row + 3) & ~3)) * sizeof(uint32_t);
+  int sort_n = 0;
+  if (flags & DSA_SORTED)
+    for (sort_n = 1; sort_n < k; sort_n <<= 1) {
+    }
+  const size_t smem = (size_t)(kHistBins + ((max_row + 3) & ~3)) * sizeof(uint32_t) + (size_t)sort_n * 8;
   static int configured_smem = 0;
   if ((int)smem > configured_smem) {
     if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -248,8 +291,8 @@ int launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int
       return DSA_ERR_CUDA;
     configured_smem = (int)smem;
   }
-  topk_kernel<<<(unsigned)rows, kTopkThreads, smem, stream>>>(scores, ld, q_pos, kv_len, T, k, max_row,
-                                                              idx, status);
+  topk_kernel<<<(unsigned)rows, kTopkThreads, smem, stream>>>(scores, ld, q_pos, kv_len, T, k, max_row, flags,
+                                                              sort_n, idx, status);
   return dsa_host::check_launch();
 }
 

@@ -57,11 +57,12 @@ def test_invalid_arguments_rejected_before_launch(L):
     p = ctypes.c_void_p(16)          # non-null, aligned dummy; never dereferenced
     bad = ctypes.c_void_p(17)        # misaligned
     n = None
-    assert L.dsa_index_keys(p, 4, 0, p, p, 10, 1, p, p, n, n) == 1              # heads < 1
-    assert L.dsa_index_keys(p, 4, 1, p, p, 10, 8, p, p, n, n) == 1              # unknown flag
-    assert L.dsa_index_keys(bad, 4, 1, p, p, 10, 1, p, p, n, n) == 1            # misaligned x
-    assert L.dsa_index_keys(n, 4, 1, p, p, 10, 1, p, p, n, n) == 1              # null x
-    assert L.dsa_index_keys(p, 0, 1, p, p, 10, 1, p, p, n, n) == 0              # empty: nothing to do
+    assert L.dsa_index_keys(p, 0, 4, 0, p, p, 10, 1, p, p, n, n) == 1           # heads < 1
+    assert L.dsa_index_keys(p, 0, 4, 1, p, p, 10, 8, p, p, n, n) == 1           # unknown flag
+    assert L.dsa_index_keys(p, 2, 4, 1, p, p, 10, 1, p, p, n, n) == 1           # unknown input type
+    assert L.dsa_index_keys(bad, 0, 4, 1, p, p, 10, 1, p, p, n, n) == 1         # misaligned x
+    assert L.dsa_index_keys(n, 1, 4, 1, p, p, 10, 1, p, p, n, n) == 1           # null x
+    assert L.dsa_index_keys(p, 0, 0, 1, p, p, 10, 1, p, p, n, n) == 0           # empty: nothing to do
     f = ctypes.c_float
     args = [p, p, p, p, p, p, p, 1, 1, 128, f(0.088), p, 128, 0, n]
     a = list(args); a[12] = 126; assert L.dsa_index_scores(*a) == 1          # ld not a multiple of 4
@@ -69,9 +70,11 @@ def test_invalid_arguments_rejected_before_launch(L):
     a = list(args); a[10] = f(0.0); assert L.dsa_index_scores(*a) == 1       # scale <= 0
     a = list(args); a[13] = 4; assert L.dsa_index_scores(*a) == 1            # unknown flag
     a = list(args); a[3] = bad; assert L.dsa_index_scores(*a) == 1          # misaligned k8
-    assert L.dsa_topk(p, 130, p, p, 1, 1, 8, p, n) == 1                      # ld % 4
-    assert L.dsa_topk(p, 128, p, p, 1, 1, 0, p, n) == 1                      # k < 1
-    assert L.dsa_topk(p, 128, p, p, 0, 1, 8, p, n) == 1                      # B < 1
+    assert L.dsa_topk(p, 130, p, p, 1, 1, 8, 0, p, n) == 1                   # ld % 4
+    assert L.dsa_topk(p, 128, p, p, 1, 1, 0, 0, p, n) == 1                   # k < 1
+    assert L.dsa_topk(p, 128, p, p, 0, 1, 8, 0, p, n) == 1                   # B < 1
+    assert L.dsa_topk(p, 128, p, p, 1, 1, 8, 8, p, n) == 1                   # unknown flag
+    assert L.dsa_topk(p, 128, p, p, 1, 1, 4097, 4, p, n) == 1                # DSA_SORTED with k > 4096
     assert L.dsa_sparse_mla(p, p, p, 1, 1, 16, 0, f(0.1), p, n, n, 0, n) == 1  # k < 1
     assert L.dsa_sparse_mla(p, p, p, 1, 1, 16, 4, f(-1.0), p, n, n, 0, n) == 1
     assert L.dsa_sparse_mla(p, bad, p, 1, 1, 16, 4, f(0.1), p, n, n, 0, n) == 1

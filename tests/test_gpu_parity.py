@@ -44,6 +44,20 @@ def test_index_keys_queries(table_dev, hadamard):
     P.check_codes(codes.cpu().numpy(), scales.cpu().numpy(), x, pos[:, None], TABLE, hadamard)
 
 
+def test_index_keys_bf16_input(table_dev):
+    """bf16 rows: the kernel widens them exactly, so the oracle runs on the widened fp32 values."""
+    rng = np.random.default_rng(21)
+    xf = rng.standard_normal((29, 64, 128)).astype(np.float32) * 3.0
+    bits = DI.bf16_bits_from_f32(xf)
+    x_wide = (bits.astype(np.uint32) << 16).view(np.float32)
+    pos = rng.integers(0, 16384, 29).astype(np.int32)
+    xb = torch.from_numpy(bits).cuda().view(torch.bfloat16)
+    codes, scales = dsa.dsa_index_keys(xb, P.to_dev(pos), table_dev)
+    torch.cuda.synchronize()
+    assert _status() == 0
+    P.check_codes(codes.cpu().numpy(), scales.cpu().numpy(), x_wide, pos[:, None], TABLE, True)
+
+
 def test_index_keys_cache_write(table_dev):
     """Keys scattered into a [B, S_max, 128] cache through dst_row; untouched rows keep their bytes."""
     B, S = 2, 300
@@ -183,6 +197,24 @@ def test_topk_exact_on_synthetic_scores(table_dev, k):
     got = _gpu_topk(sc, q_pos, kv_len, k)
     assert _status() == 0
     want = O.topk_indices(sc.astype(np.float64), q_pos, kv_len, k)
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("k", [1, 7, 300, 2048, 4096])
+def test_topk_sorted_on_synthetic_scores(table_dev, k):
+    """DSA_SORTED: the selection in descending-score order (ties by position), exactly the oracle's
+    stable sort, including rows with fewer visible keys than k."""
+    rng = np.random.default_rng(40 + k)
+    B, T, S = 2, 4, 5000
+    sc = rng.standard_normal((B, T, S)).astype(np.float32)
+    sc[0] = np.round(sc[0] * 4) / 4                     # heavy ties
+    sc[1, 0, :100] = 0.0
+    sc[1, 0, 100:200] = -0.0
+    q_pos = np.array([[4999, 10, 1999, 4095], [4999, 0, 2047, 3000]], np.int32)
+    kv_len = np.array([5000, 4500], np.int32)
+    got = dsa.dsa_topk(P.to_dev(sc), P.to_dev(q_pos), P.to_dev(kv_len), k, flags=dsa.DSA_SORTED).cpu().numpy()
+    assert _status() == 0
+    want = O.topk_indices(sc.astype(np.float64), q_pos, kv_len, k, sorted_by_score=True)
     assert np.array_equal(got, want)
 
 
@@ -332,4 +364,9 @@ def test_pipeline_end_to_end(table_dev, name):
     # moves a score by a small fraction of its term magnitude: swaps are allowed only there
     P.check_topk_near_ties(gidx.reshape(B * T, k), ref_idx.reshape(B * T, k), ref.reshape(B * T, -1),
                            mag.reshape(B * T, -1), k, band=20.0)
+    # on the GPU's own score buffer the selection is bit-exact, in both output orders
+    own = sc.cpu().numpy().astype(np.float64)
+    assert np.array_equal(gidx, O.topk_indices(own, inp.q_pos, inp.kv_len, k))
+    gs = dsa.dsa_topk(sc, P.to_dev(inp.q_pos), P.to_dev(inp.kv_len), k, flags=dsa.DSA_SORTED).cpu().numpy()
+    assert np.array_equal(gs, O.topk_indices(own, inp.q_pos, inp.kv_len, k, sorted_by_score=True))
     _check_mla(out.float().cpu().numpy(), lse.cpu().numpy(), inp.mla_q, inp.mla_kv, gidx)

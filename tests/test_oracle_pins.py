@@ -363,3 +363,18 @@ def test_sparse_mla_empty_row():
     rng = np.random.default_rng(13)
     out, lse = O.sparse_mla(_bf16(rng, (1, 1, 2, 576)), _bf16(rng, (1, 4, 576)), np.full((1, 1, 3), -1, np.int32))
     assert np.all(out == 0) and np.all(np.isneginf(lse))
+
+
+def test_topk_sorted_order_against_python_sort():
+    """sorted_by_score is the order of Python's stable sort by (-score, position) (tiny rows with
+    forced ties and negative zero), truncated to k and padded with -1."""
+    rng = np.random.default_rng(11)
+    for trial in range(200):
+        n = int(rng.integers(1, 12))
+        row = rng.choice([-1.5, -0.0, 0.0, 0.25, 2.0, 3.0], size=n).astype(np.float32)
+        k = int(rng.integers(1, 14))
+        got = O.topk_indices(row[None, None, :], np.array([[n - 1]], np.int32), np.array([n], np.int32), k,
+                             sorted_by_score=True)[0, 0]
+        want = sorted(range(n), key=lambda s: (-float(row[s]), s))[:k]
+        want = want + [-1] * (k - len(want))
+        assert got.tolist() == want, (row, k)
