@@ -69,6 +69,8 @@ constexpr int kOffV = kOffQ + kQBytes;
 constexpr int kOffRest = kOffV + kVSlots * kVSlotBytes;
 constexpr int kOffBar = kOffRest + kRestSlots * kRestSlotBytes;
 constexpr int kSmemBytes = 1024 + kOffBar + 256;
+constexpr int kStageRow = 256 + 4;                 // floats per staged output row (1040 B: conflict-free)
+static_assert(kOffV + kHeads * kStageRow * 4 <= kOffBar, "output staging fits in the KV rings");
 constexpr int kSoftmaxWarps = 4, kPvWarp = 4, kGatherWarp = 5, kGatherWarps = 4, kQkWarp = 9, kQkWarps = kSBufs;
 constexpr int kMlaThreads = (kSoftmaxWarps + 1 + kGatherWarps + kQkWarps) * 32;
 constexpr int kMaxSlots = 2048;                    // selected slots per CTA (split chunk cap)
@@ -443,9 +445,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     const bool have_o = ntiles > 0 && ok &&
                         __all_sync(0xffffffffu, mbar_wait(o_full, 0, &abort_flag, p.status, DSA_SITE_MLA_O_FULL));
     if (have_o) tc_fence_after();
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    if (p.nsplit == 1) {
-      uint16_t* dst = p.out + (bt * kHeads + h) * kDv + 256 * half;
+    // Stage this CTA's 128 x 256 output block in the (now idle) KV rings, one padded 1040-byte row
+    // per head (thread), then copy it out with each warp writing 512 contiguous bytes per store
+    // (a row per thread would scatter every warp store over 32 rows).
+    const bool final_out = p.nsplit == 1;
+    const float scale = final_out ? (l > 0.f ? 1.f / l : 0.f) : 1.f;
+    float* stage = reinterpret_cast<float*>(smem + kOffV);
+    {
+      float4* srow = reinterpret_cast<float4*>(stage + h * kStageRow);
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
         uint32_t o[32];
@@ -456,36 +463,36 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0u;
         }
-        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          d4[i] = make_uint4(pack_bf16(__uint_as_float(o[8 * i]) * inv, __uint_as_float(o[8 * i + 1]) * inv),
-                             pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv),
-                             pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv),
-                             pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv));
+        for (int i = 0; i < 8; ++i)
+          srow[c * 8 + i] = make_float4(__uint_as_float(o[4 * i]) * scale, __uint_as_float(o[4 * i + 1]) * scale,
+                                        __uint_as_float(o[4 * i + 2]) * scale, __uint_as_float(o[4 * i + 3]) * scale);
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxWarps * 32) : "memory");   // the softmax warps only
+    if (final_out) {
+      // bf16 out[bt][head][256*half + ...]: 32 chunks of 8 features per head row
+      for (int i = tid; i < kHeads * 32; i += kSoftmaxWarps * 32) {
+        const int r = i >> 5, c = i & 31;
+        const float4* src = reinterpret_cast<const float4*>(stage + r * kStageRow + c * 8);
+        const float4 u = src[0], v = src[1];
+        *reinterpret_cast<uint4*>(p.out + (bt * kHeads + r) * kDv + 256 * half + c * 8) =
+            make_uint4(pack_bf16(u.x, u.y), pack_bf16(u.z, u.w), pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
       }
       if (p.lse && half == 0)
         p.lse[bt * kHeads + h] = l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
     } else {
-      const int64_t prow = (bt * p.nsplit + split) * kHeads + h;
-      float* dst = p.part_o + prow * kDv + 256 * half;
-#pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        uint32_t o[32];
-        if (have_o) {
-          tmem_ld32(t_row + kTmemO + c * 32, o);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0u;
-        }
-        float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          d4[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                              __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+      // fp32 partial O[bt][split][head][256*half + ...]: 64 chunks of 4 features per head row
+      for (int i = tid; i < kHeads * 64; i += kSoftmaxWarps * 32) {
+        const int r = i >> 6, c = i & 63;
+        const int64_t prow = (bt * p.nsplit + split) * kHeads + r;
+        *reinterpret_cast<float4*>(p.part_o + prow * kDv + 256 * half + c * 4) =
+            *reinterpret_cast<const float4*>(stage + r * kStageRow + c * 4);
       }
-      if (half == 0) *reinterpret_cast<float2*>(p.part_ml + prow * 2) = make_float2(m, l);
+      if (half == 0) {
+        const int64_t prow = (bt * p.nsplit + split) * kHeads + h;
+        *reinterpret_cast<float2*>(p.part_ml + prow * 2) = make_float2(m, l);
+      }
     }
   }
 
