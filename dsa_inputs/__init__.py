@@ -166,3 +166,31 @@ def make_custom(batch: int, queries: int, s_max: int, topk: int, *, decode: bool
         for r, g in scale_rows.items():
             inp.idx_k[:, r, :] *= np.float32(g)
     return inp
+
+
+def paged_layout(batch: int, max_pages: int, page_size: int, seed: int, spare_pages: int = 3,
+                 kv_len=None, past_end=-1):
+    """A seeded block table for a paged cache: each (sequence, page) gets its own pool page, in
+    shuffled order, with ``spare_pages`` pool pages that no sequence uses. With ``kv_len``, the
+    entries of pages wholly past a sequence's length are set to ``past_end`` (they must not be
+    read). Returns (block_table int32 [batch, max_pages], num_pages)."""
+    rng = np.random.default_rng(seed)
+    num_pages = batch * max_pages + spare_pages
+    table = rng.permutation(num_pages)[:batch * max_pages].astype(np.int32).reshape(batch, max_pages)
+    if kv_len is not None:
+        for b, n in enumerate(np.asarray(kv_len).reshape(batch)):
+            table[b, (int(n) + page_size - 1) // page_size:] = past_end
+    return table, num_pages
+
+
+def to_paged(dense: np.ndarray, block_table: np.ndarray, page_size: int, num_pages: int, fill) -> np.ndarray:
+    """Lay a per-sequence cache dense [B, S, ...] (S = max_pages * page_size) out in a pool
+    [num_pages * page_size, ...] through block_table; rows of pages no entry names hold ``fill``."""
+    B, S = dense.shape[:2]
+    pool = np.full((num_pages * page_size,) + dense.shape[2:], fill, dtype=dense.dtype)
+    for b in range(B):
+        for pg in range(S // page_size):
+            dst = int(block_table[b, pg])
+            if 0 <= dst < num_pages:
+                pool[dst * page_size:(dst + 1) * page_size] = dense[b, pg * page_size:(pg + 1) * page_size]
+    return pool

@@ -200,6 +200,39 @@ DSA_API int dsa_sparse_mla_noalloc(const uint16_t* q, const uint16_t* kv, const 
 /* Size in bytes of the fixed scratch array dsa_sparse_mla_noalloc uses (32 MiB). */
 DSA_API size_t dsa_sparse_mla_noalloc_scratch_bytes(void);
 
+/*
+ * Paged caches (no counterpart on the pages: the block-table layout serving systems use for the
+ * K-cache and the latent cache; the arithmetic is exactly that of the dense calls).
+ *
+ * A pool holds num_pages pages of page_size rows; sequence b's logical position s lives in row
+ * block_table[b][s / page_size] * page_size + s % page_size of the pool. dsa_index_keys writes a
+ * paged K-cache through its dst_row argument (dst_row = that pool row).
+ *
+ *   block_table  int32 [B][max_pages], page ids in [0, num_pages) for every page that holds a
+ *                visible position (entries past a sequence's length are not read)
+ *   page_size    a multiple of 64; S_max = max_pages * page_size is the logical capacity
+ * A visible position whose page id is out of range sets DSA_ERR_DEVICE_BOUNDS (its key is
+ * skipped: score left unwritten, attention weight zero).
+ */
+
+/* dsa_index_scores over a paged K-cache: k8_pool uint8 [num_pages*page_size][128],
+ * k_scale_pool fp32 [num_pages*page_size]; everything else as dsa_index_scores. */
+DSA_API int dsa_index_scores_paged(const uint8_t* q8, const float* q_scale, const float* w,
+                                   const uint8_t* k8_pool, const float* k_scale_pool, int64_t num_pages,
+                                   const int32_t* block_table, int max_pages, int page_size,
+                                   const int32_t* q_pos, const int32_t* kv_len, int B, int T,
+                                   float softmax_scale, float* scores, int64_t ld, uint32_t flags,
+                                   dsa_stream_t stream);
+
+/* dsa_sparse_mla over a paged latent cache: kv_pool bf16 [num_pages*page_size][576]; idx holds
+ * logical positions (as dsa_topk writes them); everything else as dsa_sparse_mla (same
+ * workspace size). */
+DSA_API int dsa_sparse_mla_paged(const uint16_t* q, const uint16_t* kv_pool, int64_t num_pages,
+                                 const int32_t* block_table, int max_pages, int page_size,
+                                 const int32_t* idx, int B, int T, int k, float softmax_scale,
+                                 uint16_t* out, float* lse, void* workspace, size_t ws_bytes,
+                                 dsa_stream_t stream);
+
 /* Bytes of device scratch dsa_sparse_mla needs for this shape (0 when it needs none). */
 DSA_API size_t dsa_sparse_mla_workspace_size(int B, int T, int k);
 

@@ -357,6 +357,29 @@ def dense_mla(q_bits, kv_bits, q_pos, kv_len, softmax_scale: float = MLA_SOFTMAX
     return sparse_mla(q_bits, kv_bits, idx, softmax_scale, d_v)
 
 
+def paged_gather(pool, block_table, page_size: int, seq_len) -> np.ndarray:
+    """Dense per-sequence view [B, max_pages * page_size, ...] of a paged cache.
+
+    The pages say nothing of paging. READING: the block-table layout of paged KV caches in
+    serving systems -- sequence b's position s is pool row
+    block_table[b, s // page_size] * page_size + s % page_size. Positions at or past seq_len[b]
+    are not read (their table entries may be anything) and come out zero; a position below it
+    whose page id is outside the pool is an error.
+    """
+    pool = np.asarray(pool)
+    block_table = np.asarray(block_table)
+    B, max_pages = block_table.shape
+    num_pages = pool.shape[0] // page_size
+    out = np.zeros((B, max_pages * page_size) + pool.shape[1:], dtype=pool.dtype)
+    for b in range(B):
+        for s in range(int(np.asarray(seq_len).reshape(B)[b])):
+            page = int(block_table[b, s // page_size])
+            if not 0 <= page < num_pages:
+                raise IndexError(f"sequence {b} position {s}: page id {page} outside the pool")
+            out[b, s] = pool[page * page_size + s % page_size]
+    return out
+
+
 def f64_to_bf16_bits(x) -> np.ndarray:
     """Round float64 to bf16 (via the nearest fp32; the double rounding is far below the 2e-2 bar)."""
     f = np.asarray(x, dtype=np.float32)

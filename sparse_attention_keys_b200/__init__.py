@@ -16,6 +16,7 @@ __all__ = [
     "DsaError", "lib", "lib_path", "DSA_HADAMARD", "DSA_FILL_MASKED", "DSA_SORTED", "DSA_F32", "DSA_BF16", "INDEXER_SOFTMAX_SCALE",
     "MLA_SOFTMAX_SCALE", "dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk",
     "dsa_sparse_mla", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_noalloc",
+    "dsa_index_scores_paged", "dsa_sparse_mla_paged",
     "dsa_sparse_mla_noalloc_scratch_bytes", "dsa_get_device_status", "dsa_get_error_detail",
     "dsa_selftest_wait_timeout", "dsa_status_string", "dsa_device_supported", "dsa_version",
     "SITE_NAMES",
@@ -61,6 +62,9 @@ def _load():
     L.dsa_topk.argtypes = [vp, i64, vp, vp, i32, i32, i32, u32, vp, vp]
     L.dsa_sparse_mla.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
     L.dsa_sparse_mla_workspace_size.argtypes = [i32, i32, i32]
+    L.dsa_index_scores_paged.argtypes = [vp, vp, vp, vp, vp, i64, vp, i32, i32, vp, vp, i32, i32, f32, vp, i64, u32,
+                                         vp]
+    L.dsa_sparse_mla_paged.argtypes = [vp, vp, i64, vp, i32, i32, vp, i32, i32, i32, f32, vp, vp, vp, sz, vp]
     L.dsa_sparse_mla_workspace_size.restype = sz
     L.dsa_sparse_mla_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp]
     L.dsa_sparse_mla_noalloc_scratch_bytes.argtypes = []
@@ -185,6 +189,32 @@ def dsa_index_scores(q8, q_scale, w, k8, k_scale, q_pos, kv_len, softmax_scale: 
     return scores
 
 
+def dsa_index_scores_paged(q8, q_scale, w, k8_pool, k_scale_pool, block_table, page_size: int, q_pos, kv_len,
+                           softmax_scale: float = INDEXER_SOFTMAX_SCALE, scores=None, ld=None, flags: int = 0,
+                           stream=None):
+    """dsa_index_scores over a paged K-cache: k8_pool u8 [num_pages*page_size,128], k_scale_pool f32
+    [num_pages*page_size], block_table i32 [B,max_pages] -> scores fp32 [B,T,ld], ld >= max_pages*page_size."""
+    for t, dt, n in ((q8, torch.uint8, "q8"), (q_scale, torch.float32, "q_scale"), (w, torch.float32, "w"),
+                     (k8_pool, torch.uint8, "k8_pool"), (k_scale_pool, torch.float32, "k_scale_pool"),
+                     (block_table, torch.int32, "block_table"), (q_pos, torch.int32, "q_pos"),
+                     (kv_len, torch.int32, "kv_len")):
+        _need(t, dt, n)
+    B, T = q8.shape[0], q8.shape[1]
+    max_pages = block_table.shape[1]
+    num_pages = k8_pool.shape[0] // int(page_size)
+    S = max_pages * int(page_size)
+    if ld is None:
+        ld = S
+    if scores is None:
+        scores = torch.empty((B, T, ld), dtype=torch.float32, device=q8.device)
+    _need(scores, torch.float32, "scores")
+    rc = _lib.dsa_index_scores_paged(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8_pool), _ptr(k_scale_pool), num_pages,
+                                     _ptr(block_table), max_pages, int(page_size), _ptr(q_pos), _ptr(kv_len), B, T,
+                                     float(softmax_scale), _ptr(scores), int(ld), int(flags), _stream(stream))
+    _check(rc, "dsa_index_scores_paged")
+    return scores
+
+
 def dsa_topk(scores, q_pos, kv_len, k: int, idx=None, flags: int = 0, stream=None):
     """scores fp32 [B,T,ld] -> idx int32 [B,T,k] (ascending positions, or by descending score with
     flags=DSA_SORTED; -1 padded)."""
@@ -225,6 +255,32 @@ def dsa_sparse_mla(q, kv, idx, softmax_scale: float = MLA_SOFTMAX_SCALE, out=Non
                              _ptr(lse), _ptr(workspace), 0 if workspace is None else workspace.numel(),
                              _stream(stream))
     _check(rc, "dsa_sparse_mla")
+    return out, lse
+
+
+def dsa_sparse_mla_paged(q, kv_pool, block_table, page_size: int, idx, softmax_scale: float = MLA_SOFTMAX_SCALE,
+                         out=None, lse=None, workspace=None, want_lse: bool = True, stream=None):
+    """dsa_sparse_mla over a paged latent cache: kv_pool bf16 [num_pages*page_size,576], block_table
+    i32 [B,max_pages]; idx holds logical positions -> (out bf16 [B,T,128,512], lse fp32)."""
+    _need(q, torch.bfloat16, "q")
+    _need(kv_pool, torch.bfloat16, "kv_pool")
+    _need(block_table, torch.int32, "block_table")
+    _need(idx, torch.int32, "idx")
+    B, T = q.shape[0], q.shape[1]
+    k = idx.shape[-1]
+    max_pages = block_table.shape[1]
+    num_pages = kv_pool.shape[0] // int(page_size)
+    if out is None:
+        out = torch.empty((B, T, 128, 512), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, T, 128), dtype=torch.float32, device=q.device)
+    ws_bytes = dsa_sparse_mla_workspace_size(B, T, k)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    rc = _lib.dsa_sparse_mla_paged(_ptr(q), _ptr(kv_pool), num_pages, _ptr(block_table), max_pages, int(page_size),
+                                   _ptr(idx), B, T, int(k), float(softmax_scale), _ptr(out), _ptr(lse),
+                                   _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
+    _check(rc, "dsa_sparse_mla_paged")
     return out, lse
 
 

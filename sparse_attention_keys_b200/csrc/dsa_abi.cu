@@ -267,6 +267,53 @@ int dsa_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, in
                                 (cudaStream_t)stream, status);
 }
 
+// Shared checks of the paged-cache arguments: page ids are int32 and pool rows index int32.
+static bool paged_args_ok(int64_t num_pages, const int32_t* block_table, int max_pages, int page_size) {
+  if (num_pages < 1 || max_pages < 1 || page_size < 64 || page_size % 64 != 0) return false;
+  if (num_pages * page_size > 0x7fffffffLL || (int64_t)max_pages * page_size > 0x7fffffffLL) return false;
+  return block_table != nullptr && (reinterpret_cast<uintptr_t>(block_table) & 3) == 0;
+}
+
+int dsa_index_scores_paged(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8_pool,
+                           const float* k_scale_pool, int64_t num_pages, const int32_t* block_table, int max_pages,
+                           int page_size, const int32_t* q_pos, const int32_t* kv_len, int B, int T,
+                           float softmax_scale, float* scores, int64_t ld, uint32_t flags, dsa_stream_t stream) {
+  if (!paged_args_ok(num_pages, block_table, max_pages, page_size)) return DSA_ERR_INVALID_ARG;
+  const int64_t S_max = (int64_t)max_pages * page_size;
+  if (B < 1 || T < 1 || ld < S_max || (ld & 3) != 0 || (flags & ~DSA_FILL_MASKED) != 0 ||
+      !(softmax_scale > 0.f) || !isfinite(softmax_scale))
+    return DSA_ERR_INVALID_ARG;
+  if ((int64_t)B * T * 64 > 0x7fffffffLL) return DSA_ERR_INVALID_ARG;
+  if (!q8 || !q_scale || !w || !k8_pool || !k_scale_pool || !q_pos || !kv_len || !scores) return DSA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q8, q_scale, w, k8_pool, k_scale_pool, q_pos, kv_len, scores};
+  for (const void* p : ptrs)
+    if (!dsa_host::aligned16(p)) return DSA_ERR_INVALID_ARG;
+  int* status;
+  int rc = prologue(&status);
+  if (rc != DSA_OK) return rc;
+  return dsa::launch_index_scores_paged(q8, q_scale, w, k8_pool, k_scale_pool, num_pages, block_table, max_pages,
+                                        page_size, q_pos, kv_len, B, T, softmax_scale, scores, ld, flags,
+                                        (cudaStream_t)stream, status);
+}
+
+int dsa_sparse_mla_paged(const uint16_t* q, const uint16_t* kv_pool, int64_t num_pages, const int32_t* block_table,
+                         int max_pages, int page_size, const int32_t* idx, int B, int T, int k, float softmax_scale,
+                         uint16_t* out, float* lse, void* workspace, size_t ws_bytes, dsa_stream_t stream) {
+  if (!paged_args_ok(num_pages, block_table, max_pages, page_size)) return DSA_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || k < 1 || !(softmax_scale > 0.f) || !isfinite(softmax_scale)) return DSA_ERR_INVALID_ARG;
+  if ((int64_t)B * T * 2 * 1024 > 0x7fffffffLL) return DSA_ERR_INVALID_ARG;
+  if (!q || !kv_pool || !idx || !out) return DSA_ERR_INVALID_ARG;
+  if (!dsa_host::aligned16(q) || !dsa_host::aligned16(kv_pool) || !dsa_host::aligned16(idx) ||
+      !dsa_host::aligned16(out) || (lse && !dsa_host::aligned16(lse)) ||
+      (workspace && !dsa_host::aligned16(workspace)))
+    return DSA_ERR_INVALID_ARG;
+  int* status;
+  int rc = prologue(&status);
+  if (rc != DSA_OK) return rc;
+  return dsa::launch_sparse_mla_paged(q, kv_pool, num_pages, block_table, max_pages, page_size, idx, B, T, k,
+                                      softmax_scale, out, lse, workspace, ws_bytes, (cudaStream_t)stream, status);
+}
+
 int dsa_get_device_status(dsa_stream_t stream) {
   DeviceCache* c = device_cache();
   if (!c) return DSA_ERR_CUDA;

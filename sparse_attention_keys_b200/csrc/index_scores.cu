@@ -56,11 +56,22 @@ struct ScoresParams {
   float wscale;        // 64^-0.5 * softmax_scale
   uint32_t flags;
   int* status;
+  // paged K-cache (block_table == nullptr: dense [B][S_max] rows)
+  const int32_t* block_table;   // [B][max_pages]
+  int max_pages, page_size;
+  int64_t num_pages;
 };
+
+// Pool row of sequence b's logical position s in a paged K-cache, or -1 if its page id is out of
+// range (S_max = max_pages * page_size bounds s).
+__device__ __forceinline__ int64_t paged_row(const ScoresParams& p, int b, int s) {
+  const int pg = __ldg(p.block_table + (int64_t)b * p.max_pages + s / p.page_size);
+  return (pg >= 0 && pg < p.num_pages) ? (int64_t)pg * p.page_size + s % p.page_size : -1;
+}
 
 }  // namespace
 
-template <int NQ>
+template <int NQ, bool PAGED>
 __global__ void __launch_bounds__(threads_for(NQ), 1)
     index_scores_kernel(const __grid_constant__ CUtensorMap qmap,
                         const __grid_constant__ CUtensorMap kmap, const ScoresParams p) {
@@ -143,12 +154,31 @@ __global__ void __launch_bounds__(threads_for(NQ), 1)
       prefetch_tensormap(&kmap);
       mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
       tma_load_2d(q_smem, &qmap, q_full, 0, (b * p.T + t0) * 64);
+      // paged: each tile is two 64-row boxes from their pages (looked up one tile ahead); a half
+      // past S_max or on an invalid page loads from an out-of-range row, i.e. zeros
+      auto half_rows = [&](int i, int32_t (&r)[2]) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int ks0 = (kt_begin + i) * kKeysPerTile + 64 * hh;
+          int64_t row = -1;
+          if (i < my_tiles && ks0 < p.S_max) row = paged_row(p, b, ks0);
+          r[hh] = row >= 0 ? (int32_t)row : (int32_t)(p.num_pages * p.page_size);
+        }
+      };
+      int32_t rows_next[2] = {0, 0};
+      if (PAGED) half_rows(0, rows_next);
       for (int i = 0; i < my_tiles; ++i) {
         const int s = i % STAGES;
+        int32_t rows[2] = {rows_next[0], rows_next[1]};
+        if (PAGED) half_rows(i + 1, rows_next);
         if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) + 1) & 1, &abort_flag, p.status, DSA_SITE_SCORES_K_EMPTY)) break;
         mbar_arrive_expect_tx(&full[s], kTileBytes);
-        tma_load_2d(k_smem + s * kTileBytes, &kmap, &full[s], 0,
-                    b * p.S_max + (kt_begin + i) * kKeysPerTile);
+        if (PAGED) {
+          tma_load_2d(k_smem + s * kTileBytes, &kmap, &full[s], 0, rows[0]);
+          tma_load_2d(k_smem + s * kTileBytes + kTileBytes / 2, &kmap, &full[s], 0, rows[1]);
+        } else {
+          tma_load_2d(k_smem + s * kTileBytes, &kmap, &full[s], 0, b * p.S_max + (kt_begin + i) * kKeysPerTile);
+        }
       }
     }
   } else if (warp == kEpiWarps + 1) {
@@ -182,9 +212,12 @@ __global__ void __launch_bounds__(threads_for(NQ), 1)
     const bool active = q_lo < NQ;                     // NQ = 1: one warp per quadrant
     const int row_in_tile = quad * 32 + lane;          // TMEM lane = key within the tile
     const float* ks_row = p.k_scale + (int64_t)b * p.S_max;
-    auto load_ks = [&](int i) -> float {               // k_scale of this thread's key in tile i
+    auto load_ks = [&](int i) -> float {               // k_scale of this thread's key in tile i (-1: bad page)
       const int key = (kt_begin + i) * kKeysPerTile + row_in_tile;
-      return (active && i < my_tiles && key < p.S_max) ? __ldg(ks_row + key) : 0.f;
+      if (!(active && i < my_tiles && key < p.S_max)) return 0.f;
+      if (!PAGED) return __ldg(ks_row + key);
+      const int64_t row = paged_row(p, b, key);
+      return row >= 0 ? __ldg(p.k_scale + row) : -1.f;
     };
     float ks_next = load_ks(0);
     for (int i = 0; i < my_tiles; ++i) {
@@ -222,7 +255,10 @@ __global__ void __launch_bounds__(threads_for(NQ), 1)
           const int t = t0 + q;
           if (t < p.T) {
             float* dst = p.scores + ((int64_t)b * p.T + t) * p.ld;
-            if (key < nvalid[q]) dst[key] = tot * ks;
+            if (key < nvalid[q]) {
+              if (!PAGED || ks >= 0.f) dst[key] = tot * ks;
+              else set_status(p.status, DSA_ERR_DEVICE_BOUNDS);   // visible key on an invalid page
+            }
             else if ((p.flags & DSA_FILL_MASKED) && key < p.S_max) dst[key] = -INFINITY;
           }
         }
@@ -251,7 +287,7 @@ __global__ void __launch_bounds__(threads_for(NQ), 1)
   }
 }
 
-template <int NQ>
+template <int NQ, bool PAGED>
 static int launch_scores_nq(const uint8_t* q8, const uint8_t* k8, const ScoresParams& base,
                             cudaStream_t stream) {
   using Cfg = ScoresCfg<NQ>;
@@ -260,7 +296,9 @@ static int launch_scores_nq(const uint8_t* q8, const uint8_t* k8, const ScoresPa
                                       (uint64_t)base.B * base.T * 64, 128, 128, NQ * 64,
                                       CU_TENSOR_MAP_SWIZZLE_128B) ||
       !dsa_host::encode_tensor_map_2d(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, (void*)k8, 128,
-                                      (uint64_t)base.B * base.S_max, 128, 128, kKeysPerTile,
+                                      base.block_table ? (uint64_t)base.num_pages * base.page_size
+                                                       : (uint64_t)base.B * base.S_max,
+                                      128, 128, base.block_table ? kKeysPerTile / 2 : kKeysPerTile,
                                       CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
   ScoresParams p = base;
@@ -274,12 +312,12 @@ static int launch_scores_nq(const uint8_t* q8, const uint8_t* k8, const ScoresPa
   if (dev < 64 && occupancy[dev] == 0) {
     // all of the unified L1 / shared storage as shared memory, so that as many CTAs as the shared
     // memory allows are resident
-    if (cudaFuncSetAttribute(index_scores_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(index_scores_kernel<NQ, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(index_scores_kernel<NQ>, cudaFuncAttributePreferredSharedMemoryCarveout,
+        cudaFuncSetAttribute(index_scores_kernel<NQ, PAGED>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return DSA_ERR_CUDA;
-    const int per_sm = dsa_host::resident_ctas_per_sm((const void*)index_scores_kernel<NQ>, threads_for(NQ),
+    const int per_sm = dsa_host::resident_ctas_per_sm((const void*)index_scores_kernel<NQ, PAGED>, threads_for(NQ),
                                                       Cfg::kSmemBytes, Cfg::kTmemCols);
     if (per_sm < 1) return DSA_ERR_CUDA;
     occupancy[dev] = per_sm;
@@ -292,10 +330,10 @@ static int launch_scores_nq(const uint8_t* q8, const uint8_t* k8, const ScoresPa
   p.ksplit = (tiles_max + p.tiles_per_split - 1) / p.tiles_per_split;
   const int64_t grid = units * p.ksplit;
   if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;
-  if (dev >= 64 && cudaFuncSetAttribute(index_scores_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (dev >= 64 && cudaFuncSetAttribute(index_scores_kernel<NQ, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         Cfg::kSmemBytes) != cudaSuccess)
     return DSA_ERR_CUDA;
-  index_scores_kernel<NQ><<<(unsigned)grid, threads_for(NQ), Cfg::kSmemBytes, stream>>>(qmap, kmap, p);
+  index_scores_kernel<NQ, PAGED><<<(unsigned)grid, threads_for(NQ), Cfg::kSmemBytes, stream>>>(qmap, kmap, p);
   return dsa_host::check_launch();
 }
 
@@ -308,8 +346,23 @@ int launch_index_scores(const uint8_t* q8, const float* q_scale, const float* w,
   p.scores = scores; p.ld = ld; p.B = B; p.T = T; p.S_max = S_max;
   p.wscale = 0.125f * softmax_scale;   // 64^-0.5 (n_heads**-0.5 in Indexer.forward)
   p.flags = flags; p.status = status;
-  if (T >= 4) return launch_scores_nq<4>(q8, k8, p, stream);
-  return launch_scores_nq<1>(q8, k8, p, stream);
+  if (T >= 4) return launch_scores_nq<4, false>(q8, k8, p, stream);
+  return launch_scores_nq<1, false>(q8, k8, p, stream);
+}
+
+int launch_index_scores_paged(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8_pool,
+                              const float* k_scale_pool, int64_t num_pages, const int32_t* block_table,
+                              int max_pages, int page_size, const int32_t* q_pos, const int32_t* kv_len, int B,
+                              int T, float softmax_scale, float* scores, int64_t ld, uint32_t flags,
+                              cudaStream_t stream, int* status) {
+  ScoresParams p{};
+  p.q_scale = q_scale; p.w = w; p.k_scale = k_scale_pool; p.q_pos = q_pos; p.kv_len = kv_len;
+  p.scores = scores; p.ld = ld; p.B = B; p.T = T; p.S_max = max_pages * page_size;
+  p.wscale = 0.125f * softmax_scale;
+  p.flags = flags; p.status = status;
+  p.block_table = block_table; p.max_pages = max_pages; p.page_size = page_size; p.num_pages = num_pages;
+  if (T >= 4) return launch_scores_nq<4, true>(q8, k8_pool, p, stream);
+  return launch_scores_nq<1, true>(q8, k8_pool, p, stream);
 }
 
 }  // namespace dsa

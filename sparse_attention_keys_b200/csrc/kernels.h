@@ -16,10 +16,20 @@ int launch_index_scores(const uint8_t* q8, const float* q_scale, const float* w,
                         int T, int S_max, float softmax_scale, float* scores, int64_t ld,
                         uint32_t flags, cudaStream_t stream, int* status);
 
+int launch_index_scores_paged(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8_pool,
+                              const float* k_scale_pool, int64_t num_pages, const int32_t* block_table,
+                              int max_pages, int page_size, const int32_t* q_pos, const int32_t* kv_len, int B,
+                              int T, float softmax_scale, float* scores, int64_t ld, uint32_t flags,
+                              cudaStream_t stream, int* status);
+
 int launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int32_t* kv_len, int B,
                 int T, int k, uint32_t flags, int32_t* idx, cudaStream_t stream, int* status);
 
 size_t sparse_mla_workspace_size(int B, int T, int k);
+int launch_sparse_mla_paged(const uint16_t* q, const uint16_t* kv_pool, int64_t num_pages,
+                            const int32_t* block_table, int max_pages, int page_size, const int32_t* idx, int B,
+                            int T, int k, float softmax_scale, uint16_t* out, float* lse, void* workspace,
+                            size_t ws_bytes, cudaStream_t stream, int* status);
 int launch_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T,
                       int S_max, int k, float softmax_scale, uint16_t* out, float* lse,
                       void* workspace, size_t ws_bytes, cudaStream_t stream, int* status);

@@ -147,7 +147,22 @@ struct MlaParams {
   float* part_o;             // [BT][nsplit][128][512]   (nsplit > 1)
   float* part_ml;            // [BT][nsplit][128][2]     running max (log2 domain), sum
   int* status;
+  // paged latent cache: kv is a pool of num_pages pages of page_size rows, and logical position v of
+  // sequence b lives in row block_table[b][v / page_size] * page_size + v % page_size
+  const int32_t* block_table;  // [B][max_pages]
+  int max_pages, page_size;
+  int64_t num_pages;
 };
+
+// Pool row of logical position v (PAGED: pg = block_table[b][v / page_size], read one tile ahead),
+// or -1 for a slot that takes no part: padding (v < 0), v >= S_max, or a page id outside the pool.
+template <bool PAGED>
+__device__ __forceinline__ int kv_row(const MlaParams& p, int v, int pg) {
+  if (v < 0 || v >= p.S_max) return -1;
+  if (!PAGED) return v;
+  if (pg < 0 || (int64_t)pg >= p.num_pages) return -1;
+  return pg * p.page_size + v % p.page_size;
+}
 
 // Q K^T of one 32-key tile: 20 K-steps with Q from TMEM, then 16 with Q from shared memory. HALF
 // fixes which ring holds each 64-feature block, so every B descriptor is a base plus a constant.
@@ -175,6 +190,7 @@ __device__ __forceinline__ void issue_qk_tile(uint32_t d, uint32_t tq, uint32_t 
   }
 }
 
+template <bool PAGED>
 __global__ void __launch_bounds__(kMlaThreads, 1)
     sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -281,17 +297,33 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       for (int r = kQTmemRegions; r < kRegions; ++r)
         tma_load_2d(q_sm + (r - kQTmemRegions) * kQRegion, &q_map, q_full, 64 * r, (int32_t)(bt * kHeads));
     }
-    const uint16_t* kv_b = p.kv + (int64_t)b * p.S_max * kDqk;
+    const uint16_t* kv_b = PAGED ? p.kv : p.kv + (int64_t)b * p.S_max * kDqk;
+    const int32_t* pages = PAGED ? p.block_table + (int64_t)b * p.max_pages : nullptr;
     const uint32_t blk = (uint32_t)(lane >> 3) * kKvRegion;      // block of chunks L and L+32 in its ring slot
     auto load_idx = [&](int j) -> int {
       const int slot = j * kKeys + 8 * w + (lane & 7);
       return (j < ntiles && slot < nslots) ? __ldg(idx_row + slot) : -1;
     };
+    auto load_page = [&](int v) -> int { return (v >= 0 && v < p.S_max) ? __ldg(pages + v / p.page_size) : -1; };
+    // dense: indices one tile ahead; paged: indices two tiles ahead, their page ids one tile ahead
     int idx_next = idx_first;                        // load_idx(0), issued before the set-up barrier
+    int pg_next = 0, idx_next2 = -1;
+    if (PAGED) {
+      idx_next2 = load_idx(1);
+      pg_next = load_page(idx_next);
+    }
     for (int j = 0; j < ntiles; ++j) {
-      const int idx_cur = idx_next;
-      idx_next = load_idx(j + 1);                     // one tile ahead
-      if (lane < 8 && idx_cur >= p.S_max) set_status(p.status, DSA_ERR_DEVICE_BOUNDS);
+      const int idx_cur = idx_next, pg_cur = pg_next;
+      if (PAGED) {
+        idx_next = idx_next2;
+        idx_next2 = load_idx(j + 2);
+        pg_next = load_page(idx_next);
+      } else {
+        idx_next = load_idx(j + 1);
+      }
+      const int row_cur = kv_row<PAGED>(p, idx_cur, pg_cur);
+      // a selected position past the cache, or (paged) on a page outside the pool
+      if (lane < 8 && idx_cur >= 0 && row_cur < 0) set_status(p.status, DSA_ERR_DEVICE_BOUNDS);
       if (j >= kRestSlots &&
           !__all_sync(0xffffffffu, mbar_wait(&rest_empty[j % kRestSlots], ((j / kRestSlots) + 1) & 1, &abort_flag,
                                              p.status, DSA_SITE_MLA_KV_EMPTY)))
@@ -307,10 +339,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       const uint32_t d2 = r_slot + 4 * kKvRegion;                        // rotary block
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        const int v = __shfl_sync(0xffffffffu, idx_cur, kk);
-        const bool ok = v >= 0 && v < p.S_max;
+        const int row = __shfl_sync(0xffffffffu, row_cur, kk);
+        const bool ok = row >= 0;
         const uint32_t off = sw128(8 * w + kk, lane & 7);
-        const uint16_t* src = kv_b + (int64_t)(ok ? v : 0) * kDqk + lane * 8;
+        const uint16_t* src = kv_b + (int64_t)(ok ? row : 0) * kDqk + lane * 8;
         cp_async_16_zfill(d0 + off, src, ok);
         cp_async_16_zfill(d1 + off, src + 256, ok);
         if (lane < 8) cp_async_16_zfill(d2 + off, src + 512, ok);
@@ -372,16 +404,29 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     }
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    int v_next = lane < nslots ? __ldg(idx_row + lane) : -1;     // slot j * 32 + lane of the next tile
+    // slot j * 32 + lane of the next tile (paged: also the slot two tiles ahead and the next tile's page id)
+    const int32_t* pages = PAGED ? p.block_table + (int64_t)b * p.max_pages : nullptr;
+    auto load_page = [&](int v) -> int { return (v >= 0 && v < p.S_max) ? __ldg(pages + v / p.page_size) : -1; };
+    int v_next = lane < nslots ? __ldg(idx_row + lane) : -1;
+    int pg_next = 0, v_next2 = -1;
+    if (PAGED) {
+      v_next2 = kKeys + lane < nslots ? __ldg(idx_row + kKeys + lane) : -1;
+      pg_next = load_page(v_next);
+    }
 #pragma unroll 1
     for (int j = 0; ok && j < ntiles; ++j) {
       const uint32_t s_col = kTmemS + (j % kSBufs) * kKeys;
-      const int v_cur = v_next;
-      {
+      const int v_cur = v_next, pg_cur = pg_next;
+      if (PAGED) {
+        v_next = v_next2;
+        const int sn = (j + 2) * kKeys + lane;
+        v_next2 = sn < nslots ? __ldg(idx_row + sn) : -1;
+        pg_next = load_page(v_next);
+      } else {
         const int sn = (j + 1) * kKeys + lane;
         v_next = sn < nslots ? __ldg(idx_row + sn) : -1;
       }
-      const uint32_t vmask = __ballot_sync(0xffffffffu, v_cur >= 0 && v_cur < p.S_max);
+      const uint32_t vmask = __ballot_sync(0xffffffffu, kv_row<PAGED>(p, v_cur, pg_cur) >= 0);
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j % kSBufs], (j / kSBufs) & 1, &abort_flag, p.status,
                                              DSA_SITE_MLA_S_FULL))) {
         ok = false;
@@ -552,17 +597,12 @@ size_t sparse_mla_workspace_size(int B, int T, int k) {
   return (size_t)BT * s.nsplit * kHeads * (kDv + 2) * sizeof(float);
 }
 
-int launch_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T,
-                      int S_max, int k, float softmax_scale, uint16_t* out, float* lse,
-                      void* workspace, size_t ws_bytes, cudaStream_t stream, int* status) {
-  const int64_t BT = (int64_t)B * T;
+template <bool PAGED>
+static int launch_mla(const uint16_t* q, MlaParams p, cudaStream_t stream, void* workspace, size_t ws_bytes) {
+  const int64_t BT = (int64_t)p.B * p.T;
   if (BT == 0) return DSA_OK;
-  const MlaSplit s = choose_split(BT, k, dsa_host::device_sm_count());
-  MlaParams p{};
-  p.q = q; p.kv = kv; p.idx = idx; p.B = B; p.T = T; p.S_max = S_max; p.k = k;
+  const MlaSplit s = choose_split(BT, p.k, dsa_host::device_sm_count());
   p.nsplit = s.nsplit; p.chunk = s.chunk;
-  p.scale_log2 = softmax_scale * kLog2e;
-  p.out = out; p.lse = lse; p.status = status;
   if (s.nsplit > 1) {
     const size_t need = (size_t)BT * s.nsplit * kHeads * (kDv + 2) * sizeof(float);
     if (workspace == nullptr || ws_bytes < need) return DSA_ERR_WORKSPACE;
@@ -573,7 +613,7 @@ int launch_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
-    if (cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+    if (cudaFuncSetAttribute(sparse_mla_kernel<PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
         cudaSuccess)
       return DSA_ERR_CUDA;
     configured[dev] = true;
@@ -584,12 +624,34 @@ int launch_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
   if (!dsa_host::encode_tensor_map_2d(&q_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (void*)q, kDqk,
                                       (uint64_t)BT * kHeads, kDqk * 2, 64, kHeads, CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
-  sparse_mla_kernel<<<(unsigned)grid, kMlaThreads, kSmemBytes, stream>>>(q_map, p);
+  sparse_mla_kernel<PAGED><<<(unsigned)grid, kMlaThreads, kSmemBytes, stream>>>(q_map, p);
   int rc = dsa_host::check_launch();
   if (rc != DSA_OK || s.nsplit == 1) return rc;
   const int64_t rows = BT * kHeads;
   sparse_mla_combine_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p, rows);
   return dsa_host::check_launch();
+}
+
+int launch_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T,
+                      int S_max, int k, float softmax_scale, uint16_t* out, float* lse,
+                      void* workspace, size_t ws_bytes, cudaStream_t stream, int* status) {
+  MlaParams p{};
+  p.q = q; p.kv = kv; p.idx = idx; p.B = B; p.T = T; p.S_max = S_max; p.k = k;
+  p.scale_log2 = softmax_scale * kLog2e;
+  p.out = out; p.lse = lse; p.status = status;
+  return launch_mla<false>(q, p, stream, workspace, ws_bytes);
+}
+
+int launch_sparse_mla_paged(const uint16_t* q, const uint16_t* kv_pool, int64_t num_pages,
+                            const int32_t* block_table, int max_pages, int page_size, const int32_t* idx, int B,
+                            int T, int k, float softmax_scale, uint16_t* out, float* lse, void* workspace,
+                            size_t ws_bytes, cudaStream_t stream, int* status) {
+  MlaParams p{};
+  p.q = q; p.kv = kv_pool; p.idx = idx; p.B = B; p.T = T; p.S_max = max_pages * page_size; p.k = k;
+  p.scale_log2 = softmax_scale * kLog2e;
+  p.out = out; p.lse = lse; p.status = status;
+  p.block_table = block_table; p.max_pages = max_pages; p.page_size = page_size; p.num_pages = num_pages;
+  return launch_mla<true>(q, p, stream, workspace, ws_bytes);
 }
 
 }  // namespace dsa

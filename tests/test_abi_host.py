@@ -78,6 +78,22 @@ def test_invalid_arguments_rejected_before_launch(L):
     assert L.dsa_sparse_mla(p, p, p, 1, 1, 16, 0, f(0.1), p, n, n, 0, n) == 1  # k < 1
     assert L.dsa_sparse_mla(p, p, p, 1, 1, 16, 4, f(-1.0), p, n, n, 0, n) == 1
     assert L.dsa_sparse_mla(p, bad, p, 1, 1, 16, 4, f(0.1), p, n, n, 0, n) == 1
+    # paged calls: (..., num_pages, block_table, max_pages, page_size, ...)
+    sargs = [p, p, p, p, p, 8, p, 4, 64, p, p, 1, 1, f(0.088), p, 256, 0, n]
+    a = list(sargs); a[8] = 32; assert L.dsa_index_scores_paged(*a) == 1    # page_size < 64
+    a = list(sargs); a[8] = 96; assert L.dsa_index_scores_paged(*a) == 1    # page_size not a multiple of 64
+    a = list(sargs); a[5] = 0; assert L.dsa_index_scores_paged(*a) == 1     # empty pool
+    a = list(sargs); a[7] = 0; assert L.dsa_index_scores_paged(*a) == 1     # max_pages < 1
+    a = list(sargs); a[6] = n; assert L.dsa_index_scores_paged(*a) == 1     # null block table
+    a = list(sargs); a[6] = ctypes.c_void_p(18); assert L.dsa_index_scores_paged(*a) == 1   # table not int32-aligned
+    a = list(sargs); a[15] = 128; assert L.dsa_index_scores_paged(*a) == 1  # ld < max_pages * page_size
+    a = list(sargs); a[5] = 1 << 26; assert L.dsa_index_scores_paged(*a) == 1   # pool rows past int32
+    a = list(sargs); a[3] = bad; assert L.dsa_index_scores_paged(*a) == 1   # misaligned pool
+    margs = [p, p, 8, p, 4, 64, p, 1, 1, 16, f(0.1), p, n, n, 0, n]
+    a = list(margs); a[5] = 100; assert L.dsa_sparse_mla_paged(*a) == 1     # page_size
+    a = list(margs); a[3] = n; assert L.dsa_sparse_mla_paged(*a) == 1       # null block table
+    a = list(margs); a[9] = 0; assert L.dsa_sparse_mla_paged(*a) == 1       # k < 1
+    a = list(margs); a[1] = bad; assert L.dsa_sparse_mla_paged(*a) == 1     # misaligned pool
     assert L.dsa_rope_table(n, 10) == 1
     assert L.dsa_rope_table(p, 0) == 1
 

@@ -378,3 +378,44 @@ def test_topk_sorted_order_against_python_sort():
         want = sorted(range(n), key=lambda s: (-float(row[s]), s))[:k]
         want = want + [-1] * (k - len(want))
         assert got.tolist() == want, (row, k)
+
+
+# ------------------------------------------------------------------------------------ paged caches
+def test_paged_gather_worked_example():
+    # page_size 2, pool rows labelled by their own row number: sequence 0 uses pages (2, 0), so its
+    # positions 0..3 are pool rows 4, 5, 0, 1; sequence 1 uses pages (1, 3): rows 2, 3, 6, 7
+    pool = np.arange(8, dtype=np.int64)[:, None] * np.ones((1, 3), np.int64)
+    got = O.paged_gather(pool, np.array([[2, 0], [1, 3]]), 2, [4, 4])
+    assert got[:, :, 0].tolist() == [[4, 5, 0, 1], [2, 3, 6, 7]]
+    assert np.all(got == got[:, :, :1])
+
+
+def test_paged_gather_identity_table_is_a_reshape():
+    rng = np.random.default_rng(0)
+    B, max_pages, P = 3, 4, 8
+    pool = rng.standard_normal((B * max_pages * P, 5))
+    table = np.arange(B * max_pages).reshape(B, max_pages)
+    got = O.paged_gather(pool, table, P, [max_pages * P] * B)
+    assert np.array_equal(got, pool.reshape(B, max_pages * P, 5))
+
+
+def test_paged_gather_inverts_a_shuffled_layout():
+    import dsa_inputs as DI
+    rng = np.random.default_rng(1)
+    B, max_pages, P = 2, 5, 64
+    dense = rng.integers(0, 256, (B, max_pages * P, 7), dtype=np.uint8)
+    kv_len = np.array([max_pages * P, 130])
+    table, num_pages = DI.paged_layout(B, max_pages, P, seed=2, kv_len=kv_len, past_end=-7)
+    pool = DI.to_paged(dense, table, P, num_pages, fill=255)
+    got = O.paged_gather(pool, table, P, kv_len)
+    for b in range(B):
+        assert np.array_equal(got[b, :kv_len[b]], dense[b, :kv_len[b]])
+        assert np.all(got[b, kv_len[b]:] == 0)
+    assert np.all(table[1, 3:] == -7)                       # pages past the end are never read
+
+
+def test_paged_gather_rejects_a_visible_bad_page():
+    pool = np.zeros((8, 2))
+    with pytest.raises(IndexError):
+        O.paged_gather(pool, np.array([[0, 4]]), 2, [3])      # position 2 lives on page 4 of 4
+    O.paged_gather(pool, np.array([[0, 4]]), 2, [2])          # ... unless it is past the end
