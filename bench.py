@@ -7,9 +7,12 @@ resident FP8 K-cache) and on the queries, dsa_index_scores, dsa_topk and dsa_spa
 prefill step runs the same calls over all T queries and S keys. Inputs are seeded synthetic
 tensors of the workload's shapes (dsa_inputs); the caches are resident device state.
 
-Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on the launching
-stream with a 256 MiB L2-flush write between steps (outside the events); the K step times are
-summed, ranks barrier + synchronise before and after, and rank 0 reports the max over ranks.
+Timing: W untimed warm-up steps, then K steps, each a replay of a CUDA graph of the step bracketed
+by CUDA events on the launching stream, with a 256 MiB L2-flush write between steps (outside the
+events) when the inputs fit in L2; the K step times are summed, ranks barrier + synchronise before
+and after, and rank 0 reports the max over ranks. After each timed step a second graph of the same
+step, with an event pair around each ABI call, is replayed for the per-kernel durations (the
+roofline's kernel time); its event nodes would lengthen the step, so it is not part of the step time.
 Under torchrun each rank runs its own replica of the workload (independent sequences, no
 collective on the data path): weak scaling.
 
@@ -304,19 +307,27 @@ def run_ours(args, rank, world, local_rank):
             tdist.barrier()
         torch.cuda.synchronize()
 
-    # ---- device-timed region (inputs resident in HBM): the step is captured once as a CUDA graph
-    # (with an event node around each ABI call) and replayed, so no host launch gaps are timed
+    # ---- device-timed region (inputs resident in HBM). The step is captured as a CUDA graph and
+    # replayed, so no host launch gaps are timed. A second graph of the same step holds an event
+    # pair around each ABI call and is replayed after every timed step for the per-kernel
+    # durations: event nodes lengthen a replay by a few microseconds each, so they stay out of
+    # the step time.
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        cap_stream = torch.cuda.Stream()
+        cap_stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cap_stream):
+            st.run()                              # warm the capture stream (records no events)
+        torch.cuda.current_stream().wait_stream(cap_stream)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=cap_stream):
+            fn()
+        torch.cuda.synchronize()
+        return g
+
     kev = {}
-    graph = torch.cuda.CUDAGraph()
-    cap_stream = torch.cuda.Stream()
-    cap_stream.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(cap_stream):
-        st.run()                                  # warm the capture stream
-    torch.cuda.current_stream().wait_stream(cap_stream)
-    torch.cuda.synchronize()
-    with torch.cuda.graph(graph, stream=cap_stream):
-        st.run(kev)
-    torch.cuda.synchronize()
+    graph = capture(st.run)
+    graph_k = capture(lambda: st.run(kev))
     steps = []
     with ClockSampler(local_rank) as clk:
         # the sampler polls every 20 ms: keep the GPU under the same load for ~0.5 s before the
@@ -325,6 +336,8 @@ def run_ours(args, rank, world, local_rank):
         while time.perf_counter() < t_end:
             st.l2_flush()
             graph.replay()
+            st.l2_flush()
+            graph_k.replay()
             torch.cuda.synchronize()
         barrier()
         per_kernel_sum = {n: 0.0 for n in kev}
@@ -336,6 +349,8 @@ def run_ours(args, rank, world, local_rank):
             graph.replay()
             e.record()
             steps.append((s, e))
+            st.l2_flush()
+            graph_k.replay()                       # the same step with per-call event nodes
             torch.cuda.synchronize()               # read this replay's kernel events before the next
             for n, v in kev.items():
                 per_kernel_sum[n] += sum(a.elapsed_time(b) for a, b in v)
@@ -343,7 +358,7 @@ def run_ours(args, rank, world, local_rank):
     clocks = clk.summary()
     t_dev = sum(s.elapsed_time(e) for s, e in steps) / 1e3          # seconds
     per_kernel = {n: v / args.steps / 1e3 for n, v in per_kernel_sum.items()}
-    del graph
+    del graph, graph_k
     check_status(dsa, "graph replays")
 
     # ---- end to end through host buffers (pinned H2D of the step inputs, D2H of the results)
@@ -401,7 +416,9 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": weak_scaling_value(units["pairs"], args.steps, world, t_e2e), "unit": UNIT, "h2d_bytes_per_step": st.bytes_h2d(),
                 "d2h_bytes_per_step": st.bytes_d2h(), "ms_per_step": t_e2e / args.steps * 1e3},
         "gpu_launches": st.launches_per_step * args.steps,
-        "timing": "device: CUDA-graph replay of the step, CUDA events around each replay; e2e: plain API calls",
+        "timing": ("device: CUDA-graph replay of the step, CUDA events around each replay; kernel_ms and "
+                   "roofline: a replay of the same step with CUDA events around each call, after each "
+                   "timed step; e2e: plain API calls"),
         "clocks": clocks,
     }
     if not args.no_cpu_baseline and world == 1:

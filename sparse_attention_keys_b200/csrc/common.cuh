@@ -325,6 +325,18 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ------------------------------------------------------------------- bulk (TMA engine) stores
+// Copies `bytes` (a multiple of 16; both addresses 16-byte aligned) from shared to global memory.
+// The shared-memory source must be made visible to the async proxy first (fence_proxy_async_smem).
+__device__ __forceinline__ void bulk_store_s2g(void* dst_global, uint32_t src_smem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst_global), "r"(src_smem),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until this thread's committed bulk stores are complete (source read, global writes done).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 }  // namespace dsa
 
 // Host-side launch helpers shared by the entry points (defined in dsa_abi.cu).

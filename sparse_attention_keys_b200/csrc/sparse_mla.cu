@@ -490,55 +490,55 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     const bool have_o = ntiles > 0 && ok &&
                         __all_sync(0xffffffffu, mbar_wait(o_full, 0, &abort_flag, p.status, DSA_SITE_MLA_O_FULL));
     if (have_o) tc_fence_after();
-    // Stage this CTA's 128 x 256 output block in the (now idle) KV rings, one padded 1040-byte row
-    // per head (thread), then copy it out with each warp writing 512 contiguous bytes per store
-    // (a row per thread would scatter every warp store over 32 rows).
+    // Each thread stages its head's row of this CTA's 256 output features (bf16 output, or the fp32
+    // partial of a key split) in the now idle KV rings, then one bulk copy (TMA engine) per row
+    // writes it out: the row is contiguous in global memory.
     const bool final_out = p.nsplit == 1;
     const float scale = final_out ? (l > 0.f ? 1.f / l : 0.f) : 1.f;
-    float* stage = reinterpret_cast<float*>(smem + kOffV);
-    {
-      float4* srow = reinterpret_cast<float4*>(stage + h * kStageRow);
+    uint8_t* srow = smem + kOffV + h * kStageRow * 4;
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        uint32_t o[32];
-        if (have_o) {
-          tmem_ld32(t_row + kTmemO + c * 32, o);
-          tmem_ld_wait();
+    for (int c = 0; c < 8; c += 2) {
+      uint32_t o[2][32];
+      if (have_o) {
+        tmem_ld32(t_row + kTmemO + c * 32, o[0]);
+        tmem_ld32(t_row + kTmemO + (c + 1) * 32, o[1]);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[0][i] = o[1][i] = 0u;
+      }
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int f0 = (c + hh) * 32;                 // first feature of this 32-column chunk
+        if (final_out) {
+          uint4* dst = reinterpret_cast<uint4*>(srow + f0 * 2);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t* v = &o[hh][8 * i];
+            dst[i] = make_uint4(pack_bf16(__uint_as_float(v[0]) * scale, __uint_as_float(v[1]) * scale),
+                                pack_bf16(__uint_as_float(v[2]) * scale, __uint_as_float(v[3]) * scale),
+                                pack_bf16(__uint_as_float(v[4]) * scale, __uint_as_float(v[5]) * scale),
+                                pack_bf16(__uint_as_float(v[6]) * scale, __uint_as_float(v[7]) * scale));
+          }
         } else {
+          uint4* dst = reinterpret_cast<uint4*>(srow + f0 * 4);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0u;
+          for (int i = 0; i < 8; ++i) dst[i] = make_uint4(o[hh][4 * i], o[hh][4 * i + 1], o[hh][4 * i + 2], o[hh][4 * i + 3]);
         }
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          srow[c * 8 + i] = make_float4(__uint_as_float(o[4 * i]) * scale, __uint_as_float(o[4 * i + 1]) * scale,
-                                        __uint_as_float(o[4 * i + 2]) * scale, __uint_as_float(o[4 * i + 3]) * scale);
       }
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxWarps * 32) : "memory");   // the softmax warps only
+    fence_proxy_async_smem();                          // the row's generic writes -> the bulk copy's reads
     if (final_out) {
-      // bf16 out[bt][head][256*half + ...]: 32 chunks of 8 features per head row
-      for (int i = tid; i < kHeads * 32; i += kSoftmaxWarps * 32) {
-        const int r = i >> 5, c = i & 31;
-        const float4* src = reinterpret_cast<const float4*>(stage + r * kStageRow + c * 8);
-        const float4 u = src[0], v = src[1];
-        *reinterpret_cast<uint4*>(p.out + (bt * kHeads + r) * kDv + 256 * half + c * 8) =
-            make_uint4(pack_bf16(u.x, u.y), pack_bf16(u.z, u.w), pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
-      }
+      bulk_store_s2g(p.out + (bt * kHeads + h) * kDv + 256 * half, smem_u32(srow), 256 * 2);
       if (p.lse && half == 0)
         p.lse[bt * kHeads + h] = l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
     } else {
-      // fp32 partial O[bt][split][head][256*half + ...]: 64 chunks of 4 features per head row
-      for (int i = tid; i < kHeads * 64; i += kSoftmaxWarps * 32) {
-        const int r = i >> 6, c = i & 63;
-        const int64_t prow = (bt * p.nsplit + split) * kHeads + r;
-        *reinterpret_cast<float4*>(p.part_o + prow * kDv + 256 * half + c * 4) =
-            *reinterpret_cast<const float4*>(stage + r * kStageRow + c * 4);
-      }
-      if (half == 0) {
-        const int64_t prow = (bt * p.nsplit + split) * kHeads + h;
-        *reinterpret_cast<float2*>(p.part_ml + prow * 2) = make_float2(m, l);
-      }
+      const int64_t prow = (bt * p.nsplit + split) * kHeads + h;
+      bulk_store_s2g(p.part_o + prow * kDv + 256 * half, smem_u32(srow), 256 * 4);
+      if (half == 0) *reinterpret_cast<float2*>(p.part_ml + prow * 2) = make_float2(m, l);
     }
+    bulk_commit();
+    bulk_wait_all();                                   // shared memory stays valid until the copy is done
   }
 
   tc_fence_before();
@@ -549,34 +549,55 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   }
 }
 
-// Merge the key-split partials: one warp per (query, head), 16 output features per lane.
+// Merge the key-split partials: one warp per (query, head), 16 output features per lane. The
+// splits' (max, sum) pairs are read one per lane and reduced across the warp; the partial O rows
+// are then streamed four splits at a time so that their loads overlap.
 __global__ void __launch_bounds__(256) sparse_mla_combine_kernel(const MlaParams p, int64_t rows) {
   const int64_t wid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (wid >= rows) return;
   const int64_t bt = wid / kHeads;
   const int head = (int)(wid - bt * kHeads);
+  const float2* ml = reinterpret_cast<const float2*>(p.part_ml);
+  auto ml_of = [&](int s) { return __ldg(ml + (bt * p.nsplit + s) * kHeads + head); };
   float m_all = -INFINITY;
-  for (int s = 0; s < p.nsplit; ++s) {
-    const float m = p.part_ml[((bt * p.nsplit + s) * kHeads + head) * 2];
-    m_all = fmaxf(m_all, m);
+  for (int s = lane; s < p.nsplit; s += 32) m_all = fmaxf(m_all, ml_of(s).x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m_all = fmaxf(m_all, __shfl_xor_sync(0xffffffffu, m_all, o));
+  auto weight = [&](float m) { return m == -INFINITY ? 0.f : exp2f(m - m_all); };
+  float l_all = 0.f;
+  for (int s = lane; s < p.nsplit; s += 32) {
+    const float2 v = ml_of(s);
+    l_all += v.y * weight(v.x);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l_all += __shfl_xor_sync(0xffffffffu, l_all, o);
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  float l_all = 0.f;
-  for (int s = 0; s < p.nsplit; ++s) {
-    const int64_t prow = (bt * p.nsplit + s) * kHeads + head;
-    const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + prow * 2);
-    if (ml.x == -INFINITY) continue;
-    const float wgt = exp2f(ml.x - m_all);
-    l_all += ml.y * wgt;
-    const float4* src = reinterpret_cast<const float4*>(p.part_o + prow * kDv + lane * 16);
+  for (int s0 = 0; s0 < p.nsplit; s0 += 4) {
+    float4 v[4][4];
+    float wgt[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 v = src[i];
-      acc[4 * i] += v.x * wgt; acc[4 * i + 1] += v.y * wgt;
-      acc[4 * i + 2] += v.z * wgt; acc[4 * i + 3] += v.w * wgt;
+    for (int u = 0; u < 4; ++u) {
+      const int s = s0 + u;
+      wgt[u] = 0.f;
+      if (s < p.nsplit) {
+        wgt[u] = weight(ml_of(s).x);
+        const float4* src =
+            reinterpret_cast<const float4*>(p.part_o + ((bt * p.nsplit + s) * kHeads + head) * kDv + lane * 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[u][i] = __ldcs(src + i);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (wgt[u] == 0.f) continue;       // split with no selected key (or beyond nsplit)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[4 * i] += v[u][i].x * wgt[u]; acc[4 * i + 1] += v[u][i].y * wgt[u];
+        acc[4 * i + 2] += v[u][i].z * wgt[u]; acc[4 * i + 3] += v[u][i].w * wgt[u];
+      }
     }
   }
   const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
