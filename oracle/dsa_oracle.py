@@ -357,6 +357,63 @@ def dense_mla(q_bits, kv_bits, q_pos, kv_len, softmax_scale: float = MLA_SOFTMAX
     return sparse_mla(q_bits, kv_bits, idx, softmax_scale, d_v)
 
 
+# ----------------------------------------------------------------------------------------------
+# Producers of the sparse-MLA inputs and the output absorption (absorbed MQA form)
+# ----------------------------------------------------------------------------------------------
+def rope_interleaved(x, pos, table) -> np.ndarray:
+    """Rotate feature pairs (2i, 2i+1) by pair i's angle: apply_rotary_emb with interleaved=True,
+    the layout the MLA uses for q_pe and k_pe (Rotate first features page: attention pairs 2j with
+    2j+1, the indexer j with j+32). x [..., 64], pos broadcastable to x.shape[:-1]; float64 out.
+
+    READING: the excerpt widens the bf16 input to fp32 and multiplies complex64 numbers; the
+    oracle rotates in float64 (the difference is far below the bf16 rounding of the result).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    cs = np.asarray(table, dtype=np.float64)[np.asarray(pos)]     # [..., 32, 2]
+    c, s = cs[..., 0], cs[..., 1]
+    re, im = x[..., 0::2], x[..., 1::2]
+    y = np.empty_like(x)
+    y[..., 0::2] = re * c - im * s
+    y[..., 1::2] = re * s + im * c
+    return y
+
+
+def mla_q_absorb(q_nope_bits, q_pe_bits, pos, table, w_uk_bits) -> np.ndarray:
+    """The sparse-MLA query [rows, H, 576]: features 0..511 are q_nope absorbed into the latent
+    space, q[t,h,c] = sum_d q_nope[t,h,d] w_uk[h,d,c] (the MQA-decode excerpt's einsum of q_nope
+    with wkv_b[:, :qk_nope_head_dim]); features 512..575 are q_pe rotated at pos[t] (interleaved).
+
+    q_nope_bits bf16 [rows, H, 128], q_pe_bits bf16 [rows, H, 64], pos [rows],
+    w_uk_bits bf16 [H, 128, 512]. float64 out (the CUDA path rounds it to bf16).
+    """
+    qn = bf16_to_f64(q_nope_bits)
+    w = bf16_to_f64(w_uk_bits)
+    lat = np.einsum("thd,hdc->thc", qn, w)
+    rot = rope_interleaved(bf16_to_f64(q_pe_bits), np.asarray(pos)[:, None], table)
+    return np.concatenate([lat, rot], axis=-1)
+
+
+def mla_kv_entry(kv_bits, k_pe_bits, pos, table) -> np.ndarray:
+    """One latent-cache row per token [rows, 576]: the (normalised) latent kv unchanged, then k_pe
+    rotated at pos (interleaved) -- the rows the MQA-decode excerpt reads from kv_cache and
+    pe_cache, kept side by side. float64 out."""
+    return np.concatenate([bf16_to_f64(kv_bits),
+                           rope_interleaved(bf16_to_f64(k_pe_bits), np.asarray(pos), table)], axis=-1)
+
+
+def mla_out_absorb(o_bits, w_uv_bits) -> np.ndarray:
+    """Per-head value up-projection of the attention output, x[t,h,d] = sum_c o[t,h,c] w_uv[h,d,c]
+    (the excerpt's final einsum with wkv_b[:, -v_head_dim:]). o_bits bf16 [rows, H, 512],
+    w_uv_bits bf16 [H, 128, 512]; float64 [rows, H, 128] out."""
+    return np.einsum("thc,hdc->thd", bf16_to_f64(o_bits), bf16_to_f64(w_uv_bits))
+
+
+def gemm_abs_terms(a, b, spec: str) -> np.ndarray:
+    """sum over the contracted index of |a * b| for an einsum spec: the scale an fp32
+    accumulation's rounding error is measured against."""
+    return np.einsum(spec, np.abs(np.asarray(a, np.float64)), np.abs(np.asarray(b, np.float64)))
+
+
 def paged_gather(pool, block_table, page_size: int, seq_len) -> np.ndarray:
     """Dense per-sequence view [B, max_pages * page_size, ...] of a paged cache.
 

@@ -419,3 +419,89 @@ def test_paged_gather_rejects_a_visible_bad_page():
     with pytest.raises(IndexError):
         O.paged_gather(pool, np.array([[0, 4]]), 2, [3])      # position 2 lives on page 4 of 4
     O.paged_gather(pool, np.array([[0, 4]]), 2, [2])          # ... unless it is past the end
+
+
+# ---------------------------------------------------------------------------- MLA producers
+def _bf16_bits(x):
+    return torch.from_numpy(np.asarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_rope_interleaved_is_the_regrouped_noninterleaved_rotation():
+    # the excerpt's interleaved=False path regroups the halves into pairs, rotates, and restores
+    # the halves: so rotating the de-interleaved vector the non-interleaved way and interleaving
+    # the result back must give the interleaved rotation
+    rng = np.random.default_rng(3)
+    table = O.rope_table(5000)
+    x = rng.standard_normal((6, 64))
+    pos = np.array([0, 1, 17, 1000, 4095, 4999])
+    halves = np.concatenate([x[:, 0::2], x[:, 1::2]], axis=1)
+    y = O.rope_noninterleaved(halves, pos, table)
+    back = np.empty_like(x)
+    back[:, 0::2], back[:, 1::2] = y[:, :32], y[:, 32:]
+    assert np.allclose(O.rope_interleaved(x, pos, table), back, rtol=0, atol=1e-12)
+
+
+def test_rope_interleaved_complex_product_and_norms():
+    rng = np.random.default_rng(4)
+    table = O.rope_table(3000)
+    x = rng.standard_normal((5, 64))
+    pos = np.array([0, 3, 100, 2047, 2999])
+    got = O.rope_interleaved(x, pos, table)
+    z = (x[:, 0::2] + 1j * x[:, 1::2]) * (table[pos, :, 0] + 1j * table[pos, :, 1]).astype(np.complex128)
+    assert np.allclose(got[:, 0::2], z.real, atol=1e-12) and np.allclose(got[:, 1::2], z.imag, atol=1e-12)
+    pair_norm = lambda v: np.hypot(v[:, 0::2], v[:, 1::2])
+    assert np.allclose(pair_norm(got), pair_norm(x), rtol=1e-6)
+    assert np.array_equal(got[0], x[0])                          # position 0: cos 1, sin 0
+
+
+def test_q_absorb_gives_the_unabsorbed_scores():
+    # MHA prefill path: k_nope[s,h,d] = sum_c w[h,d,c] kv[s,c] (wkv_b up-projection), score =
+    # q_nope . k_nope; the absorbed query must give the same latent score q_abs . kv
+    rng = np.random.default_rng(5)
+    H, D, C, T, S = 2, 3, 5, 2, 4
+    qn = _bf16_bits(rng.standard_normal((T, H, D)))
+    qp = _bf16_bits(rng.standard_normal((T, H, 64)))
+    w = _bf16_bits(rng.standard_normal((H, D, C)))
+    kv = O.bf16_to_f64(_bf16_bits(rng.standard_normal((S, C))))
+    table = O.rope_table(16)
+    q = O.mla_q_absorb(qn, qp, np.array([3, 9]), table, w)
+    qn64, w64 = O.bf16_to_f64(qn), O.bf16_to_f64(w)
+    for t in range(T):
+        for h in range(H):
+            for s in range(S):
+                k_nope = [sum(w64[h, d, c] * kv[s, c] for c in range(C)) for d in range(D)]
+                want = sum(qn64[t, h, d] * k_nope[d] for d in range(D))
+                assert math.isclose(sum(q[t, h, c] * kv[s, c] for c in range(C)), want, rel_tol=1e-12, abs_tol=1e-12)
+    assert np.allclose(q[..., C:], O.rope_interleaved(O.bf16_to_f64(qp), np.array([[3], [9]]), table), atol=0)
+
+
+def test_out_absorb_gives_the_unabsorbed_values():
+    # MHA prefill path: v[s,h,d] = sum_c w_uv[h,d,c] kv[s,c]; out = sum_s p_s v[s]. The absorbed
+    # form up-projects the latent mix o = sum_s p_s kv[s] instead
+    rng = np.random.default_rng(6)
+    H, D, C, S = 2, 3, 4, 5
+    kv = rng.standard_normal((S, C))
+    p = rng.random((H, S))
+    p /= p.sum(axis=1, keepdims=True)
+    w = _bf16_bits(rng.standard_normal((H, D, C)))
+    o = np.einsum("hs,sc->hc", p, kv)
+    ob = _bf16_bits(o)[None]                                    # [1, H, C]
+    got = O.mla_out_absorb(ob, w)[0]
+    o64, w64 = O.bf16_to_f64(ob)[0], O.bf16_to_f64(w)
+    for h in range(H):
+        for d in range(D):
+            assert math.isclose(got[h, d], sum(o64[h, c] * w64[h, d, c] for c in range(C)), rel_tol=1e-12)
+            v = [sum(w64[h, d, c] * kv[s, c] for c in range(C)) for s in range(S)]
+            exact = sum(p[h, s] * v[s] for s in range(S))
+            assert abs(got[h, d] - exact) <= 2 ** -7 * sum(abs(o[h, c] * w64[h, d, c]) for c in range(C))
+
+
+def test_kv_entry_keeps_the_latent_and_rotates_the_rope_key():
+    rng = np.random.default_rng(7)
+    kv = _bf16_bits(rng.standard_normal((3, 512)))
+    kp = _bf16_bits(rng.standard_normal((3, 64)))
+    table = O.rope_table(64)
+    row = O.mla_kv_entry(kv, kp, np.array([0, 5, 63]), table)
+    assert np.array_equal(row[:, :512], O.bf16_to_f64(kv))
+    assert np.array_equal(row[0, 512:], O.bf16_to_f64(kp)[0])
+    assert np.allclose(row[1:, 512:], O.rope_interleaved(O.bf16_to_f64(kp)[1:], np.array([5, 63]), table), atol=0)
