@@ -194,3 +194,29 @@ def to_paged(dense: np.ndarray, block_table: np.ndarray, page_size: int, num_pag
             if 0 <= dst < num_pages:
                 pool[dst * page_size:(dst + 1) * page_size] = dense[b, pg * page_size:(pg + 1) * page_size]
     return pool
+
+
+@dataclass
+class MlaProducerInputs:
+    """Inputs of the MLA producers and output absorption for ``rows`` tokens (bf16 bit patterns)."""
+    q_nope: np.ndarray    # [rows, 128, 128]
+    q_pe: np.ndarray      # [rows, 128, 64]
+    kv: np.ndarray        # [rows, 512]  (the normalised latent)
+    k_pe: np.ndarray      # [rows, 64]
+    o: np.ndarray         # [rows, 128, 512]  (a sparse-MLA output)
+    wkv_b: np.ndarray     # [128, 256, 512]: rows 0..127 of each head are w_uk, 128..255 w_uv
+    pos: np.ndarray       # int32 [rows]
+
+
+def make_mla_producer_inputs(rows: int, seed: int = 0, max_pos: int = MAX_SEQ_LEN) -> MlaProducerInputs:
+    """N(0,1) activations, wkv_b ~ N(0, 1/512) (unit-scale outputs), positions uniform in [0, max_pos).
+    Draw order: q_nope, q_pe, kv, k_pe, o, wkv_b, pos."""
+    rng = np.random.default_rng(seed)
+    q_nope = bf16_bits_from_f32(_normal_f32(rng, (rows, H_MLA, 128)))
+    q_pe = bf16_bits_from_f32(_normal_f32(rng, (rows, H_MLA, D_ROPE)))
+    kv = bf16_bits_from_f32(_normal_f32(rng, (rows, D_LATENT)))
+    k_pe = bf16_bits_from_f32(_normal_f32(rng, (rows, D_ROPE)))
+    o = bf16_bits_from_f32(_normal_f32(rng, (rows, H_MLA, D_LATENT)))
+    wkv_b = bf16_bits_from_f32(_normal_f32(rng, (H_MLA, 256, D_LATENT)) * np.float32(D_LATENT ** -0.5))
+    pos = rng.integers(0, max_pos, size=rows).astype(np.int32)
+    return MlaProducerInputs(q_nope, q_pe, kv, k_pe, o, wkv_b, pos)

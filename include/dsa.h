@@ -233,6 +233,40 @@ DSA_API int dsa_sparse_mla_paged(const uint16_t* q, const uint16_t* kv_pool, int
                                  uint16_t* out, float* lse, void* workspace, size_t ws_bytes,
                                  dsa_stream_t stream);
 
+/*
+ * Producers of the sparse-MLA inputs and the output absorption (absorbed MQA form). Source: the
+ * "Similarities" page, MQA-decode excerpt (q_nope times wkv_b[:, :qk_nope_head_dim]; the latent
+ * and rotary caches; the latent-weighted sum times wkv_b[:, -v_head_dim:]); the "Rotate first
+ * features" page (MLA RoPE pairs features 2j and 2j+1, the interleaved layout). bf16 in and out,
+ * fp32 arithmetic. Weights: head h's [128][512] matrix starts w_head_stride elements after head
+ * h-1's (rows of 512 contiguous): w_uk = wkv_b, w_uv = wkv_b + 128*512, stride 256*512 for the
+ * reference's wkv_b viewed as [128 heads][256][512]. Pointers 16-byte aligned; w_head_stride a
+ * multiple of 8 and >= 128*512; rows >= 0 (0: nothing to do); rows >= 2^31 is rejected.
+ */
+
+/* q_out[t][h][0:512] = sum_d q_nope[t][h][d] * w_uk[h][d][0:512];
+ * q_out[t][h][512:576] = interleaved RoPE_64 of q_pe[t][h] at pos[t] (rope_cs as dsa_index_keys).
+ *   q_nope bf16 [rows][128][128], q_pe bf16 [rows][128][64], pos int32 [rows] in [0, max_pos),
+ *   q_out bf16 [rows][128][576] -- the q argument of dsa_sparse_mla.
+ * A position outside the table sets DSA_ERR_DEVICE_BOUNDS (that row's rotary part is zero). */
+DSA_API int dsa_mla_q_absorb(const uint16_t* q_nope, const uint16_t* q_pe, const int32_t* pos,
+                             const float* rope_cs, int max_pos, const uint16_t* w_uk, int64_t w_head_stride,
+                             int64_t rows, uint16_t* q_out, dsa_stream_t stream);
+
+/* Latent-cache write: kv_cache[dst_row[t]][0:512] = kv[t] (the normalised latent, copied) and
+ * kv_cache[dst_row[t]][512:576] = interleaved RoPE_64 of k_pe[t] at pos[t].
+ *   kv bf16 [rows][512], k_pe bf16 [rows][64], pos int32 [rows], dst_row int64 [rows] in
+ *   [0, cache_rows), kv_cache bf16 [cache_rows][576] (dense [B][S_max][576] with row b*S_max+s, or a
+ *   paged pool). A bad dst_row or position skips the row and sets DSA_ERR_DEVICE_BOUNDS. */
+DSA_API int dsa_mla_kv_entry(const uint16_t* kv, const uint16_t* k_pe, const int32_t* pos,
+                             const float* rope_cs, int max_pos, int64_t rows, const int64_t* dst_row,
+                             uint16_t* kv_cache, int64_t cache_rows, dsa_stream_t stream);
+
+/* out[t][h][0:128] = sum_c o[t][h][c] * w_uv[h][0:128][c].
+ *   o bf16 [rows][128][512] (dsa_sparse_mla's out), out bf16 [rows][128][128]. */
+DSA_API int dsa_mla_out_absorb(const uint16_t* o, const uint16_t* w_uv, int64_t w_head_stride, int64_t rows,
+                               uint16_t* out, dsa_stream_t stream);
+
 /* Bytes of device scratch dsa_sparse_mla needs for this shape (0 when it needs none). */
 DSA_API size_t dsa_sparse_mla_workspace_size(int B, int T, int k);
 
@@ -261,6 +295,11 @@ DSA_API int dsa_get_device_status(dsa_stream_t stream);
 #define DSA_SITE_MLA_P_EMPTY 0x26       /* sparse MLA: softmax waits for P V before rescaling O  */
 #define DSA_SITE_MLA_O_FULL 0x27        /* sparse MLA: epilogue waits for the last P V           */
 #define DSA_SITE_SELFTEST 0x31          /* dsa_selftest_wait_timeout                             */
+#define DSA_SITE_ABSORB_W 0x41          /* MLA absorption: MMA waits for the resident weights    */
+#define DSA_SITE_ABSORB_A_FULL 0x42     /* MLA absorption: MMA waits for an activation stage     */
+#define DSA_SITE_ABSORB_A_EMPTY 0x43    /* MLA absorption: TMA waits for a free stage            */
+#define DSA_SITE_ABSORB_ACC_FULL 0x44   /* MLA absorption: epilogue waits for an accumulator     */
+#define DSA_SITE_ABSORB_ACC_EMPTY 0x45  /* MLA absorption: MMA waits for a drained accumulator   */
 
 /*
  * dsa_get_error_detail - the detail recorded with the last non-OK code that

@@ -16,7 +16,8 @@ __all__ = [
     "DsaError", "lib", "lib_path", "DSA_HADAMARD", "DSA_FILL_MASKED", "DSA_SORTED", "DSA_F32", "DSA_BF16", "INDEXER_SOFTMAX_SCALE",
     "MLA_SOFTMAX_SCALE", "dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk",
     "dsa_sparse_mla", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_noalloc",
-    "dsa_index_scores_paged", "dsa_sparse_mla_paged",
+    "dsa_index_scores_paged", "dsa_sparse_mla_paged", "dsa_mla_q_absorb", "dsa_mla_kv_entry",
+    "dsa_mla_out_absorb",
     "dsa_sparse_mla_noalloc_scratch_bytes", "dsa_get_device_status", "dsa_get_error_detail",
     "dsa_selftest_wait_timeout", "dsa_status_string", "dsa_device_supported", "dsa_version",
     "SITE_NAMES",
@@ -37,7 +38,8 @@ SITE_NAMES = {
     0x11: "scores:q", 0x12: "scores:k_full", 0x13: "scores:k_empty", 0x14: "scores:acc_full",
     0x15: "scores:acc_empty", 0x21: "mla:q", 0x22: "mla:kv_full", 0x23: "mla:kv_empty",
     0x24: "mla:s_full", 0x25: "mla:p_full", 0x26: "mla:p_empty", 0x27: "mla:o_full",
-    0x31: "selftest",
+    0x31: "selftest", 0x41: "absorb:w", 0x42: "absorb:a_full", 0x43: "absorb:a_empty",
+    0x44: "absorb:acc_full", 0x45: "absorb:acc_empty",
 }
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -65,6 +67,9 @@ def _load():
     L.dsa_index_scores_paged.argtypes = [vp, vp, vp, vp, vp, i64, vp, i32, i32, vp, vp, i32, i32, f32, vp, i64, u32,
                                          vp]
     L.dsa_sparse_mla_paged.argtypes = [vp, vp, i64, vp, i32, i32, vp, i32, i32, i32, f32, vp, vp, vp, sz, vp]
+    L.dsa_mla_q_absorb.argtypes = [vp, vp, vp, vp, i32, vp, i64, i64, vp, vp]
+    L.dsa_mla_kv_entry.argtypes = [vp, vp, vp, vp, i32, i64, vp, vp, i64, vp]
+    L.dsa_mla_out_absorb.argtypes = [vp, vp, i64, i64, vp, vp]
     L.dsa_sparse_mla_workspace_size.restype = sz
     L.dsa_sparse_mla_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp]
     L.dsa_sparse_mla_noalloc_scratch_bytes.argtypes = []
@@ -282,6 +287,62 @@ def dsa_sparse_mla_paged(q, kv_pool, block_table, page_size: int, idx, softmax_s
                                    _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
     _check(rc, "dsa_sparse_mla_paged")
     return out, lse
+
+
+def _head_weights(w, name):
+    """A [128 heads][128][512] bf16 view whose rows of 512 are contiguous (e.g. a slice of wkv_b
+    viewed as [128][256][512]) -> (tensor, elements between heads)."""
+    if not isinstance(w, torch.Tensor) or w.dtype != torch.bfloat16 or not w.is_cuda:
+        raise TypeError(f"{name} must be a bfloat16 CUDA tensor")
+    if tuple(w.shape) != (128, 128, 512) or w.stride(2) != 1 or w.stride(1) != 512:
+        raise ValueError(f"{name} must be [128, 128, 512] with contiguous rows of 512")
+    return w, int(w.stride(0))
+
+
+def dsa_mla_q_absorb(q_nope, q_pe, pos, rope_cs, w_uk, q_out=None, stream=None):
+    """q_nope bf16 [rows,128,128], q_pe bf16 [rows,128,64], pos i32 [rows], w_uk bf16 [128,128,512]
+    (head, d, c) -> the sparse-MLA query bf16 [rows,128,576] (absorbed latent part | rotated q_pe)."""
+    _need(q_nope, torch.bfloat16, "q_nope")
+    _need(q_pe, torch.bfloat16, "q_pe")
+    _need(pos, torch.int32, "pos")
+    _need(rope_cs, torch.float32, "rope_cs")
+    w, ws = _head_weights(w_uk, "w_uk")
+    rows = q_nope.shape[0]
+    if q_out is None:
+        q_out = torch.empty((rows, 128, 576), dtype=torch.bfloat16, device=q_nope.device)
+    _need(q_out, torch.bfloat16, "q_out")
+    rc = _lib.dsa_mla_q_absorb(_ptr(q_nope), _ptr(q_pe), _ptr(pos), _ptr(rope_cs), rope_cs.shape[0], _ptr(w), ws,
+                               rows, _ptr(q_out), _stream(stream))
+    _check(rc, "dsa_mla_q_absorb")
+    return q_out
+
+
+def dsa_mla_kv_entry(kv, k_pe, pos, rope_cs, dst_row, kv_cache, stream=None):
+    """Write latent-cache rows: kv_cache[dst_row[t]] = [kv[t] | interleaved RoPE of k_pe[t] at pos[t]].
+    kv bf16 [rows,512], k_pe bf16 [rows,64], dst_row i64 [rows], kv_cache bf16 [..., 576]."""
+    _need(kv, torch.bfloat16, "kv")
+    _need(k_pe, torch.bfloat16, "k_pe")
+    _need(pos, torch.int32, "pos")
+    _need(rope_cs, torch.float32, "rope_cs")
+    _need(dst_row, torch.int64, "dst_row")
+    _need(kv_cache, torch.bfloat16, "kv_cache")
+    rc = _lib.dsa_mla_kv_entry(_ptr(kv), _ptr(k_pe), _ptr(pos), _ptr(rope_cs), rope_cs.shape[0], kv.shape[0],
+                               _ptr(dst_row), _ptr(kv_cache), kv_cache.numel() // 576, _stream(stream))
+    _check(rc, "dsa_mla_kv_entry")
+    return kv_cache
+
+
+def dsa_mla_out_absorb(o, w_uv, out=None, stream=None):
+    """o bf16 [rows,128,512] (sparse-MLA output), w_uv bf16 [128,128,512] (head, d, c) -> bf16 [rows,128,128]."""
+    _need(o, torch.bfloat16, "o")
+    w, ws = _head_weights(w_uv, "w_uv")
+    rows = o.shape[0]
+    if out is None:
+        out = torch.empty((rows, 128, 128), dtype=torch.bfloat16, device=o.device)
+    _need(out, torch.bfloat16, "out")
+    rc = _lib.dsa_mla_out_absorb(_ptr(o), _ptr(w), ws, rows, _ptr(out), _stream(stream))
+    _check(rc, "dsa_mla_out_absorb")
+    return out
 
 
 def dsa_sparse_mla_noalloc_scratch_bytes() -> int:

@@ -140,6 +140,18 @@ bool encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, void* bas
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_tensor_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, void* base, const uint64_t dims[3],
+                          const uint64_t strides[2], const uint32_t box[3], CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  const cuuint64_t st[2] = {strides[0], strides[1]};
+  const cuuint32_t bx[3] = {box[0], box[1], box[2]};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, dtype, 3, base, d, st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace dsa_host
 
 // ------------------------------------------------------------------------------------------------
@@ -265,6 +277,54 @@ int dsa_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, in
   if (rc != DSA_OK) return rc;
   return dsa::launch_sparse_mla(q, kv, idx, B, T, S_max, k, softmax_scale, out, lse, workspace, ws_bytes,
                                 (cudaStream_t)stream, status);
+}
+
+static bool weights_ok(const uint16_t* w, int64_t w_head_stride) {
+  return w && dsa_host::aligned16(w) && w_head_stride >= 128 * 512 && w_head_stride % 8 == 0 &&
+         w_head_stride <= ((int64_t)1 << 40);
+}
+
+int dsa_mla_q_absorb(const uint16_t* q_nope, const uint16_t* q_pe, const int32_t* pos, const float* rope_cs,
+                     int max_pos, const uint16_t* w_uk, int64_t w_head_stride, int64_t rows, uint16_t* q_out,
+                     dsa_stream_t stream) {
+  if (rows < 0 || rows >= 0x80000000LL || max_pos < 1 || !weights_ok(w_uk, w_head_stride)) return DSA_ERR_INVALID_ARG;
+  if (!q_nope || !q_pe || !pos || !rope_cs || !q_out) return DSA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q_nope, q_pe, pos, rope_cs, q_out};
+  for (const void* p : ptrs)
+    if (!dsa_host::aligned16(p)) return DSA_ERR_INVALID_ARG;
+  if (rows == 0) return DSA_OK;
+  int* status;
+  int rc = prologue(&status);
+  if (rc != DSA_OK) return rc;
+  return dsa::launch_mla_q_absorb(q_nope, q_pe, pos, rope_cs, max_pos, w_uk, w_head_stride, rows, q_out,
+                                  (cudaStream_t)stream, status);
+}
+
+int dsa_mla_kv_entry(const uint16_t* kv, const uint16_t* k_pe, const int32_t* pos, const float* rope_cs,
+                     int max_pos, int64_t rows, const int64_t* dst_row, uint16_t* kv_cache, int64_t cache_rows,
+                     dsa_stream_t stream) {
+  if (rows < 0 || rows >= 0x80000000LL || max_pos < 1 || cache_rows < 1) return DSA_ERR_INVALID_ARG;
+  if (!kv || !k_pe || !pos || !rope_cs || !dst_row || !kv_cache) return DSA_ERR_INVALID_ARG;
+  const void* ptrs[] = {kv, k_pe, pos, rope_cs, dst_row, kv_cache};
+  for (const void* p : ptrs)
+    if (!dsa_host::aligned16(p)) return DSA_ERR_INVALID_ARG;
+  if (rows == 0) return DSA_OK;
+  int* status;
+  int rc = prologue(&status);
+  if (rc != DSA_OK) return rc;
+  return dsa::launch_mla_kv_entry(kv, k_pe, pos, rope_cs, max_pos, rows, dst_row, kv_cache, cache_rows,
+                                  (cudaStream_t)stream, status);
+}
+
+int dsa_mla_out_absorb(const uint16_t* o, const uint16_t* w_uv, int64_t w_head_stride, int64_t rows, uint16_t* out,
+                       dsa_stream_t stream) {
+  if (rows < 0 || rows >= 0x80000000LL || !weights_ok(w_uv, w_head_stride)) return DSA_ERR_INVALID_ARG;
+  if (!o || !out || !dsa_host::aligned16(o) || !dsa_host::aligned16(out)) return DSA_ERR_INVALID_ARG;
+  if (rows == 0) return DSA_OK;
+  int* status;
+  int rc = prologue(&status);
+  if (rc != DSA_OK) return rc;
+  return dsa::launch_mla_out_absorb(o, w_uv, w_head_stride, rows, out, (cudaStream_t)stream, status);
 }
 
 // Shared checks of the paged-cache arguments: page ids are int32 and pool rows index int32.

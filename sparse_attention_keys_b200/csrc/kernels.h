@@ -30,6 +30,14 @@ int launch_sparse_mla_paged(const uint16_t* q, const uint16_t* kv_pool, int64_t 
                             const int32_t* block_table, int max_pages, int page_size, const int32_t* idx, int B,
                             int T, int k, float softmax_scale, uint16_t* out, float* lse, void* workspace,
                             size_t ws_bytes, cudaStream_t stream, int* status);
+int launch_mla_q_absorb(const uint16_t* q_nope, const uint16_t* q_pe, const int32_t* pos, const float* rope_cs,
+                        int max_pos, const uint16_t* w_uk, int64_t w_head_stride, int64_t rows, uint16_t* q_out,
+                        cudaStream_t stream, int* status);
+int launch_mla_kv_entry(const uint16_t* kv, const uint16_t* k_pe, const int32_t* pos, const float* rope_cs,
+                        int max_pos, int64_t rows, const int64_t* dst_row, uint16_t* kv_cache, int64_t cache_rows,
+                        cudaStream_t stream, int* status);
+int launch_mla_out_absorb(const uint16_t* o, const uint16_t* w_uv, int64_t w_head_stride, int64_t rows,
+                          uint16_t* out, cudaStream_t stream, int* status);
 int launch_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T,
                       int S_max, int k, float softmax_scale, uint16_t* out, float* lse,
                       void* workspace, size_t ws_bytes, cudaStream_t stream, int* status);

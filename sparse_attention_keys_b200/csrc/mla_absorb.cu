@@ -1,0 +1,496 @@
+// Producers and output projection of the sparse MLA in its absorbed (MQA) form.
+//
+//   q_absorb   q[t][h][0:512]   = sum_d q_nope[t][h][d] * w_uk[h][d][0:512]        (bf16 MMA, fp32 acc)
+//              q[t][h][512:576] = interleaved RoPE_64 of q_pe[t][h] at pos[t]
+//   kv_entry   cache[dst][0:512] = kv[t];  cache[dst][512:576] = interleaved RoPE_64 of k_pe[t]
+//   out_absorb x[t][h][0:128]   = sum_c o[t][h][c] * w_uv[h][0:128][c]
+//
+// "DeepSeek-V3.2-Exp - Similarities" page, MQA-decode excerpt: q_nope is multiplied into the latent
+// space by wkv_b[:, :qk_nope_head_dim], scores combine the latent and rotary caches, and the
+// latent-weighted sum is projected by wkv_b[:, -v_head_dim:]; "Rotate first features" page: MLA
+// RoPE pairs features 2j and 2j+1. The q_absorb and out_absorb GEMMs stream their activations once
+// and are bound by memory (at decode by the 16.8 MB of weights each reads): TMA tiles with 128-byte
+// swizzle, tcgen05 MMAs from shared memory into a double-buffered TMEM accumulator, and one bulk
+// copy (TMA engine) per output row.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dsa {
+namespace {
+
+constexpr int kHeadsA = 128;       // MLA heads
+constexpr int kNope = 128;         // qk_nope_head_dim
+constexpr int kLat = 512;          // kv_lora_rank
+constexpr int kRopeD = 64;         // qk_rope_head_dim
+constexpr int kVd = 128;           // v_head_dim
+constexpr int kQk = kLat + kRopeD;  // 576
+constexpr int kRows = 128;         // rows (tokens) per tile = MMA M = TMEM lanes
+constexpr int kThreads = 192;      // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue
+constexpr int kRegion = 16384;     // one 128-row x 128-byte swizzled tile region
+
+struct AbsorbParams {
+  const uint16_t* q_pe;      // q_absorb: [rows][128][64]
+  const int32_t* pos;        // q_absorb: [rows]
+  const float* rope_cs;      // [max_pos][32][2]
+  int max_pos;
+  int64_t rows;
+  int tiles_per_cta;         // row tiles each CTA runs (for one head and one output part)
+  uint16_t* out;             // q_absorb [rows][128][576]; out_absorb [rows][128][128]
+  int* status;
+};
+
+// 8 packed bf16 pairs (2i, 2i+1) rotated by the (cos, sin) of pairs p0..p0+3 of a table row.
+__device__ __forceinline__ uint4 rope_pairs4(uint4 x, const float4* cs2) {
+  const float4 c01 = __ldg(cs2), c23 = __ldg(cs2 + 1);       // (cos, sin) of 4 pairs
+  const float cs[8] = {c01.x, c01.y, c01.z, c01.w, c23.x, c23.y, c23.z, c23.w};
+  const uint32_t in[4] = {x.x, x.y, x.z, x.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float a = __uint_as_float(in[i] << 16), b = __uint_as_float(in[i] & 0xFFFF0000u);
+    const float c = cs[2 * i], s = cs[2 * i + 1];
+    o[i] = pack_bf16(__fsub_rn(__fmul_rn(a, c), __fmul_rn(b, s)), __fadd_rn(__fmul_rn(a, s), __fmul_rn(b, c)));
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Interleaved RoPE of one 64-feature row (128 B at src) into dst (16-byte aligned). Returns false
+// (and writes zeros) for a position outside the table.
+__device__ __forceinline__ bool rope_row(const uint16_t* src, int pos, const AbsorbParams& p, uint4* dst) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+  if (pos < 0 || pos >= p.max_pos) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+    return false;
+  }
+  const float4* cs = reinterpret_cast<const float4*>(p.rope_cs + (int64_t)pos * kRopeD);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) dst[i] = rope_pairs4(__ldg(s4 + i), cs + 2 * i);
+  return true;
+}
+
+// fp32 TMEM columns -> bf16 in shared memory: 32 columns become 64 bytes
+__device__ __forceinline__ void store_bf16_32(uint8_t* dst, const uint32_t (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t* w = &v[8 * i];
+    d[i] = make_uint4(pack_bf16(__uint_as_float(w[0]), __uint_as_float(w[1])),
+                      pack_bf16(__uint_as_float(w[2]), __uint_as_float(w[3])),
+                      pack_bf16(__uint_as_float(w[4]), __uint_as_float(w[5])),
+                      pack_bf16(__uint_as_float(w[6]), __uint_as_float(w[7])));
+  }
+}
+
+// ------------------------------------------------------------------------------------ q_absorb
+// CTA = (group of row tiles, head h, output part n): latent features [256n, 256n + 256) of head h,
+// the part n = 1 also writes the rotated q_pe (features 512..575 follow its 256 features).
+// Shared memory: w_uk[h][:, 256n : 256n+256] as 4 MN-major regions (64 c x 128 d rows), resident;
+// two stages of the q_nope tile (2 K-major regions of 128 rows x 64 d); a staging row per tile row.
+namespace qa {
+constexpr int kOffB = 0;
+constexpr int kOffA = 4 * kRegion;
+constexpr int kAStage = 2 * kRegion;
+constexpr int kRowBytes = 656;                        // 640 B (256 + 64 bf16) + 16 B pad
+constexpr int kOffStage = kOffA + 2 * kAStage;
+constexpr int kOffBar = kOffStage + kRows * kRowBytes;
+constexpr int kSmemBytes = kOffBar + 128 + 1024;       // + alignment slack
+constexpr int kTmemCols = 512;                        // two 128 x 256 fp32 accumulators
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+}  // namespace qa
+
+__global__ void __launch_bounds__(kThreads, 1)
+    q_absorb_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constant__ CUtensorMap w_map,
+                    const AbsorbParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + qa::kOffBar);
+  uint64_t* b_full = bars;               // weights landed
+  uint64_t* a_full = bars + 1;           // [2] q_nope tile landed
+  uint64_t* a_empty = bars + 3;          // [2] MMAs done reading the tile
+  uint64_t* acc_full = bars + 5;         // [2] accumulator ready
+  uint64_t* acc_empty = bars + 7;        // [2] accumulator drained (128 arrivals)
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x & 1;
+  const int h = (blockIdx.x >> 1) % kHeadsA;
+  const int64_t g = (blockIdx.x >> 1) / kHeadsA;
+  const int64_t ntiles = (p.rows + kRows - 1) / kRows;
+  const int64_t tile0 = g * p.tiles_per_cta;
+  const int my_tiles = (int)max((int64_t)0, min((int64_t)p.tiles_per_cta, ntiles - tile0));
+
+  if (tid == 0) {
+    abort_flag = 0;
+    mbar_init(b_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&a_full[i], 1);
+      mbar_init(&a_empty[i], 1);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4 * 32);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, qa::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && my_tiles > 0) {
+      prefetch_tensormap(&a_map);
+      prefetch_tensormap(&w_map);
+      mbar_arrive_expect_tx(b_full, 4 * kRegion);
+      for (int j = 0; j < 4; ++j) tma_load_3d(smem + qa::kOffB + j * kRegion, &w_map, b_full, 256 * n + 64 * j, 0, h);
+      for (int i = 0; i < my_tiles; ++i) {
+        const int s = i & 1;
+        if (i >= 2 && !mbar_wait(&a_empty[s], ((i >> 1) + 1) & 1, &abort_flag, p.status, DSA_SITE_ABSORB_A_EMPTY))
+          break;
+        mbar_arrive_expect_tx(&a_full[s], qa::kAStage);
+        const int32_t t = (int32_t)((tile0 + i) * kRows);
+        uint8_t* dst = smem + qa::kOffA + s * qa::kAStage;
+        tma_load_3d(dst, &a_map, &a_full[s], 0, h, t);
+        tma_load_3d(dst + kRegion, &a_map, &a_full[s], 64, h, t);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && my_tiles > 0) {
+      constexpr uint32_t idesc = idesc_f32acc(1, 1, kRows, 256, 0, 1 /*B MN-major*/);
+      const uint32_t b_addr = smem_u32(smem + qa::kOffB);
+      bool ok = mbar_wait(b_full, 0, &abort_flag, p.status, DSA_SITE_ABSORB_W);
+      for (int i = 0; ok && i < my_tiles; ++i) {
+        const int s = i & 1, a = i & 1;
+        if (i >= 2 && !mbar_wait(&acc_empty[a], ((i >> 1) + 1) & 1, &abort_flag, p.status, DSA_SITE_ABSORB_ACC_EMPTY))
+          break;
+        if (!mbar_wait(&a_full[s], (i >> 1) & 1, &abort_flag, p.status, DSA_SITE_ABSORB_A_FULL)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + qa::kOffA + s * qa::kAStage);
+#pragma unroll
+        for (int ks = 0; ks < kNope / 16; ++ks) {
+          const uint64_t ad = sdesc_kmajor_sw128(a_addr + (ks >> 2) * kRegion + (ks & 3) * 32);
+          const uint64_t bd = sdesc_mnmajor_sw128(b_addr + ks * 2048, kRegion, 1024);   // 16 d-rows per K-step
+          mma_f16_ss(tmem + a * 256, ad, bd, idesc, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(&a_empty[s]);
+        mma_commit(&acc_full[a]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (warps 2-5)
+    // warp w reads TMEM lane quadrant w % 4: one tile row per thread
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    uint8_t* srow = smem + qa::kOffStage + r * qa::kRowBytes;
+    for (int i = 0; i < my_tiles; ++i) {
+      const int a = i & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[a], (i >> 1) & 1, &abort_flag, p.status,
+                                             DSA_SITE_ABSORB_ACC_FULL)))
+        break;
+      tc_fence_after();
+      const int64_t t = (tile0 + i) * kRows + r;
+      if (i > 0) bulk_wait_read();                   // the previous row's copy has read the staging row
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + a * 256;
+#pragma unroll 1
+      for (int c = 0; c < 8; c += 2) {
+        uint32_t v0[32], v1[32];
+        tmem_ld32(taddr + c * 32, v0);
+        tmem_ld32(taddr + (c + 1) * 32, v1);
+        tmem_ld_wait();
+        store_bf16_32(srow + c * 64, v0);
+        store_bf16_32(srow + (c + 1) * 64, v1);
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[a]);
+      if (t < p.rows) {
+        if (n == 1) {
+          const int pos = __ldg(p.pos + t);
+          if (!rope_row(p.q_pe + (t * kHeadsA + h) * kRopeD, pos, p, reinterpret_cast<uint4*>(srow + 512)))
+            set_status(p.status, DSA_ERR_DEVICE_BOUNDS);
+        }
+        fence_proxy_async_smem();
+        bulk_store_s2g(p.out + (t * kHeadsA + h) * kQk + 256 * n, smem_u32(srow), n ? 640u : 512u);
+        bulk_commit();
+      }
+    }
+    bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, qa::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------ out_absorb
+// CTA = (group of row tiles, head h): x[t][h][0:128] for its tiles. K (512 latent features) streams
+// in 8 chunks of 64 through a 4-stage ring; each stage holds the o chunk (128 rows x 64 c, K-major)
+// and the w_uv chunk (128 d rows x 64 c, K-major). Accumulator: 128 x 128 fp32, double-buffered.
+namespace oa {
+constexpr int kStages = 4;
+constexpr int kStageBytes = 2 * kRegion;
+constexpr int kRowBytes = 272;                        // 256 B (128 bf16) + 16 B pad
+constexpr int kOffStage = kStages * kStageBytes;
+constexpr int kOffBar = kOffStage + kRows * kRowBytes;
+constexpr int kSmemBytes = kOffBar + 128 + 1024;
+constexpr int kTmemCols = 256;
+constexpr int kChunks = kLat / 64;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+}  // namespace oa
+
+__global__ void __launch_bounds__(kThreads, 1)
+    out_absorb_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constant__ CUtensorMap w_map,
+                      const AbsorbParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + oa::kOffBar);
+  uint64_t* full = bars;                          // [kStages]
+  uint64_t* empty = bars + oa::kStages;           // [kStages]
+  uint64_t* acc_full = bars + 2 * oa::kStages;    // [2]
+  uint64_t* acc_empty = acc_full + 2;             // [2]
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.x % kHeadsA;
+  const int64_t g = blockIdx.x / kHeadsA;
+  const int64_t ntiles = (p.rows + kRows - 1) / kRows;
+  const int64_t tile0 = g * p.tiles_per_cta;
+  const int my_tiles = (int)max((int64_t)0, min((int64_t)p.tiles_per_cta, ntiles - tile0));
+
+  if (tid == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < oa::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4 * 32);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, oa::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const int nsteps = my_tiles * oa::kChunks;
+
+  if (warp == 0) {
+    if (lane == 0 && my_tiles > 0) {
+      prefetch_tensormap(&a_map);
+      prefetch_tensormap(&w_map);
+      for (int q = 0; q < nsteps; ++q) {
+        const int s = q % oa::kStages, kc = q % oa::kChunks;
+        if (q >= oa::kStages &&
+            !mbar_wait(&empty[s], ((q / oa::kStages) + 1) & 1, &abort_flag, p.status, DSA_SITE_ABSORB_A_EMPTY))
+          break;
+        mbar_arrive_expect_tx(&full[s], oa::kStageBytes);
+        const int32_t t = (int32_t)((tile0 + q / oa::kChunks) * kRows);
+        uint8_t* dst = smem + s * oa::kStageBytes;
+        tma_load_3d(dst, &a_map, &full[s], 64 * kc, h, t);
+        tma_load_3d(dst + kRegion, &w_map, &full[s], 64 * kc, 0, h);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && my_tiles > 0) {
+      constexpr uint32_t idesc = idesc_f32acc(1, 1, kRows, kVd, 0, 0);
+      bool ok = true;
+      for (int i = 0; ok && i < my_tiles; ++i) {
+        const int a = i & 1;
+        if (i >= 2 && !mbar_wait(&acc_empty[a], ((i >> 1) + 1) & 1, &abort_flag, p.status, DSA_SITE_ABSORB_ACC_EMPTY))
+          break;
+        for (int kc = 0; kc < oa::kChunks; ++kc) {
+          const int q = i * oa::kChunks + kc, s = q % oa::kStages;
+          if (!mbar_wait(&full[s], (q / oa::kStages) & 1, &abort_flag, p.status, DSA_SITE_ABSORB_A_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t base = smem_u32(smem + s * oa::kStageBytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16_ss(tmem + a * kVd, sdesc_kmajor_sw128(base + kk * 32), sdesc_kmajor_sw128(base + kRegion + kk * 32),
+                       idesc, (kc | kk) ? 1u : 0u);
+          mma_commit(&empty[s]);
+        }
+        if (ok) mma_commit(&acc_full[a]);
+      }
+    }
+  } else {
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    uint8_t* srow = smem + oa::kOffStage + r * oa::kRowBytes;
+    for (int i = 0; i < my_tiles; ++i) {
+      const int a = i & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[a], (i >> 1) & 1, &abort_flag, p.status,
+                                             DSA_SITE_ABSORB_ACC_FULL)))
+        break;
+      tc_fence_after();
+      const int64_t t = (tile0 + i) * kRows + r;
+      if (i > 0) bulk_wait_read();
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + a * kVd;
+#pragma unroll 1
+      for (int c = 0; c < 4; c += 2) {
+        uint32_t v0[32], v1[32];
+        tmem_ld32(taddr + c * 32, v0);
+        tmem_ld32(taddr + (c + 1) * 32, v1);
+        tmem_ld_wait();
+        store_bf16_32(srow + c * 64, v0);
+        store_bf16_32(srow + (c + 1) * 64, v1);
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[a]);
+      if (t < p.rows) {
+        fence_proxy_async_smem();
+        bulk_store_s2g(p.out + (t * kHeadsA + h) * kVd, smem_u32(srow), kVd * 2);
+        bulk_commit();
+      }
+    }
+    bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, oa::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------ kv_entry
+// One warp per token: lanes copy the 1 KB latent row (two 16-byte chunks each) and rotate one
+// rotary pair each into the cache row dst_row[t].
+__global__ void __launch_bounds__(256) kv_entry_kernel(const uint16_t* kv, const uint16_t* k_pe, const int32_t* pos,
+                                                       const float* rope_cs, int max_pos, int64_t rows,
+                                                       const int64_t* dst_row, uint16_t* cache, int64_t cache_rows,
+                                                       int* status) {
+  const int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= rows) return;
+  const int64_t dst = __ldg(dst_row + t);
+  const int ps = __ldg(pos + t);
+  if (dst < 0 || dst >= cache_rows || ps < 0 || ps >= max_pos) {
+    if (lane == 0) set_status(status, DSA_ERR_DEVICE_BOUNDS);
+    return;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(kv + t * kLat);
+  uint4* out = reinterpret_cast<uint4*>(cache + dst * kQk);
+  const uint4 v0 = __ldg(src + lane), v1 = __ldg(src + 32 + lane);
+  const uint32_t x = __ldg(reinterpret_cast<const uint32_t*>(k_pe + t * kRopeD) + lane);
+  const float2 cs = __ldg(reinterpret_cast<const float2*>(rope_cs + (int64_t)ps * kRopeD) + lane);
+  const float a = __uint_as_float(x << 16), b = __uint_as_float(x & 0xFFFF0000u);
+  out[lane] = v0;
+  out[32 + lane] = v1;
+  reinterpret_cast<uint32_t*>(cache + dst * kQk + kLat)[lane] =
+      pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)), __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
+}
+
+// Row tiles per CTA: enough CTAs for about eight per SM over the whole grid, at least one tile each.
+int tiles_per_cta(int64_t ntiles, int64_t ctas_per_group) {
+  const int64_t target = (int64_t)dsa_host::device_sm_count() * 8;
+  int64_t tpc = (ntiles * ctas_per_group + target - 1) / target;
+  return (int)std::max<int64_t>(1, std::min<int64_t>(tpc, ntiles));
+}
+
+bool configure(const void* func, int smem_bytes) {
+  return cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) == cudaSuccess;
+}
+
+}  // namespace
+
+int launch_mla_q_absorb(const uint16_t* q_nope, const uint16_t* q_pe, const int32_t* pos, const float* rope_cs,
+                        int max_pos, const uint16_t* w_uk, int64_t w_head_stride, int64_t rows, uint16_t* q_out,
+                        cudaStream_t stream, int* status) {
+  if (rows == 0) return DSA_OK;
+  CUtensorMap a_map, w_map;
+  const uint64_t a_dims[3] = {kNope, kHeadsA, (uint64_t)rows};
+  const uint64_t a_str[2] = {kNope * 2, (uint64_t)kHeadsA * kNope * 2};
+  const uint32_t a_box[3] = {64, 1, kRows};
+  const uint64_t w_dims[3] = {kLat, kNope, kHeadsA};
+  const uint64_t w_str[2] = {kLat * 2, (uint64_t)w_head_stride * 2};
+  const uint32_t w_box[3] = {64, kNope, 1};
+  if (!dsa_host::encode_tensor_map_3d(&a_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (void*)q_nope, a_dims, a_str, a_box,
+                                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !dsa_host::encode_tensor_map_3d(&w_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (void*)w_uk, w_dims, w_str, w_box,
+                                      CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    if (!configure((const void*)q_absorb_kernel, qa::kSmemBytes)) return DSA_ERR_CUDA;
+    configured[dev] = true;
+  }
+  const int64_t ntiles = (rows + kRows - 1) / kRows;
+  AbsorbParams p{};
+  p.q_pe = q_pe; p.pos = pos; p.rope_cs = rope_cs; p.max_pos = max_pos; p.rows = rows;
+  p.tiles_per_cta = tiles_per_cta(ntiles, 2 * kHeadsA);
+  p.out = q_out; p.status = status;
+  const int64_t grid = (ntiles + p.tiles_per_cta - 1) / p.tiles_per_cta * 2 * kHeadsA;
+  if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;
+  q_absorb_kernel<<<(unsigned)grid, kThreads, qa::kSmemBytes, stream>>>(a_map, w_map, p);
+  return dsa_host::check_launch();
+}
+
+int launch_mla_out_absorb(const uint16_t* o, const uint16_t* w_uv, int64_t w_head_stride, int64_t rows,
+                          uint16_t* out, cudaStream_t stream, int* status) {
+  if (rows == 0) return DSA_OK;
+  CUtensorMap a_map, w_map;
+  const uint64_t a_dims[3] = {kLat, kHeadsA, (uint64_t)rows};
+  const uint64_t a_str[2] = {kLat * 2, (uint64_t)kHeadsA * kLat * 2};
+  const uint32_t a_box[3] = {64, 1, kRows};
+  const uint64_t w_dims[3] = {kLat, kVd, kHeadsA};
+  const uint64_t w_str[2] = {kLat * 2, (uint64_t)w_head_stride * 2};
+  const uint32_t w_box[3] = {64, kVd, 1};
+  if (!dsa_host::encode_tensor_map_3d(&a_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (void*)o, a_dims, a_str, a_box,
+                                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !dsa_host::encode_tensor_map_3d(&w_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (void*)w_uv, w_dims, w_str, w_box,
+                                      CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    if (!configure((const void*)out_absorb_kernel, oa::kSmemBytes)) return DSA_ERR_CUDA;
+    configured[dev] = true;
+  }
+  const int64_t ntiles = (rows + kRows - 1) / kRows;
+  AbsorbParams p{};
+  p.rows = rows;
+  p.tiles_per_cta = tiles_per_cta(ntiles, kHeadsA);
+  p.out = out; p.status = status;
+  const int64_t grid = (ntiles + p.tiles_per_cta - 1) / p.tiles_per_cta * kHeadsA;
+  if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;
+  out_absorb_kernel<<<(unsigned)grid, kThreads, oa::kSmemBytes, stream>>>(a_map, w_map, p);
+  return dsa_host::check_launch();
+}
+
+int launch_mla_kv_entry(const uint16_t* kv, const uint16_t* k_pe, const int32_t* pos, const float* rope_cs,
+                        int max_pos, int64_t rows, const int64_t* dst_row, uint16_t* kv_cache, int64_t cache_rows,
+                        cudaStream_t stream, int* status) {
+  if (rows == 0) return DSA_OK;
+  const int64_t grid = (rows + 7) / 8;
+  if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;
+  kv_entry_kernel<<<(unsigned)grid, 256, 0, stream>>>(kv, k_pe, pos, rope_cs, max_pos, rows, dst_row, kv_cache,
+                                                      cache_rows, status);
+  return dsa_host::check_launch();
+}
+
+}  // namespace dsa

@@ -118,11 +118,6 @@ MlaSplit choose_split(int64_t BT, int k, int sms) {
   return best;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
 // byte offset of 16-byte chunk `c` of row `r` in a 128B-swizzled tile of 128-byte rows
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 

@@ -94,6 +94,18 @@ def test_invalid_arguments_rejected_before_launch(L):
     a = list(margs); a[3] = n; assert L.dsa_sparse_mla_paged(*a) == 1       # null block table
     a = list(margs); a[9] = 0; assert L.dsa_sparse_mla_paged(*a) == 1       # k < 1
     a = list(margs); a[1] = bad; assert L.dsa_sparse_mla_paged(*a) == 1     # misaligned pool
+    # MLA producers: (q_nope, q_pe, pos, rope_cs, max_pos, w, w_head_stride, rows, q_out, stream)
+    ws = 256 * 512
+    assert L.dsa_mla_q_absorb(p, p, p, p, 16, p, ws, 0, p, n) == 0            # no rows: nothing to do
+    assert L.dsa_mla_q_absorb(p, p, p, p, 16, p, 1000, 4, p, n) == 1         # head stride < 128*512
+    assert L.dsa_mla_q_absorb(p, p, p, p, 16, p, ws + 4, 4, p, n) == 1       # head stride not 16-byte
+    assert L.dsa_mla_q_absorb(p, p, p, p, 0, p, ws, 4, p, n) == 1            # empty table
+    assert L.dsa_mla_q_absorb(p, p, p, p, 16, bad, ws, 4, p, n) == 1         # misaligned weights
+    assert L.dsa_mla_q_absorb(p, p, p, p, 16, p, ws, -1, p, n) == 1          # negative rows
+    assert L.dsa_mla_out_absorb(p, p, ws, 1 << 31, p, n) == 1                # rows past int32
+    assert L.dsa_mla_out_absorb(p, n, ws, 4, p, n) == 1                      # null weights
+    assert L.dsa_mla_kv_entry(p, p, p, p, 16, 4, p, p, 0, n) == 1            # empty cache
+    assert L.dsa_mla_kv_entry(p, p, p, p, 16, 4, bad, p, 8, n) == 1          # misaligned dst_row
     assert L.dsa_rope_table(n, 10) == 1
     assert L.dsa_rope_table(p, 0) == 1
 
