@@ -70,6 +70,18 @@ def work_units(inp):
     }
 
 
+def producer_units(rows):
+    """Algorithmic bytes (read + written) and flops of the MLA producers for `rows` tokens: the
+    activations in and out once, the 16.8 MB per-head weight matrix once, the RoPE table row."""
+    w = 128 * 128 * 512 * 2
+    return {
+        "q_absorb": {"bytes": rows * 128 * (128 + 64 + 576) * 2 + w + rows * (4 + 256),
+                     "flops": rows * 128 * 128 * 512 * 2},
+        "kv_entry": {"bytes": rows * ((512 + 64) * 2 + 8 + 4 + 256 + 576 * 2), "flops": 0},
+        "out_absorb": {"bytes": rows * 128 * (512 + 128) * 2 + w, "flops": rows * 128 * 512 * 128 * 2},
+    }
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -381,6 +393,9 @@ def run_ours(args, rank, world, local_rank):
     t_e2e = sum(s.elapsed_time(e) for s, e in e2e) / 1e3
     check_status(dsa, "end-to-end steps")
 
+    producers = None if (args.no_producers or st.kv is None) else time_producers(st, args, dev)
+    paged = None if (args.no_producers or st.kv is None) else time_paged(st, args, dev)
+
     # ---- max over ranks
     t_dev, t_e2e = max_over_ranks([t_dev, t_e2e], world, dev)
     if rank != 0:
@@ -421,9 +436,145 @@ def run_ours(args, rank, world, local_rank):
                    "timed step; e2e: plain API calls"),
         "clocks": clocks,
     }
+    if producers is not None:
+        line["mla_producers"] = producer_rooflines(producers, peaks)
+    if paged is not None:
+        line["paged_caches"] = paged_rooflines(paged, units, peaks, args)
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_budget)
     return line
+
+
+def time_producers(st, args, dev):
+    """Device time of each MLA producer call for this workload's tokens (B*T rows): each call is
+    captured alone as a CUDA graph and replayed `steps` times after warm-up, each replay after an
+    L2 flush and bracketed by CUDA events. Outside the step: the step is the indexer + sparse
+    MLA path the metric names."""
+    import torch
+    import sparse_attention_keys_b200 as dsa
+    rows = st.B * st.T
+    pin = DI.make_mla_producer_inputs(rows, seed=1)
+    dv = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    bf = lambda a: dv(a).view(torch.bfloat16)
+    wkv_b = bf(pin.wkv_b)
+    q_nope, q_pe, kv, k_pe, o = bf(pin.q_nope), bf(pin.q_pe), bf(pin.kv), bf(pin.k_pe), bf(pin.o)
+    pos = dv(pin.pos)
+    q_out = torch.empty((rows, 128, 576), dtype=torch.bfloat16, device=dev)
+    x = torch.empty((rows, 128, 128), dtype=torch.bfloat16, device=dev)
+    cache = torch.empty((rows, 576), dtype=torch.bfloat16, device=dev)
+    dst = torch.arange(rows, dtype=torch.int64, device=dev)
+    calls = {
+        "q_absorb": lambda: dsa.dsa_mla_q_absorb(q_nope, q_pe, pos, st.table, wkv_b[:, :128], q_out=q_out),
+        "kv_entry": lambda: dsa.dsa_mla_kv_entry(kv, k_pe, pos, st.table, dst, cache),
+        "out_absorb": lambda: dsa.dsa_mla_out_absorb(o, wkv_b[:, 128:], out=x),
+    }
+    out = {"rows": rows}
+    for name, fn in calls.items():
+        out[name] = _graph_time(st, fn, args)
+    check_status(dsa, "MLA producers")
+    return out
+
+
+def _graph_time(st, fn, args):
+    """Mean device time of `fn` captured alone as a CUDA graph: warm-up replays, then `steps`
+    replays, each after an L2 flush and bracketed by CUDA events."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cs):
+        fn()
+    torch.cuda.current_stream().wait_stream(cs)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=cs):
+        fn()
+    for _ in range(max(3, args.warmup)):
+        st.l2_flush()
+        g.replay()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(max(5, args.steps)):
+        st.l2_flush()
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record()
+        g.replay()
+        e.record()
+        torch.cuda.synchronize()
+        ts.append(s.elapsed_time(e) / 1e3)
+    del g
+    return sum(ts) / len(ts)
+
+
+def time_paged(st, args, dev, page_size=64):
+    """The step's index scores and sparse MLA over paged copies of its caches (pages of 64 rows laid
+    out in a seeded random order), each timed alone beside the same call on the dense caches; the
+    paged outputs are checked bit for bit against the dense ones."""
+    import torch
+    import sparse_attention_keys_b200 as dsa
+    B, T, S = st.B, st.T, st.S
+    max_pages = S // page_size
+    num_pages = B * max_pages
+    gen = torch.Generator().manual_seed(5)
+    perm = torch.randperm(num_pages, generator=gen).to(dev)
+    table = perm.view(B, max_pages).to(torch.int32).contiguous()
+
+    def to_pool(dense, row_shape):
+        pool = torch.empty((num_pages, page_size) + row_shape, dtype=dense.dtype, device=dev)
+        pool[perm.long()] = dense.reshape((num_pages, page_size) + row_shape)
+        return pool.view((num_pages * page_size,) + row_shape)
+
+    k8p, ksp, kvp = to_pool(st.kcache, (128,)), to_pool(st.kscale, ()), to_pool(st.kv, (576,))
+    d = st.d
+    q8, qs = st.q8.view(B, T, 64, 128), st.qs.view(B, T, 64)
+    sp = torch.empty_like(st.scores)
+    outp, lsep = torch.empty_like(st.out), torch.empty_like(st.lse)
+    calls = {
+        "index_scores": lambda: dsa.dsa_index_scores(q8, qs, d["w"], st.kcache, st.kscale, d["q_pos"], d["kv_len"],
+                                                     scores=st.scores, ld=st.ld),
+        "index_scores_paged": lambda: dsa.dsa_index_scores_paged(q8, qs, d["w"], k8p, ksp, table, page_size, d["q_pos"],
+                                                                 d["kv_len"], scores=sp, ld=st.ld),
+        "sparse_mla": lambda: dsa.dsa_sparse_mla(d["mq"], st.kv, st.idx, out=st.out, lse=st.lse, workspace=st.ws),
+        "sparse_mla_paged": lambda: dsa.dsa_sparse_mla_paged(d["mq"], kvp, table, page_size, st.idx, out=outp,
+                                                             lse=lsep, workspace=st.ws),
+    }
+    t = {n: _graph_time(st, fn, args) for n, fn in calls.items()}
+    check_status(dsa, "paged caches")
+    if not (torch.equal(outp, st.out) and torch.equal(lsep, st.lse)):
+        raise RuntimeError("paged sparse MLA differs from the dense call")
+    nv = np.clip(np.minimum(st.inp.q_pos.astype(np.int64) + 1, st.inp.kv_len[:, None]), 0, None)
+    a, b = st.scores.cpu().numpy(), sp.cpu().numpy()
+    for bb in range(B):
+        for tt in range(T):
+            if not np.array_equal(a[bb, tt, :nv[bb, tt]], b[bb, tt, :nv[bb, tt]]):
+                raise RuntimeError("paged index scores differ from the dense call")
+    t["page_size"] = page_size
+    return t
+
+
+def paged_rooflines(t, units, peaks, args):
+    res = {"page_size": t["page_size"], "layout": "seeded random page order", "timing": "graph of the call alone, L2 flushed before each replay",
+           "check": "paged outputs equal the dense ones bit for bit"}
+    for name in ("index_scores", "sparse_mla"):
+        r = roofline_entry(name, t[f"{name}_paged"], units, peaks, args)
+        res[name] = {"dense_us": t[name] * 1e6, "paged_us": t[f"{name}_paged"] * 1e6, "bound": r["bound"],
+                     "achieved": r["achieved"], "peak": r["peak"], "unit": r["unit"], "frac": r["frac"]}
+    return res
+
+
+def producer_rooflines(t, peaks):
+    """Per producer: device time, algorithmic bytes / flops and the HBM roofline (all three are
+    below the bf16 ridge: bound by memory)."""
+    units = producer_units(t["rows"])
+    res = {"rows": t["rows"], "timing": "graph of the call alone, L2 flushed before each replay"}
+    for name in ("q_absorb", "kv_entry", "out_absorb"):
+        sec = t[name]
+        u = units[name]
+        ach = u["bytes"] / sec / 1e9
+        res[name] = {"us": sec * 1e6, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": ach / peaks["hbm_gbs"], "algorithmic_bytes": u["bytes"],
+                     "tflops": u["flops"] / sec / 1e12 if u["flops"] else None}
+    return res
 
 
 def roofline_entry(name, seconds, units, peaks, args):
@@ -575,6 +726,7 @@ def main():
     ap.add_argument("--workload", default="decode_b8", choices=sorted(DI.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-producers", action="store_true", help="skip timing the MLA producer calls")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:

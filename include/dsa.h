@@ -210,7 +210,7 @@ DSA_API size_t dsa_sparse_mla_noalloc_scratch_bytes(void);
  *
  *   block_table  int32 [B][max_pages], page ids in [0, num_pages) for every page that holds a
  *                visible position (entries past a sequence's length are not read)
- *   page_size    a multiple of 64; S_max = max_pages * page_size is the logical capacity
+ *   page_size    a power of two, at least 64; S_max = max_pages * page_size is the logical capacity
  * A visible position whose page id is out of range sets DSA_ERR_DEVICE_BOUNDS (its key is
  * skipped: score left unwritten, attention weight zero).
  */

@@ -327,9 +327,10 @@ int dsa_mla_out_absorb(const uint16_t* o, const uint16_t* w_uv, int64_t w_head_s
   return dsa::launch_mla_out_absorb(o, w_uv, w_head_stride, rows, out, (cudaStream_t)stream, status);
 }
 
-// Shared checks of the paged-cache arguments: page ids are int32 and pool rows index int32.
+// Shared checks of the paged-cache arguments: page_size a power of two >= 64; page ids are int32
+// and pool rows index int32.
 static bool paged_args_ok(int64_t num_pages, const int32_t* block_table, int max_pages, int page_size) {
-  if (num_pages < 1 || max_pages < 1 || page_size < 64 || page_size % 64 != 0) return false;
+  if (num_pages < 1 || max_pages < 1 || page_size < 64 || (page_size & (page_size - 1)) != 0) return false;
   if (num_pages * page_size > 0x7fffffffLL || (int64_t)max_pages * page_size > 0x7fffffffLL) return false;
   return block_table != nullptr && (reinterpret_cast<uintptr_t>(block_table) & 3) == 0;
 }

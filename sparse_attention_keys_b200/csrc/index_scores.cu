@@ -58,15 +58,15 @@ struct ScoresParams {
   int* status;
   // paged K-cache (block_table == nullptr: dense [B][S_max] rows)
   const int32_t* block_table;   // [B][max_pages]
-  int max_pages, page_size;
+  int max_pages, page_size, page_shift;   // page_size = 1 << page_shift
   int64_t num_pages;
 };
 
 // Pool row of sequence b's logical position s in a paged K-cache, or -1 if its page id is out of
 // range (S_max = max_pages * page_size bounds s).
 __device__ __forceinline__ int64_t paged_row(const ScoresParams& p, int b, int s) {
-  const int pg = __ldg(p.block_table + (int64_t)b * p.max_pages + s / p.page_size);
-  return (pg >= 0 && pg < p.num_pages) ? (int64_t)pg * p.page_size + s % p.page_size : -1;
+  const int pg = __ldg(p.block_table + (int64_t)b * p.max_pages + (s >> p.page_shift));
+  return (pg >= 0 && pg < p.num_pages) ? ((int64_t)pg << p.page_shift) + (s & (p.page_size - 1)) : -1;
 }
 
 }  // namespace
@@ -212,18 +212,26 @@ __global__ void __launch_bounds__(threads_for(NQ), 1)
     const bool active = q_lo < NQ;                     // NQ = 1: one warp per quadrant
     const int row_in_tile = quad * 32 + lane;          // TMEM lane = key within the tile
     const float* ks_row = p.k_scale + (int64_t)b * p.S_max;
-    auto load_ks = [&](int i) -> float {               // k_scale of this thread's key in tile i (-1: bad page)
-      const int key = (kt_begin + i) * kKeysPerTile + row_in_tile;
-      if (!(active && i < my_tiles && key < p.S_max)) return 0.f;
-      if (!PAGED) return __ldg(ks_row + key);
-      const int64_t row = paged_row(p, b, key);
-      return row >= 0 ? __ldg(p.k_scale + row) : -1.f;
+    // k_scale of this thread's key in tile i, one tile ahead; paged: its page id two tiles ahead
+    // (-2: no key in that tile) and the scale one tile ahead (-1: the page is outside the pool)
+    auto tile_key = [&](int i) { return (kt_begin + i) * kKeysPerTile + row_in_tile; };
+    auto has_key = [&](int i) { return active && i < my_tiles && tile_key(i) < p.S_max; };
+    auto load_pg = [&](int i) -> int {
+      return has_key(i) ? __ldg(p.block_table + (int64_t)b * p.max_pages + (tile_key(i) >> p.page_shift)) : -2;
     };
-    float ks_next = load_ks(0);
+    auto load_ks = [&](int i, int pg) -> float {
+      if (!PAGED) return has_key(i) ? __ldg(ks_row + tile_key(i)) : 0.f;
+      if (pg == -2) return 0.f;
+      if (pg < 0 || pg >= p.num_pages) return -1.f;
+      return __ldg(p.k_scale + ((int64_t)pg << p.page_shift) + (tile_key(i) & (p.page_size - 1)));
+    };
+    int pg_next = PAGED ? load_pg(1) : 0;
+    float ks_next = load_ks(0, PAGED ? load_pg(0) : 0);
     for (int i = 0; i < my_tiles; ++i) {
       const int a = i % kAcc;
       const float ks = ks_next;
-      ks_next = load_ks(i + 1);                        // one tile ahead
+      ks_next = load_ks(i + 1, pg_next);               // one tile ahead
+      if (PAGED) pg_next = load_pg(i + 2);             // two tiles ahead
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[a], (i / kAcc) & 1, &abort_flag, p.status, DSA_SITE_SCORES_ACC_FULL))) break;
       tc_fence_after();
       if (active) {
@@ -361,6 +369,7 @@ int launch_index_scores_paged(const uint8_t* q8, const float* q_scale, const flo
   p.wscale = 0.125f * softmax_scale;
   p.flags = flags; p.status = status;
   p.block_table = block_table; p.max_pages = max_pages; p.page_size = page_size; p.num_pages = num_pages;
+  p.page_shift = __builtin_ctz((unsigned)page_size);
   if (T >= 4) return launch_scores_nq<4, true>(q8, k8_pool, p, stream);
   return launch_scores_nq<1, true>(q8, k8_pool, p, stream);
 }

@@ -145,18 +145,20 @@ struct MlaParams {
   // paged latent cache: kv is a pool of num_pages pages of page_size rows, and logical position v of
   // sequence b lives in row block_table[b][v / page_size] * page_size + v % page_size
   const int32_t* block_table;  // [B][max_pages]
-  int max_pages, page_size;
+  int max_pages, page_size, page_shift;   // page_size = 1 << page_shift
   int64_t num_pages;
 };
 
 // Pool row of logical position v (PAGED: pg = block_table[b][v / page_size], read one tile ahead),
 // or -1 for a slot that takes no part: padding (v < 0), v >= S_max, or a page id outside the pool.
 template <bool PAGED>
+__device__ __forceinline__ bool kv_valid(const MlaParams& p, int v, int pg) {
+  return v >= 0 && v < p.S_max && (!PAGED || (pg >= 0 && (int64_t)pg < p.num_pages));
+}
+template <bool PAGED>
 __device__ __forceinline__ int kv_row(const MlaParams& p, int v, int pg) {
-  if (v < 0 || v >= p.S_max) return -1;
-  if (!PAGED) return v;
-  if (pg < 0 || (int64_t)pg >= p.num_pages) return -1;
-  return pg * p.page_size + v % p.page_size;
+  if (!kv_valid<PAGED>(p, v, pg)) return -1;
+  return PAGED ? (pg << p.page_shift) + (v & (p.page_size - 1)) : v;
 }
 
 // Q K^T of one 32-key tile: 20 K-steps with Q from TMEM, then 16 with Q from shared memory. HALF
@@ -299,7 +301,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       const int slot = j * kKeys + 8 * w + (lane & 7);
       return (j < ntiles && slot < nslots) ? __ldg(idx_row + slot) : -1;
     };
-    auto load_page = [&](int v) -> int { return (v >= 0 && v < p.S_max) ? __ldg(pages + v / p.page_size) : -1; };
+    auto load_page = [&](int v) -> int { return (v >= 0 && v < p.S_max) ? __ldg(pages + (v >> p.page_shift)) : -1; };
     // dense: indices one tile ahead; paged: indices two tiles ahead, their page ids one tile ahead
     int idx_next = idx_first;                        // load_idx(0), issued before the set-up barrier
     int pg_next = 0, idx_next2 = -1;
@@ -401,7 +403,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     bool ok = true;
     // slot j * 32 + lane of the next tile (paged: also the slot two tiles ahead and the next tile's page id)
     const int32_t* pages = PAGED ? p.block_table + (int64_t)b * p.max_pages : nullptr;
-    auto load_page = [&](int v) -> int { return (v >= 0 && v < p.S_max) ? __ldg(pages + v / p.page_size) : -1; };
+    auto load_page = [&](int v) -> int { return (v >= 0 && v < p.S_max) ? __ldg(pages + (v >> p.page_shift)) : -1; };
     int v_next = lane < nslots ? __ldg(idx_row + lane) : -1;
     int pg_next = 0, v_next2 = -1;
     if (PAGED) {
@@ -421,7 +423,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         const int sn = (j + 1) * kKeys + lane;
         v_next = sn < nslots ? __ldg(idx_row + sn) : -1;
       }
-      const uint32_t vmask = __ballot_sync(0xffffffffu, kv_row<PAGED>(p, v_cur, pg_cur) >= 0);
+      const uint32_t vmask = __ballot_sync(0xffffffffu, kv_valid<PAGED>(p, v_cur, pg_cur));
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j % kSBufs], (j / kSBufs) & 1, &abort_flag, p.status,
                                              DSA_SITE_MLA_S_FULL))) {
         ok = false;
@@ -667,6 +669,7 @@ int launch_sparse_mla_paged(const uint16_t* q, const uint16_t* kv_pool, int64_t 
   p.scale_log2 = softmax_scale * kLog2e;
   p.out = out; p.lse = lse; p.status = status;
   p.block_table = block_table; p.max_pages = max_pages; p.page_size = page_size; p.num_pages = num_pages;
+  p.page_shift = __builtin_ctz((unsigned)page_size);
   return launch_mla<true>(q, p, stream, workspace, ws_bytes);
 }
 

@@ -81,7 +81,8 @@ def test_invalid_arguments_rejected_before_launch(L):
     # paged calls: (..., num_pages, block_table, max_pages, page_size, ...)
     sargs = [p, p, p, p, p, 8, p, 4, 64, p, p, 1, 1, f(0.088), p, 256, 0, n]
     a = list(sargs); a[8] = 32; assert L.dsa_index_scores_paged(*a) == 1    # page_size < 64
-    a = list(sargs); a[8] = 96; assert L.dsa_index_scores_paged(*a) == 1    # page_size not a multiple of 64
+    a = list(sargs); a[8] = 96; assert L.dsa_index_scores_paged(*a) == 1    # page_size not a power of two
+    a = list(sargs); a[8] = 192; assert L.dsa_index_scores_paged(*a) == 1   # page_size not a power of two
     a = list(sargs); a[5] = 0; assert L.dsa_index_scores_paged(*a) == 1     # empty pool
     a = list(sargs); a[7] = 0; assert L.dsa_index_scores_paged(*a) == 1     # max_pages < 1
     a = list(sargs); a[6] = n; assert L.dsa_index_scores_paged(*a) == 1     # null block table

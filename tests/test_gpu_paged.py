@@ -52,7 +52,7 @@ def _scores_both(q8, qs, w, k8, ks, q_pos, kv_len, table, k8_pool, ks_pool, page
 
 # ---------------------------------------------------------------------------------- index scores
 @pytest.mark.parametrize("page_size,past_end,decode", [(64, -1, False), (128, 1_000_000, False),
-                                                        (64, 1_000_000, True), (192, -1, True)])
+                                                        (64, 1_000_000, True), (256, -1, True)])
 def test_index_scores_paged_matches_dense_and_oracle(table_dev, page_size, past_end, decode):
     max_pages = (700 + page_size - 1) // page_size
     S = max_pages * page_size
