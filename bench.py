@@ -222,7 +222,8 @@ class Step:
                                [self.kcache, self.kscale] + ([self.kv] if self.kv is not None else []) +
                                list(self.d.values()))
         self.flush_writes = self.input_bytes <= 2 * L2_BYTES
-        self.flush = torch.empty(L2_FLUSH_BYTES // 4 if self.flush_writes else 1, dtype=torch.float32, device=dev)
+        self.flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.flush_src = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
         self.h_idx = torch.empty((B, T, self.k), dtype=torch.int32).pin_memory()
         self.h_out = torch.empty((B, T, 128, 512), dtype=torch.bfloat16).pin_memory() if self.out is not None else None
         self.h_lse = torch.empty((B, T, 128), dtype=torch.float32).pin_memory() if self.out is not None else None
@@ -280,13 +281,17 @@ class Step:
             rec("sparse_mla", lambda: dsa.dsa_sparse_mla(d["mq"], self.kv, self.idx, out=self.out, lse=self.lse,
                                                          workspace=self.ws))
 
-    def l2_flush(self):
-        if self.flush_writes:
+    def l2_flush(self, force=False):
+        """Evict the step's data from the L2 (when the step's inputs fit in it, or `force`): write a
+        buffer larger than the L2, then read another one, so that the write-back of the dirty flush
+        lines happens here, outside the timed events, and the step starts on a cold, clean L2."""
+        if self.flush_writes or force:
             self.flush.zero_()
+            self.flush_sum = self.flush_src.sum()
 
     def l2_policy(self):
         if self.flush_writes:
-            return f"{L2_FLUSH_BYTES >> 20} MiB flush write between timed steps"
+            return f"{L2_FLUSH_BYTES >> 20} MiB flush write, then a {L2_FLUSH_BYTES >> 20} MiB read, between timed steps"
         return f"inputs larger than L2: {self.input_bytes / 2**20:.0f} MiB resident per step, no flush"
 
 
@@ -477,7 +482,7 @@ def time_producers(st, args, dev):
 
 def _graph_time(st, fn, args):
     """Mean device time of `fn` captured alone as a CUDA graph: warm-up replays, then `steps`
-    replays, each after an L2 flush and bracketed by CUDA events."""
+    replays, each after an L2 flush (whatever the step's own policy) and bracketed by CUDA events."""
     import torch
     g = torch.cuda.CUDAGraph()
     cs = torch.cuda.Stream()
@@ -489,12 +494,12 @@ def _graph_time(st, fn, args):
     with torch.cuda.graph(g, stream=cs):
         fn()
     for _ in range(max(3, args.warmup)):
-        st.l2_flush()
+        st.l2_flush(force=True)
         g.replay()
     torch.cuda.synchronize()
     ts = []
     for _ in range(max(5, args.steps)):
-        st.l2_flush()
+        st.l2_flush(force=True)
         s = torch.cuda.Event(enable_timing=True)
         e = torch.cuda.Event(enable_timing=True)
         s.record()

@@ -374,6 +374,230 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------------------------ few rows
+// Decode shapes (rows <= 64): one CTA per head in the swapped orientation, weights on M and the
+// tokens on N (rows rounded up to 16), so each head's 128 KB of weights is read once, by one CTA,
+// in under one wave. The weight chunks land behind per-chunk barriers and the MMAs start as they
+// arrive; after the last MMA the weight buffer stages the output rows (one bulk copy per token).
+namespace fr {
+constexpr int kMaxRows = 64;
+constexpr int kOffW = 0;                          // 8 regions of 16 KB (weights)
+constexpr int kOffX = 8 * kRegion;                // activation regions, kMaxRows x 128 B each
+constexpr int kXRegion = kMaxRows * 128;
+constexpr int kOffBar = kOffX + 8 * kXRegion;
+constexpr int kSmemBytes = kOffBar + 128 + 1024;
+constexpr int kTmemCols = 256;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+}  // namespace fr
+
+__device__ __forceinline__ void st_shared_u16(uint8_t* p, uint16_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(smem_u32(p)), "h"(v) : "memory");
+}
+__device__ __forceinline__ uint16_t bf16_bits(float x) {
+  return (uint16_t)(pack_bf16(x, 0.f) & 0xFFFFu);
+}
+
+// q_absorb, rows <= 64: D^T[c][t] = sum_d w_uk[h][d][c] q_nope[t][h][d]; A = the weights as four
+// 128-c M blocks (MN-major: c contiguous), B = the q_nope rows (K-major), N = n_pad.
+__global__ void __launch_bounds__(kThreads, 1)
+    q_absorb_few_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constant__ CUtensorMap w_map,
+                        const AbsorbParams p, int n_pad) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + fr::kOffBar);
+  uint64_t* w_full = bars;          // [4] weights of M block m landed
+  uint64_t* x_full = bars + 4;      // q_nope rows landed
+  uint64_t* acc_full = bars + 5;    // all MMAs done
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.x;
+  const int rows = (int)p.rows;
+  if (tid == 0) {
+    abort_flag = 0;
+    for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, fr::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(x_full, 2 * n_pad * 128);
+      for (int r = 0; r < 2; ++r) tma_load_3d(smem + fr::kOffX + r * fr::kXRegion, &a_map, x_full, 64 * r, h, 0);
+      for (int m = 0; m < 4; ++m) {
+        mbar_arrive_expect_tx(&w_full[m], 2 * kRegion);
+        for (int j = 2 * m; j < 2 * m + 2; ++j)
+          tma_load_3d(smem + fr::kOffW + j * kRegion, &w_map, &w_full[m], 64 * j, 0, h);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f32acc(1, 1, kRows, (uint32_t)n_pad, 1 /*A MN-major*/, 0);
+      const uint32_t w_addr = smem_u32(smem + fr::kOffW), x_addr = smem_u32(smem + fr::kOffX);
+      bool ok = mbar_wait(x_full, 0, &abort_flag, p.status, DSA_SITE_ABSORB_A_FULL);
+      for (int m = 0; ok && m < 4; ++m) {
+        if (!mbar_wait(&w_full[m], 0, &abort_flag, p.status, DSA_SITE_ABSORB_W)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < kNope / 16; ++ks) {
+          const uint64_t ad = sdesc_mnmajor_sw128(w_addr + 2 * m * kRegion + ks * 2048, kRegion, 1024);
+          const uint64_t bd = sdesc_kmajor_sw128(x_addr + (ks >> 2) * fr::kXRegion + (ks & 3) * 32);
+          mma_f16_ss(tmem + m * n_pad, ad, bd, idesc, ks > 0 ? 1u : 0u);
+        }
+      }
+      if (ok) mma_commit(acc_full);
+    }
+  } else {
+    const int quad = warp & 3, et = tid - 64;           // epilogue thread 0..127
+    uint8_t* stage = smem + fr::kOffW;                   // rows of 1152 B over the consumed weights
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, &abort_flag, p.status, DSA_SITE_ABSORB_ACC_FULL));
+    if (ok) {
+      tc_fence_after();
+      for (int m = 0; m < 4; ++m) {
+        const int c = 128 * m + 32 * quad + lane;
+        for (int cc = 0; cc < n_pad; cc += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + m * n_pad + cc, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (cc + j < rows) st_shared_u16(stage + (cc + j) * (kQk * 2) + c * 2, bf16_bits(__uint_as_float(v[j])));
+        }
+      }
+      // rotary part: thread = (token, pair)
+      for (int i = et; i < rows * 32; i += 128) {
+        const int t = i >> 5, pr = i & 31;
+        const int ps = __ldg(p.pos + t);
+        uint32_t o = 0u;
+        if (ps >= 0 && ps < p.max_pos) {
+          const uint32_t x = __ldg(reinterpret_cast<const uint32_t*>(p.q_pe + ((int64_t)t * kHeadsA + h) * kRopeD) + pr);
+          const float2 cs = __ldg(reinterpret_cast<const float2*>(p.rope_cs + (int64_t)ps * kRopeD) + pr);
+          const float a = __uint_as_float(x << 16), b = __uint_as_float(x & 0xFFFF0000u);
+          o = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)), __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
+        } else if (pr == 0) {
+          set_status(p.status, DSA_ERR_DEVICE_BOUNDS);
+        }
+        *reinterpret_cast<uint32_t*>(stage + t * (kQk * 2) + kLat * 2 + pr * 4) = o;
+      }
+      fence_proxy_async_smem();
+    }
+    // every epilogue warp reaches the barrier, whether or not its wait succeeded
+    asm volatile("bar.sync 1, 128;" ::: "memory");        // the epilogue warps' rows are complete
+    if (ok) {
+      for (int t = et; t < rows; t += 128) {
+        bulk_store_s2g(p.out + ((int64_t)t * kHeadsA + h) * kQk, smem_u32(stage + t * (kQk * 2)), kQk * 2);
+        bulk_commit();
+      }
+      bulk_wait_all();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, fr::kTmemCols);
+  }
+}
+
+// out_absorb, rows <= 64: D^T[d][t] = sum_c w_uv[h][d][c] o[t][h][c]; A = the weights (K-major),
+// B = the o rows (K-major), K streamed in 8 chunks of 64 behind per-chunk barriers.
+__global__ void __launch_bounds__(kThreads, 1)
+    out_absorb_few_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constant__ CUtensorMap w_map,
+                          const AbsorbParams p, int n_pad) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + fr::kOffBar);
+  uint64_t* full = bars;            // [8] chunk kc (weights + rows) landed
+  uint64_t* acc_full = bars + 8;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.x;
+  const int rows = (int)p.rows;
+  if (tid == 0) {
+    abort_flag = 0;
+    for (int i = 0; i < 9; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, fr::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int kc = 0; kc < 8; ++kc) {
+        mbar_arrive_expect_tx(&full[kc], kRegion + n_pad * 128);
+        tma_load_3d(smem + fr::kOffW + kc * kRegion, &w_map, &full[kc], 64 * kc, 0, h);
+        tma_load_3d(smem + fr::kOffX + kc * fr::kXRegion, &a_map, &full[kc], 64 * kc, h, 0);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f32acc(1, 1, kRows, (uint32_t)n_pad, 0, 0);
+      const uint32_t w_addr = smem_u32(smem + fr::kOffW), x_addr = smem_u32(smem + fr::kOffX);
+      bool ok = true;
+      for (int kc = 0; ok && kc < 8; ++kc) {
+        if (!mbar_wait(&full[kc], 0, &abort_flag, p.status, DSA_SITE_ABSORB_A_FULL)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f16_ss(tmem, sdesc_kmajor_sw128(w_addr + kc * kRegion + kk * 32),
+                     sdesc_kmajor_sw128(x_addr + kc * fr::kXRegion + kk * 32), idesc, (kc | kk) ? 1u : 0u);
+      }
+      if (ok) mma_commit(acc_full);
+    }
+  } else {
+    const int quad = warp & 3, et = tid - 64;
+    uint8_t* stage = smem + fr::kOffW;                   // rows of 256 B over the consumed weights
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, &abort_flag, p.status, DSA_SITE_ABSORB_ACC_FULL));
+    if (ok) {
+      tc_fence_after();
+      const int d = 32 * quad + lane;
+      for (int cc = 0; cc < n_pad; cc += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + cc, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (cc + j < rows) st_shared_u16(stage + (cc + j) * (kVd * 2) + d * 2, bf16_bits(__uint_as_float(v[j])));
+      }
+      fence_proxy_async_smem();
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");        // reached by every epilogue warp
+    if (ok) {
+      for (int t = et; t < rows; t += 128) {
+        bulk_store_s2g(p.out + ((int64_t)t * kHeadsA + h) * kVd, smem_u32(stage + t * (kVd * 2)), kVd * 2);
+        bulk_commit();
+      }
+      bulk_wait_all();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, fr::kTmemCols);
+  }
+}
+
 // ------------------------------------------------------------------------------------ kv_entry
 // One warp per token: lanes copy the 1 KB latent row (two 16-byte chunks each) and rotate one
 // rotary pair each into the cache row dst_row[t].
@@ -435,12 +659,26 @@ int launch_mla_q_absorb(const uint16_t* q_nope, const uint16_t* q_pe, const int3
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
-    if (!configure((const void*)q_absorb_kernel, qa::kSmemBytes)) return DSA_ERR_CUDA;
+    if (!configure((const void*)q_absorb_kernel, qa::kSmemBytes) ||
+        !configure((const void*)q_absorb_few_kernel, fr::kSmemBytes))
+      return DSA_ERR_CUDA;
     configured[dev] = true;
   }
   const int64_t ntiles = (rows + kRows - 1) / kRows;
   AbsorbParams p{};
   p.q_pe = q_pe; p.pos = pos; p.rope_cs = rope_cs; p.max_pos = max_pos; p.rows = rows;
+  if (rows <= fr::kMaxRows) {
+    const int n_pad = (int)((rows + 15) / 16 * 16);
+    const uint32_t x_box[3] = {64, 1, (uint32_t)n_pad};
+    CUtensorMap x_map;
+    if (!dsa_host::encode_tensor_map_3d(&x_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (void*)q_nope, a_dims, a_str,
+                                        x_box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return DSA_ERR_CUDA;
+    p.tiles_per_cta = 1;
+    p.out = q_out; p.status = status;
+    q_absorb_few_kernel<<<kHeadsA, kThreads, fr::kSmemBytes, stream>>>(x_map, w_map, p, n_pad);
+    return dsa_host::check_launch();
+  }
   p.tiles_per_cta = tiles_per_cta(ntiles, 2 * kHeadsA);
   p.out = q_out; p.status = status;
   const int64_t grid = (ntiles + p.tiles_per_cta - 1) / p.tiles_per_cta * 2 * kHeadsA;
@@ -468,12 +706,26 @@ int launch_mla_out_absorb(const uint16_t* o, const uint16_t* w_uv, int64_t w_hea
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
-    if (!configure((const void*)out_absorb_kernel, oa::kSmemBytes)) return DSA_ERR_CUDA;
+    if (!configure((const void*)out_absorb_kernel, oa::kSmemBytes) ||
+        !configure((const void*)out_absorb_few_kernel, fr::kSmemBytes))
+      return DSA_ERR_CUDA;
     configured[dev] = true;
   }
   const int64_t ntiles = (rows + kRows - 1) / kRows;
   AbsorbParams p{};
   p.rows = rows;
+  if (rows <= fr::kMaxRows) {
+    const int n_pad = (int)((rows + 15) / 16 * 16);
+    const uint32_t x_box[3] = {64, 1, (uint32_t)n_pad};
+    CUtensorMap x_map;
+    if (!dsa_host::encode_tensor_map_3d(&x_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (void*)o, a_dims, a_str, x_box,
+                                        CU_TENSOR_MAP_SWIZZLE_128B))
+      return DSA_ERR_CUDA;
+    p.tiles_per_cta = 1;
+    p.out = out; p.status = status;
+    out_absorb_few_kernel<<<kHeadsA, kThreads, fr::kSmemBytes, stream>>>(x_map, w_map, p, n_pad);
+    return dsa_host::check_launch();
+  }
   p.tiles_per_cta = tiles_per_cta(ntiles, kHeadsA);
   p.out = out; p.status = status;
   const int64_t grid = (ntiles + p.tiles_per_cta - 1) / p.tiles_per_cta * kHeadsA;

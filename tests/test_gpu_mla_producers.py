@@ -45,7 +45,7 @@ def _weights(inp):
     return wkv_b, wkv_b[:, :128], wkv_b[:, 128:]
 
 
-@pytest.mark.parametrize("rows", [1, 8, 130, 300])
+@pytest.mark.parametrize("rows", [1, 8, 33, 64, 65, 130, 300])    # <= 64: one CTA per head
 def test_q_absorb(table_dev, rows):
     inp = DI.make_mla_producer_inputs(rows, seed=rows)
     _, w_uk, _ = _weights(inp)
@@ -59,15 +59,16 @@ def test_q_absorb(table_dev, rows):
     _within(got[..., 512:], ref[..., 512:], np.zeros_like(ref[..., 512:]) + 2.0 ** -4, "rotary part")
 
 
-def test_q_absorb_position_out_of_range_sets_status(table_dev):
-    inp = DI.make_mla_producer_inputs(4, seed=9)
+@pytest.mark.parametrize("rows", [4, 100])
+def test_q_absorb_position_out_of_range_sets_status(table_dev, rows):
+    inp = DI.make_mla_producer_inputs(rows, seed=9)
     inp.pos[2] = 16384
     _, w_uk, _ = _weights(inp)
     dsa.dsa_mla_q_absorb(P.bf16_dev(inp.q_nope), P.bf16_dev(inp.q_pe), P.to_dev(inp.pos), table_dev, w_uk)
     assert _status() == DSA_ERR_DEVICE_BOUNDS
 
 
-@pytest.mark.parametrize("rows", [1, 8, 200])
+@pytest.mark.parametrize("rows", [1, 8, 50, 64, 65, 200])
 def test_out_absorb(table_dev, rows):
     inp = DI.make_mla_producer_inputs(rows, seed=100 + rows)
     _, _, w_uv = _weights(inp)
