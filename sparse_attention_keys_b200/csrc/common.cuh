@@ -341,6 +341,16 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// ------------------------------------------------------------------- programmatic dependent launch
+// Kernels are launched so that the next kernel on the stream may start while this one finishes.
+// grid_dep_wait: block until the preceding kernel on the stream has completed and its writes are
+// visible (a no-op when the kernel was launched without the attribute). Every kernel calls it
+// before reading a buffer an earlier kernel of the stream writes, and before its own writes.
+// grid_dep_launch: allow the next kernel's CTAs to be scheduled now (each kernel calls it once its
+// own CTAs are set up, so the next kernel's set-up overlaps this one's work).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------- bulk (TMA engine) stores
 // Copies `bytes` (a multiple of 16; both addresses 16-byte aligned) from shared to global memory.
 // The shared-memory source must be made visible to the async proxy first (fence_proxy_async_smem).
@@ -367,6 +377,22 @@ int device_sm_count();
 // TMEM-column limits, from the kernel's own attributes (the runtime's occupancy query does not
 // count these kernels' residency correctly). 0 if the attributes cannot be read.
 int resident_ctas_per_sm(const void* func, int threads, int dyn_smem, int tmem_cols);
+// Launch `kernel` on `stream` allowing programmatic dependent launch (it may begin while the
+// previous kernel on the stream finishes; the kernel's grid_dep_wait orders the data).
+template <typename... KArgs, typename... Args>
+int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
 bool encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, void* base,
                           uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
                           uint32_t box_outer, CUtensorMapSwizzle swizzle);

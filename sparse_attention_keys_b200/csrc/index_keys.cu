@@ -42,6 +42,8 @@ __global__ void __launch_bounds__(256) index_keys_kernel(const In* __restrict__ 
                                                           int* status) {
   const int lane = threadIdx.x & 31;
   const int64_t blk = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  grid_dep_wait();
+  grid_dep_launch();
   if (blk >= blocks) return;
   const int64_t row = blk / heads;
   const int head = (int)(blk - row * heads);
@@ -122,14 +124,12 @@ int launch_index_keys(const void* x, int x_dtype, int64_t rows, int heads, const
   const int warps = 8;
   const int64_t grid = (blocks + warps - 1) / warps;
   if (x_dtype == DSA_BF16)
-    index_keys_kernel<uint16_t><<<(unsigned)grid, warps * 32, 0, stream>>>(
-        static_cast<const uint16_t*>(x), blocks, heads, pos, rope_cs, max_pos, flags, out_fp8, out_scale, dst_row,
-        status);
-  else
-    index_keys_kernel<float><<<(unsigned)grid, warps * 32, 0, stream>>>(
-        static_cast<const float*>(x), blocks, heads, pos, rope_cs, max_pos, flags, out_fp8, out_scale, dst_row,
-        status);
-  return dsa_host::check_launch();
+    return dsa_host::launch(index_keys_kernel<uint16_t>, dim3((unsigned)grid), dim3(warps * 32), 0, stream,
+                            static_cast<const uint16_t*>(x), blocks, heads, pos, rope_cs, max_pos, flags, out_fp8,
+                            out_scale, dst_row, status);
+  return dsa_host::launch(index_keys_kernel<float>, dim3((unsigned)grid), dim3(warps * 32), 0, stream,
+                          static_cast<const float*>(x), blocks, heads, pos, rope_cs, max_pos, flags, out_fp8,
+                          out_scale, dst_row, status);
 }
 
 }  // namespace dsa

@@ -117,6 +117,8 @@ __global__ void __launch_bounds__(threads_for(NQ), 1)
     tmem_alloc(&tmem_base_sh, Cfg::kTmemCols);
     tmem_relinquish();
   }
+  grid_dep_wait();                       // q_scale, w and the caches come from earlier kernels
+  grid_dep_launch();
   for (int i = threadIdx.x; i < NQ * 64; i += kThreads) {   // folded head weights
     const int q = i >> 6, j = i & 63;
     const int t = t0 + q;
@@ -341,8 +343,8 @@ static int launch_scores_nq(const uint8_t* q8, const uint8_t* k8, const ScoresPa
   if (dev >= 64 && cudaFuncSetAttribute(index_scores_kernel<NQ, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         Cfg::kSmemBytes) != cudaSuccess)
     return DSA_ERR_CUDA;
-  index_scores_kernel<NQ, PAGED><<<(unsigned)grid, threads_for(NQ), Cfg::kSmemBytes, stream>>>(qmap, kmap, p);
-  return dsa_host::check_launch();
+  return dsa_host::launch(index_scores_kernel<NQ, PAGED>, dim3((unsigned)grid), dim3(threads_for(NQ)),
+                          Cfg::kSmemBytes, stream, qmap, kmap, p);
 }
 
 int launch_index_scores(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8,

@@ -144,6 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  grid_dep_wait();                       // activations and outputs are shared with earlier kernels
+  grid_dep_launch();
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -290,6 +292,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  grid_dep_wait();                       // activations and outputs are shared with earlier kernels
+  grid_dep_launch();
   const int nsteps = my_tiles * oa::kChunks;
 
   if (warp == 0) {
@@ -426,6 +430,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  grid_dep_wait();                       // activations and outputs are shared with earlier kernels
+  grid_dep_launch();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -537,6 +543,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  grid_dep_wait();                       // activations and outputs are shared with earlier kernels
+  grid_dep_launch();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -607,6 +615,8 @@ __global__ void __launch_bounds__(256) kv_entry_kernel(const uint16_t* kv, const
                                                        int* status) {
   const int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  grid_dep_wait();
+  grid_dep_launch();
   if (t >= rows) return;
   const int64_t dst = __ldg(dst_row + t);
   const int ps = __ldg(pos + t);
@@ -676,15 +686,15 @@ int launch_mla_q_absorb(const uint16_t* q_nope, const uint16_t* q_pe, const int3
       return DSA_ERR_CUDA;
     p.tiles_per_cta = 1;
     p.out = q_out; p.status = status;
-    q_absorb_few_kernel<<<kHeadsA, kThreads, fr::kSmemBytes, stream>>>(x_map, w_map, p, n_pad);
-    return dsa_host::check_launch();
+    return dsa_host::launch(q_absorb_few_kernel, dim3(kHeadsA), dim3(kThreads), fr::kSmemBytes, stream, x_map, w_map,
+                            p, n_pad);
   }
   p.tiles_per_cta = tiles_per_cta(ntiles, 2 * kHeadsA);
   p.out = q_out; p.status = status;
   const int64_t grid = (ntiles + p.tiles_per_cta - 1) / p.tiles_per_cta * 2 * kHeadsA;
   if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;
-  q_absorb_kernel<<<(unsigned)grid, kThreads, qa::kSmemBytes, stream>>>(a_map, w_map, p);
-  return dsa_host::check_launch();
+  return dsa_host::launch(q_absorb_kernel, dim3((unsigned)grid), dim3(kThreads), qa::kSmemBytes, stream, a_map, w_map,
+                          p);
 }
 
 int launch_mla_out_absorb(const uint16_t* o, const uint16_t* w_uv, int64_t w_head_stride, int64_t rows,
@@ -723,15 +733,15 @@ int launch_mla_out_absorb(const uint16_t* o, const uint16_t* w_uv, int64_t w_hea
       return DSA_ERR_CUDA;
     p.tiles_per_cta = 1;
     p.out = out; p.status = status;
-    out_absorb_few_kernel<<<kHeadsA, kThreads, fr::kSmemBytes, stream>>>(x_map, w_map, p, n_pad);
-    return dsa_host::check_launch();
+    return dsa_host::launch(out_absorb_few_kernel, dim3(kHeadsA), dim3(kThreads), fr::kSmemBytes, stream, x_map,
+                            w_map, p, n_pad);
   }
   p.tiles_per_cta = tiles_per_cta(ntiles, kHeadsA);
   p.out = out; p.status = status;
   const int64_t grid = (ntiles + p.tiles_per_cta - 1) / p.tiles_per_cta * kHeadsA;
   if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;
-  out_absorb_kernel<<<(unsigned)grid, kThreads, oa::kSmemBytes, stream>>>(a_map, w_map, p);
-  return dsa_host::check_launch();
+  return dsa_host::launch(out_absorb_kernel, dim3((unsigned)grid), dim3(kThreads), oa::kSmemBytes, stream, a_map,
+                          w_map, p);
 }
 
 int launch_mla_kv_entry(const uint16_t* kv, const uint16_t* k_pe, const int32_t* pos, const float* rope_cs,
@@ -740,9 +750,8 @@ int launch_mla_kv_entry(const uint16_t* kv, const uint16_t* k_pe, const int32_t*
   if (rows == 0) return DSA_OK;
   const int64_t grid = (rows + 7) / 8;
   if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;
-  kv_entry_kernel<<<(unsigned)grid, 256, 0, stream>>>(kv, k_pe, pos, rope_cs, max_pos, rows, dst_row, kv_cache,
-                                                      cache_rows, status);
-  return dsa_host::check_launch();
+  return dsa_host::launch(kv_entry_kernel, dim3((unsigned)grid), dim3(256), 0, stream, kv, k_pe, pos, rope_cs, max_pos,
+                          rows, dst_row, kv_cache, cache_rows, status);
 }
 
 }  // namespace dsa

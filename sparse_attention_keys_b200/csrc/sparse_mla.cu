@@ -217,13 +217,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   const int32_t* idx_row = p.idx + bt * p.k + slot0;
   const uint32_t v_ring = smem_u32(smem + kOffV), rest_ring = smem_u32(smem + kOffRest);
 
-  // Start the first global reads before the set-up barrier: the first tile's indices (gather warps)
-  // and, into L2, each head's Q features 0..319 (softmax warps, staged into TMEM below).
-  int idx_first = -1;
-  if (warp >= kGatherWarp && warp < kQkWarp) {
-    const int slot = 8 * (warp - kGatherWarp) + (lane & 7);
-    if (slot < nslots) idx_first = __ldg(idx_row + slot);
-  } else if (warp < kSoftmaxWarps && ntiles > 0) {
+  // Start the Q reads before the set-up barrier: each head's features 0..319 into L2 (softmax
+  // warps, staged into TMEM below). No kernel of the stream that may still be running writes Q;
+  // the indices come from the preceding kernel and are read after grid_dep_wait.
+  if (warp < kSoftmaxWarps && ntiles > 0) {
     const char* qrow = reinterpret_cast<const char*>(p.q + (bt * kHeads + tid) * kDqk);
 #pragma unroll
     for (int i = 0; i < kQTmemRegions; ++i) asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + 128 * i));
@@ -253,6 +250,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  grid_dep_launch();                                 // the next kernel may start its set-up
 
   if (warp >= kQkWarp) {
     // ------------------------------------------------------------------ Q K^T issuers
@@ -294,6 +292,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       for (int r = kQTmemRegions; r < kRegions; ++r)
         tma_load_2d(q_sm + (r - kQTmemRegions) * kQRegion, &q_map, q_full, 64 * r, (int32_t)(bt * kHeads));
     }
+    grid_dep_wait();                                 // the indices come from the preceding kernel
     const uint16_t* kv_b = PAGED ? p.kv : p.kv + (int64_t)b * p.S_max * kDqk;
     const int32_t* pages = PAGED ? p.block_table + (int64_t)b * p.max_pages : nullptr;
     const uint32_t blk = (uint32_t)(lane >> 3) * kKvRegion;      // block of chunks L and L+32 in its ring slot
@@ -303,7 +302,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     };
     auto load_page = [&](int v) -> int { return (v >= 0 && v < p.S_max) ? __ldg(pages + (v >> p.page_shift)) : -1; };
     // dense: indices one tile ahead; paged: indices two tiles ahead, their page ids one tile ahead
-    int idx_next = idx_first;                        // load_idx(0), issued before the set-up barrier
+    int idx_next = load_idx(0);
     int pg_next = 0, idx_next2 = -1;
     if (PAGED) {
       idx_next2 = load_idx(1);
@@ -399,6 +398,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       tc_fence_before();
       mbar_arrive(q_full);
     }
+    grid_dep_wait();                                 // indices (preceding kernel); outputs written below
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     // slot j * 32 + lane of the next tile (paged: also the slot two tiles ahead and the next tile's page id)
@@ -552,6 +552,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 __global__ void __launch_bounds__(256) sparse_mla_combine_kernel(const MlaParams p, int64_t rows) {
   const int64_t wid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  grid_dep_wait();                                   // the partials come from the preceding kernel
+  grid_dep_launch();
   if (wid >= rows) return;
   const int64_t bt = wid / kHeads;
   const int head = (int)(wid - bt * kHeads);
@@ -642,12 +644,11 @@ static int launch_mla(const uint16_t* q, MlaParams p, cudaStream_t stream, void*
   if (!dsa_host::encode_tensor_map_2d(&q_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (void*)q, kDqk,
                                       (uint64_t)BT * kHeads, kDqk * 2, 64, kHeads, CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
-  sparse_mla_kernel<PAGED><<<(unsigned)grid, kMlaThreads, kSmemBytes, stream>>>(q_map, p);
-  int rc = dsa_host::check_launch();
+  int rc = dsa_host::launch(sparse_mla_kernel<PAGED>, dim3((unsigned)grid), dim3(kMlaThreads), kSmemBytes, stream,
+                            q_map, p);
   if (rc != DSA_OK || s.nsplit == 1) return rc;
   const int64_t rows = BT * kHeads;
-  sparse_mla_combine_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p, rows);
-  return dsa_host::check_launch();
+  return dsa_host::launch(sparse_mla_combine_kernel, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, stream, p, rows);
 }
 
 int launch_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T,

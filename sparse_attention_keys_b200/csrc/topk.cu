@@ -98,6 +98,8 @@ __global__ void __launch_bounds__(kTopkThreads, 4) topk_kernel(const float* __re
   const int64_t row = blockIdx.x;
   const int b = (int)(row / T);
   const int tid = threadIdx.x;
+  grid_dep_wait();                             // the scores come from the preceding kernel
+  grid_dep_launch();
   int32_t* out = idx + row * (int64_t)k;
   int n = min(q_pos[row] + 1, kv_len[b]);
   if (n < 0) n = 0;
@@ -291,9 +293,8 @@ int launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int
       return DSA_ERR_CUDA;
     configured_smem = (int)smem;
   }
-  topk_kernel<<<(unsigned)rows, kTopkThreads, smem, stream>>>(scores, ld, q_pos, kv_len, T, k, max_row, flags,
-                                                              sort_n, idx, status);
-  return dsa_host::check_launch();
+  return dsa_host::launch(topk_kernel, dim3((unsigned)rows), dim3(kTopkThreads), smem, stream, scores, ld, q_pos,
+                          kv_len, T, k, max_row, flags, sort_n, idx, status);
 }
 
 }  // namespace dsa
