@@ -11,6 +11,8 @@
 // radix select (12, 10, 10 bits) finds the k-th largest key with shared-memory histograms, and a
 // compaction (four keys per lane, warp shuffle scans of the per-lane counts) writes the selected
 // positions in order. HBM-bound: 4 B read per visible score, 4 B written per selected index.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -58,6 +60,32 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool acti
   if (active) atomicAdd(&hist[bin], 1u);
 }
 
+// The radix digit holding the `remaining`-th largest key: bins are scanned from the top; thread t
+// owns bins nb-1-t*c .. nb-(t+1)*c (c = nb / threads). Writes the digit and how many keys of that
+// digit are still needed to *digit / *rem (shared); all threads call it; ends with a barrier.
+__device__ void select_digit(const uint32_t* hist, int nb, uint32_t remaining, uint32_t* warp_tot,
+                             uint32_t* digit, uint32_t* rem) {
+  const int tid = threadIdx.x;
+  const int c = nb / kTopkThreads;
+  uint32_t local = 0;
+  for (int j = 0; j < c; ++j) local += hist[nb - 1 - tid * c - j];
+  const uint32_t incl = block_inclusive_scan(local, warp_tot);
+  uint32_t before = incl - local;
+  if (before < remaining && remaining <= incl) {
+    for (int j = 0; j < c; ++j) {
+      const int bin = nb - 1 - tid * c - j;
+      const uint32_t h = hist[bin];
+      if (before + h >= remaining) {
+        *digit = (uint32_t)bin;
+        *rem = remaining - before;
+        break;
+      }
+      before += h;
+    }
+  }
+  __syncthreads();
+}
+
 // Ascending bitonic sort of buf[0, n) (n a power of two) by the CTA, then out[i] = the position in
 // the low word of buf[i] for i < count, and -1 for count <= i < k.
 __device__ void sort_and_write(uint64_t* buf, int n, int count, int k, int32_t* out) {
@@ -82,22 +110,25 @@ __global__ void __launch_bounds__(kTopkThreads, 4) topk_kernel(const float* __re
                                                             int64_t ld,
                                                             const int32_t* __restrict__ q_pos,
                                                             const int32_t* __restrict__ kv_len,
-                                                            int T, int k, int max_row,
+                                                            int T, int k, int max_row, int cand_cap,
                                                             uint32_t flags, int sort_n,
                                                             int32_t* __restrict__ idx,
                                                             int* status) {
   extern __shared__ __align__(16) uint32_t smem[];
   uint32_t* hist = smem;                       // kHistBins
   uint32_t* keys = smem + kHistBins;           // max_row (rounded up to 4)
+  uint32_t* cand = keys + ((max_row + 3) & ~3);  // cand_cap positions (a multiple of 4)
   // DSA_SORTED: sort_n (a power of two >= k) 64-bit keys, (~score key) << 32 | position
-  uint64_t* sbuf = reinterpret_cast<uint64_t*>(smem + kHistBins + ((max_row + 3) & ~3));
+  uint64_t* sbuf = reinterpret_cast<uint64_t*>(cand + cand_cap);
   const bool sorted = (flags & DSA_SORTED) != 0;
   __shared__ uint32_t warp_tot[kTopkWarps];
-  __shared__ uint32_t sel_digit, sel_remaining;
+  __shared__ uint32_t sel_digit, sel_remaining, n_cand_sh;
+  __shared__ uint32_t gt_off[kTopkWarps], eq_off[kTopkWarps];
 
   const int64_t row = blockIdx.x;
   const int b = (int)(row / T);
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   grid_dep_wait();                             // the scores come from the preceding kernel
   grid_dep_launch();
   int32_t* out = idx + row * (int64_t)k;
@@ -114,7 +145,11 @@ __global__ void __launch_bounds__(kTopkThreads, 4) topk_kernel(const float* __re
     return;
   }
 
-  // Stage the visible scores as keys (zero-padded to a multiple of four).
+  // Stage the visible scores as keys (zero-padded to a multiple of four) and histogram their top
+  // 12 bits (the first radix digit) on the way.
+  for (int i = tid; i < kHistBins; i += kTopkThreads) hist[i] = 0;
+  if (tid == 0) n_cand_sh = 0;
+  __syncthreads();
   const float* src = scores + row * ld;
   const int n4 = n >> 2;
   constexpr int kInFlight = 4;                 // float4 loads issued before any is used
@@ -128,14 +163,21 @@ __global__ void __launch_bounds__(kTopkThreads, 4) topk_kernel(const float* __re
 #pragma unroll
     for (int u = 0; u < kInFlight; ++u) {
       const int i = i0 + u * kTopkThreads + tid;
-      if (i < n4)
-        reinterpret_cast<uint4*>(keys)[i] =
-            make_uint4(order_key(f[u].x), order_key(f[u].y), order_key(f[u].z), order_key(f[u].w));
+      if (i < n4) {
+        const uint4 kk = make_uint4(order_key(f[u].x), order_key(f[u].y), order_key(f[u].z), order_key(f[u].w));
+        reinterpret_cast<uint4*>(keys)[i] = kk;
+        atomicAdd(&hist[kk.x >> 20], 1u);
+        atomicAdd(&hist[kk.y >> 20], 1u);
+        atomicAdd(&hist[kk.z >> 20], 1u);
+        atomicAdd(&hist[kk.w >> 20], 1u);
+      }
     }
   }
   if (tid < 4 && (n4 << 2) + tid < ((n + 3) & ~3)) {   // the n % 4 tail
     const int i = (n4 << 2) + tid;
-    keys[i] = i < n ? order_key(src[i]) : 0u;
+    const uint32_t kv = i < n ? order_key(src[i]) : 0u;
+    keys[i] = kv;
+    if (i < n) atomicAdd(&hist[kv >> 20], 1u);
   }
   __syncthreads();
 
@@ -146,60 +188,59 @@ __global__ void __launch_bounds__(kTopkThreads, 4) topk_kernel(const float* __re
     return;
   }
 
-  // Radix select of the k-th largest key: digits of 12, 10 and 10 bits from the top.
-  uint32_t prefix = 0, prefix_mask = 0, remaining = (uint32_t)k;
-#pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = pass == 0 ? 20 : (pass == 1 ? 10 : 0);
-    const int nb = pass == 0 ? 4096 : 1024;
-    {
-      for (int i = tid; i < nb; i += kTopkThreads) hist[i] = 0;
-      __syncthreads();
-      // four keys per thread per step (the keys array is zero-padded to a multiple of four)
-      for (int i4 = tid; 4 * i4 < n; i4 += kTopkThreads) {
-        const uint4 kk = reinterpret_cast<const uint4*>(keys)[i4];
-        const int i = 4 * i4;
-        hist_add(hist, (kk.x >> shift) & (nb - 1), (kk.x & prefix_mask) == prefix);
-        hist_add(hist, (kk.y >> shift) & (nb - 1), i + 1 < n && (kk.y & prefix_mask) == prefix);
-        hist_add(hist, (kk.z >> shift) & (nb - 1), i + 2 < n && (kk.z & prefix_mask) == prefix);
-        hist_add(hist, (kk.w >> shift) & (nb - 1), i + 3 < n && (kk.w & prefix_mask) == prefix);
-      }
-    }
-    __syncthreads();
-    // thread t owns bins nb-1-t*c .. nb-(t+1)*c (descending); c = nb / threads
-    const int c = nb / kTopkThreads;
-    uint32_t local = 0;
-    for (int j = 0; j < c; ++j) local += hist[nb - 1 - tid * c - j];
-    const uint32_t incl = block_inclusive_scan(local, warp_tot);
-    uint32_t before = incl - local;
-    if (before < remaining && remaining <= incl) {
-      for (int j = 0; j < c; ++j) {
-        const int bin = nb - 1 - tid * c - j;
-        const uint32_t h = hist[bin];
-        if (before + h >= remaining) {
-          sel_digit = (uint32_t)bin;
-          sel_remaining = remaining - before;
-          break;
-        }
-        before += h;
-      }
-    }
-    __syncthreads();
-    prefix |= sel_digit << shift;
-    prefix_mask |= (uint32_t)(nb - 1) << shift;
-    remaining = sel_remaining;
-    __syncthreads();
-  }
-  const uint32_t thr = prefix;           // the k-th largest key
-  const uint32_t need_eq = remaining;    // how many keys equal to thr are selected
+  // First digit (12 bits) of the k-th largest key, from the staged histogram.
+  select_digit(hist, 4096, (uint32_t)k, warp_tot, &sel_digit, &sel_remaining);
+  const uint32_t d1 = sel_digit;
+  const uint32_t rem1 = sel_remaining;
 
-  // Compaction in ascending position order. Warp w owns a contiguous chunk of whole 128-key steps;
-  // in each step lane l holds keys 4l..4l+3 (one 16-byte shared-memory load).
-  const int warp = tid >> 5, lane = tid & 31;
+  // Warp w owns a contiguous chunk of whole 128-key steps; in each step lane l holds keys
+  // 4l..4l+3 (one 16-byte shared-memory load).
   const int steps = (n + 127) / 128;
   const int per_warp = (steps + kTopkWarps - 1) / kTopkWarps;
   const int s_beg = min(steps, warp * per_warp), s_end = min(steps, s_beg + per_warp);
-  auto classify = [&](int st, uint32_t& gt4, uint32_t& eq4) {   // 4-bit masks of keys > thr, == thr
+
+  // Candidate sweep: keys above the first digit are selected for sure (counted per warp); the
+  // positions of keys on it are collected (in no particular order) for the last two digits.
+  uint32_t n_def = 0;
+  for (int st = s_beg; st < s_end; ++st) {
+    const int i = st * 128 + 4 * lane;
+    uint32_t def4 = 0, cand4 = 0;
+    if (i < n) {
+      const uint4 kk = reinterpret_cast<const uint4*>(keys)[i >> 2];
+      const uint32_t v[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const bool in = i + u < n;
+        def4 |= (uint32_t)(in && (v[u] >> 20) > d1) << u;
+        cand4 |= (uint32_t)(in && (v[u] >> 20) == d1) << u;
+      }
+    }
+    n_def += __popc(def4);
+    const uint32_t c = __popc(cand4);
+    uint32_t incl = c;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint32_t o = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += o;
+    }
+    const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+    uint32_t base = 0;
+    if (lane == 0 && total) base = atomicAdd(&n_cand_sh, total);
+    uint32_t slot = __shfl_sync(0xffffffffu, base, 0) + incl - c;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if ((cand4 >> u) & 1u) {
+        if (slot < (uint32_t)cand_cap) cand[slot] = (uint32_t)(i + u);
+        ++slot;
+      }
+  }
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) n_def += __shfl_xor_sync(0xffffffffu, n_def, d);
+  if (lane == 0) { gt_off[warp] = n_def; eq_off[warp] = 0; }
+  __syncthreads();
+  const uint32_t n_cand = n_cand_sh;
+
+  auto classify = [&](int st, uint32_t thr, uint32_t& gt4, uint32_t& eq4) {   // 4-bit masks of keys > thr, == thr
     const int i = st * 128 + 4 * lane;
     gt4 = 0; eq4 = 0;
     if (i < n) {
@@ -213,22 +254,78 @@ __global__ void __launch_bounds__(kTopkThreads, 4) topk_kernel(const float* __re
       }
     }
   };
-  uint32_t n_gt = 0, n_eq = 0;
-  for (int st = s_beg; st < s_end; ++st) {
-    uint32_t g4, e4;
-    classify(st, g4, e4);
-    n_gt += __popc(g4);
-    n_eq += __popc(e4);
-  }
+
+  uint32_t thr, need_eq;
+  if (n_cand <= (uint32_t)cand_cap) {
+    // digits 2 and 3 (10 bits each) over the candidates only
+    uint32_t prefix = d1 << 20, mask = 0xFFF00000u, remaining = rem1;
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+      const int shift = pass == 0 ? 10 : 0;
+      for (int i = tid; i < 1024; i += kTopkThreads) hist[i] = 0;
+      __syncthreads();
+      for (uint32_t j = tid; j < n_cand; j += kTopkThreads) {
+        const uint32_t kv = keys[cand[j]];
+        if ((kv & mask) == prefix) atomicAdd(&hist[(kv >> shift) & 1023u], 1u);
+      }
+      __syncthreads();
+      select_digit(hist, 1024, remaining, warp_tot, &sel_digit, &sel_remaining);
+      prefix |= sel_digit << shift;
+      mask |= 1023u << shift;
+      remaining = sel_remaining;
+      __syncthreads();
+    }
+    thr = prefix;
+    need_eq = remaining;
+    // the candidates above / at the threshold, added to their warp chunk's counts
+    for (uint32_t j = tid; j < n_cand; j += kTopkThreads) {
+      const uint32_t pos = cand[j];
+      const uint32_t kv = keys[pos];
+      const int w = (int)(pos >> 7) / per_warp;
+      if (kv > thr) atomicAdd(&gt_off[w], 1u);
+      else if (kv == thr) atomicAdd(&eq_off[w], 1u);
+    }
+  } else {
+    // too many keys on the first digit: digits 2 and 3 over all keys, then per-warp counts
+    uint32_t prefix = d1 << 20, mask = 0xFFF00000u, remaining = rem1;
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+      const int shift = pass == 0 ? 10 : 0;
+      for (int i = tid; i < 1024; i += kTopkThreads) hist[i] = 0;
+      __syncthreads();
+      for (int i4 = tid; 4 * i4 < n; i4 += kTopkThreads) {
+        const uint4 kk = reinterpret_cast<const uint4*>(keys)[i4];
+        const int i = 4 * i4;
+        hist_add(hist, (kk.x >> shift) & 1023u, (kk.x & mask) == prefix);
+        hist_add(hist, (kk.y >> shift) & 1023u, i + 1 < n && (kk.y & mask) == prefix);
+        hist_add(hist, (kk.z >> shift) & 1023u, i + 2 < n && (kk.z & mask) == prefix);
+        hist_add(hist, (kk.w >> shift) & 1023u, i + 3 < n && (kk.w & mask) == prefix);
+      }
+      __syncthreads();
+      select_digit(hist, 1024, remaining, warp_tot, &sel_digit, &sel_remaining);
+      prefix |= sel_digit << shift;
+      mask |= 1023u << shift;
+      remaining = sel_remaining;
+      __syncthreads();
+    }
+    thr = prefix;
+    need_eq = remaining;
+    uint32_t n_gt = 0, n_eq = 0;
+    for (int st = s_beg; st < s_end; ++st) {
+      uint32_t g4, e4;
+      classify(st, thr, g4, e4);
+      n_gt += __popc(g4);
+      n_eq += __popc(e4);
+    }
 #pragma unroll
-  for (int d = 16; d > 0; d >>= 1) {
-    n_gt += __shfl_xor_sync(0xffffffffu, n_gt, d);
-    n_eq += __shfl_xor_sync(0xffffffffu, n_eq, d);
+    for (int d = 16; d > 0; d >>= 1) {
+      n_gt += __shfl_xor_sync(0xffffffffu, n_gt, d);
+      n_eq += __shfl_xor_sync(0xffffffffu, n_eq, d);
+    }
+    if (lane == 0) { gt_off[warp] = n_gt; eq_off[warp] = n_eq; }
   }
-  // exclusive offsets across warps (lane 0 of each warp contributes its counts)
-  __shared__ uint32_t gt_off[kTopkWarps], eq_off[kTopkWarps];
-  if (lane == 0) { gt_off[warp] = n_gt; eq_off[warp] = n_eq; }
   __syncthreads();
+  // exclusive offsets across warps
   if (tid == 0) {
     uint32_t g = 0, e = 0;
     for (int w = 0; w < kTopkWarps; ++w) {
@@ -238,10 +335,13 @@ __global__ void __launch_bounds__(kTopkThreads, 4) topk_kernel(const float* __re
     }
   }
   __syncthreads();
+
+  // Write sweep in ascending position order: keys above the threshold, and the first need_eq keys
+  // equal to it (ties go to the smaller position).
   uint32_t gt_seen = gt_off[warp], eq_seen = eq_off[warp];
   for (int st = s_beg; st < s_end; ++st) {
     uint32_t g4, e4;
-    classify(st, g4, e4);
+    classify(st, thr, g4, e4);
     // exclusive prefix of the per-lane counts (lane order = position order)
     uint32_t gi = __popc(g4), ei = __popc(e4);
 #pragma unroll
@@ -285,7 +385,9 @@ int launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int
   if (flags & DSA_SORTED)
     for (sort_n = 1; sort_n < k; sort_n <<= 1) {
     }
-  const size_t smem = (size_t)(kHistBins + ((max_row + 3) & ~3)) * sizeof(uint32_t) + (size_t)sort_n * 8;
+  // candidate positions on the first radix digit: a quarter of the longest row (at least 256)
+  const int cand_cap = std::max(256, ((max_row + 3) & ~3) / 4 / 4 * 4);
+  const size_t smem = (size_t)(kHistBins + ((max_row + 3) & ~3) + cand_cap) * sizeof(uint32_t) + (size_t)sort_n * 8;
   static int configured_smem = 0;
   if ((int)smem > configured_smem) {
     if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -294,7 +396,7 @@ int launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int
     configured_smem = (int)smem;
   }
   return dsa_host::launch(topk_kernel, dim3((unsigned)rows), dim3(kTopkThreads), smem, stream, scores, ld, q_pos,
-                          kv_len, T, k, max_row, flags, sort_n, idx, status);
+                          kv_len, T, k, max_row, cand_cap, flags, sort_n, idx, status);
 }
 
 }  // namespace dsa

@@ -218,6 +218,33 @@ def test_topk_sorted_on_synthetic_scores(table_dev, k):
     assert np.array_equal(got, want)
 
 
+@pytest.mark.parametrize("in_band", [1024, 1025, 2500])
+def test_topk_first_digit_crowded(table_dev, in_band):
+    """Rows whose k-th largest score sits in a band of `in_band` keys sharing the top 12 key bits
+    ([1.0, 1.125): sign, exponent and 3 mantissa bits). Rows of 4096 hold up to 1024 such candidate
+    positions for the last two radix digits; past that the kernel runs those digits over every key.
+    Both paths must give the oracle's selection, in both output orders."""
+    rng = np.random.default_rng(50 + in_band)
+    S, k = 4096, 2048
+    above = 1500                                         # larger than the band: always selected
+    rows = []
+    for _ in range(3):
+        v = np.empty(S, np.float32)
+        v[:above] = rng.uniform(2.0, 3.0, above)
+        v[above:above + in_band] = 1.0 + rng.uniform(0.0, 0.124, in_band)
+        v[above + in_band:] = rng.uniform(-3.0, 0.9, S - above - in_band)
+        v[above + 5:above + 40] = v[above + 5]           # ties inside the band
+        rows.append(rng.permutation(v))
+    sc = np.stack(rows)[None]                            # [1, 3, S]
+    q_pos = np.full((1, 3), S - 1, np.int32)
+    kv_len = np.array([S], np.int32)
+    got = _gpu_topk(sc, q_pos, kv_len, k)
+    gs = dsa.dsa_topk(P.to_dev(sc), P.to_dev(q_pos), P.to_dev(kv_len), k, flags=dsa.DSA_SORTED).cpu().numpy()
+    assert _status() == 0
+    assert np.array_equal(got, O.topk_indices(sc.astype(np.float64), q_pos, kv_len, k))
+    assert np.array_equal(gs, O.topk_indices(sc.astype(np.float64), q_pos, kv_len, k, sorted_by_score=True))
+
+
 def test_topk_longest_row_and_overlong_row(table_dev):
     rng = np.random.default_rng(31)
     S = 32768
