@@ -7,10 +7,13 @@
 // ascending position, via a bitonic sort in shared memory), then -1 padding.
 //
 // One CTA per score row. The row's visible scores are staged once into shared memory as
-// order-preserving 32-bit keys (coalesced 16-byte loads, four in flight per thread); a 3-pass
-// radix select (12, 10, 10 bits) finds the k-th largest key with shared-memory histograms, and a
-// compaction (four keys per lane, warp shuffle scans of the per-lane counts) writes the selected
-// positions in order. HBM-bound: 4 B read per visible score, 4 B written per selected index.
+// order-preserving 32-bit keys (coalesced 16-byte loads, four in flight per thread), histogramming
+// their top 12 bits on the way. A radix select finds the k-th largest key: the first digit (12 bits)
+// from that histogram, then one sweep counts the keys above it per warp chunk and collects the
+// positions of the keys on it, and the last two digits (10 bits each) run over those candidates only
+// (over every key if they exceed a quarter of the row). A compaction (four keys per lane, warp
+// shuffle scans of the per-lane counts) writes the selected positions in order. HBM-bound: 4 B read
+// per visible score, 4 B written per selected index.
 #include <algorithm>
 
 #include "common.cuh"
