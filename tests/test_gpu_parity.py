@@ -397,3 +397,32 @@ def test_pipeline_end_to_end(table_dev, name):
     gs = dsa.dsa_topk(sc, P.to_dev(inp.q_pos), P.to_dev(inp.kv_len), k, flags=dsa.DSA_SORTED).cpu().numpy()
     assert np.array_equal(gs, O.topk_indices(own, inp.q_pos, inp.kv_len, k, sorted_by_score=True))
     _check_mla(out.float().cpu().numpy(), lse.cpu().numpy(), inp.mla_q, inp.mla_kv, gidx)
+
+
+def test_pipeline_degenerate_sequences(table_dev):
+    """Decode over sequences with nothing visible (kv_len 0), one visible key, and a ragged normal
+    context: masked scores are -inf, an empty selection is all -1 and gives zero output with
+    lse -inf, a single key gets all the weight (the output is that latent row), and the normal
+    sequence matches the oracle."""
+    kv_len = [0, 1, 300]
+    B, S, k = 3, 320, 64
+    inp = DI.make_custom(B, 1, S, k, decode=True, seed=60, kv_len=kv_len)
+    q8, qs, k8, ks = _quantised(inp)
+    ld = S
+    sc = torch.full((B, 1, ld), 5.0, dtype=torch.float32, device="cuda")
+    dsa.dsa_index_scores(P.to_dev(q8), P.to_dev(qs), P.to_dev(inp.idx_w), P.to_dev(k8), P.to_dev(ks),
+                         P.to_dev(inp.q_pos), P.to_dev(inp.kv_len), scores=sc, ld=ld, flags=dsa.DSA_FILL_MASKED)
+    idx = dsa.dsa_topk(sc, P.to_dev(inp.q_pos), P.to_dev(inp.kv_len), k)
+    out, lse = dsa.dsa_sparse_mla(P.bf16_dev(inp.mla_q), P.bf16_dev(inp.mla_kv), idx)
+    assert _status() == 0
+    s, i, o, l = sc.cpu().numpy(), idx.cpu().numpy(), out.float().cpu().numpy(), lse.cpu().numpy()
+    assert np.all(np.isneginf(s[0, 0])) and np.all(i[0, 0] == -1)
+    assert np.all(o[0] == 0) and np.all(np.isneginf(l[0]))
+    assert np.all(np.isneginf(s[1, 0, 1:])) and np.isfinite(s[1, 0, 0])
+    assert i[1, 0, 0] == 0 and np.all(i[1, 0, 1:] == -1)
+    assert np.array_equal(o[1, 0], np.broadcast_to(O.bf16_to_f64(inp.mla_kv[1, 0, :512]), (128, 512)))
+    ref = O.index_scores(q8, qs, inp.idx_w, k8, ks, inp.q_pos, inp.kv_len)
+    mag = O.index_score_magnitude(q8, qs, inp.idx_w, k8, ks, inp.q_pos, inp.kv_len)
+    P.check_scores(s[2], ref[2], mag[2], O.valid_len(inp.q_pos, inp.kv_len)[2])
+    assert np.array_equal(i[2], O.topk_indices(s[2:3].astype(np.float64), inp.q_pos[2:3], inp.kv_len[2:3], k)[0])
+    _check_mla(o[2:3], l[2:3], inp.mla_q[2:3], inp.mla_kv[2:3], i[2:3])
