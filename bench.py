@@ -13,6 +13,10 @@ events) when the inputs fit in L2; the K step times are summed, ranks barrier + 
 and after, and rank 0 reports the max over ranks. After each timed step a second graph of the same
 step, with an event pair around each ABI call, is replayed for the per-kernel durations (the
 roofline's kernel time); its event nodes would lengthen the step, so it is not part of the step time.
+The end-to-end figure (`e2e`) goes through the public API with host buffers: each step copies its
+inputs host -> device from pinned memory and reads its results back, and the steps rotate over
+independent slots on their own streams so that copies overlap kernels. Each slot's copies and
+calls are captured once as a CUDA graph and replayed; `e2e.eager` issues them from Python every step.
 Under torchrun each rank runs its own replica of the workload (independent sequences, no
 collective on the data path): weak scaling.
 
@@ -164,7 +168,7 @@ class ClockSampler:
 class Step:
     """Device-resident state and the ABI calls of one step."""
 
-    def __init__(self, inp, device):
+    def __init__(self, inp, device, flush_buffers=True):
         import torch
         import sparse_attention_keys_b200 as dsa
         self.dsa, self.torch, self.inp = dsa, torch, inp
@@ -222,8 +226,9 @@ class Step:
                                [self.kcache, self.kscale] + ([self.kv] if self.kv is not None else []) +
                                list(self.d.values()))
         self.flush_writes = self.input_bytes <= 2 * L2_BYTES
-        self.flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-        self.flush_src = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        fb = L2_FLUSH_BYTES // 4 if flush_buffers else 1
+        self.flush = torch.empty(fb, dtype=torch.float32, device=dev)
+        self.flush_src = torch.ones(fb, dtype=torch.float32, device=dev)
         self.h_idx = torch.empty((B, T, self.k), dtype=torch.int32).pin_memory()
         self.h_out = torch.empty((B, T, 128, 512), dtype=torch.bfloat16).pin_memory() if self.out is not None else None
         self.h_lse = torch.empty((B, T, 128), dtype=torch.float32).pin_memory() if self.out is not None else None
@@ -378,31 +383,77 @@ def run_ours(args, rank, world, local_rank):
     del graph, graph_k
     check_status(dsa, "graph replays")
 
-    # ---- end to end through host buffers (pinned H2D of the step inputs, D2H of the results)
-    for _ in range(max(1, args.warmup)):
-        st.l2_flush()
-        st.h2d(); st.run(); st.d2h()
-    barrier()
-    e2e = []
-    for _ in range(args.steps):
-        st.l2_flush()
+    # ---- end to end through the public API with host buffers: every step copies its inputs host ->
+    # device from pinned memory, runs the calls and reads its results back. Steps rotate over
+    # independent slots (device state, pinned buffers, a stream each), so one step's copies overlap
+    # another's kernels, as a serving loop would run them. When the step's inputs fit in the L2,
+    # enough slots rotate that their data exceeds twice the L2: no slot finds its own data resident.
+    n_slots = 2
+    if st.flush_writes:
+        n_slots = max(2, math.ceil(2 * L2_BYTES / max(1, st.input_bytes)) + 1)
+    slots = [st] + [Step(inp, dev, flush_buffers=False) for _ in range(n_slots - 1)]
+    streams = [torch.cuda.Stream() for _ in slots]
+
+    def e2e_step(i):
+        j = i % n_slots
+        with torch.cuda.stream(streams[j]):
+            slots[j].h2d()
+            slots[j].run()
+            slots[j].d2h()
+
+    def timed_rotation(step_fn):
+        cur = torch.cuda.current_stream()
         s = torch.cuda.Event(enable_timing=True)
         e = torch.cuda.Event(enable_timing=True)
-        s.record()
-        st.h2d()
-        st.run()
-        st.d2h()
-        e.record()
-        e2e.append((s, e))
+        s.record(cur)
+        for sj in streams:
+            sj.wait_event(s)
+        for i in range(args.steps):
+            step_fn(i)
+        for sj in streams:
+            cur.wait_stream(sj)
+        e.record(cur)
+        torch.cuda.synchronize()
+        barrier()
+        return s.elapsed_time(e) / 1e3
+
+    for i in range(max(1, args.warmup) * n_slots):
+        e2e_step(i)
+    torch.cuda.synchronize()
     barrier()
-    t_e2e = sum(s.elapsed_time(e) for s, e in e2e) / 1e3
+    t_e2e_eager = timed_rotation(e2e_step)      # each call issued from Python every step
     check_status(dsa, "end-to-end steps")
+    # The same steps with each slot's copies and API calls captured once as a CUDA graph on its
+    # stream and replayed: every replay still copies the inputs in and the results out.
+    graphs = []
+    for j, sl in enumerate(slots):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=streams[j]):
+            sl.h2d()
+            sl.run()
+            sl.d2h()
+        graphs.append(g)
+    torch.cuda.synchronize()
+
+    def graph_step(i):
+        j = i % n_slots
+        with torch.cuda.stream(streams[j]):
+            graphs[j].replay()
+
+    for i in range(max(1, args.warmup) * n_slots):
+        graph_step(i)
+    torch.cuda.synchronize()
+    barrier()
+    t_e2e = timed_rotation(graph_step)
+    check_status(dsa, "end-to-end graph steps")
+    del graphs
+    del slots[1:]
 
     producers = None if (args.no_producers or st.kv is None) else time_producers(st, args, dev)
     paged = None if (args.no_producers or st.kv is None) else time_paged(st, args, dev)
 
     # ---- max over ranks
-    t_dev, t_e2e = max_over_ranks([t_dev, t_e2e], world, dev)
+    t_dev, t_e2e, t_e2e_eager = max_over_ranks([t_dev, t_e2e, t_e2e_eager], world, dev)
     if rank != 0:
         return None
 
@@ -434,11 +485,16 @@ def run_ours(args, rank, world, local_rank):
         "kernel_ms": {n: v * 1e3 for n, v in per_kernel.items()},
         "roofline": roof,
         "e2e": {"value": weak_scaling_value(units["pairs"], args.steps, world, t_e2e), "unit": UNIT, "h2d_bytes_per_step": st.bytes_h2d(),
-                "d2h_bytes_per_step": st.bytes_d2h(), "ms_per_step": t_e2e / args.steps * 1e3},
+                "d2h_bytes_per_step": st.bytes_d2h(), "ms_per_step": t_e2e / args.steps * 1e3,
+                "pipelined_slots": n_slots,
+                "eager": {"value": weak_scaling_value(units["pairs"], args.steps, world, t_e2e_eager),
+                          "ms_per_step": t_e2e_eager / args.steps * 1e3}},
         "gpu_launches": st.launches_per_step * args.steps,
         "timing": ("device: CUDA-graph replay of the step, CUDA events around each replay; kernel_ms and "
                    "roofline: a replay of the same step with CUDA events around each call, after each "
-                   "timed step; e2e: plain API calls"),
+                   "timed step; e2e: the API calls with host copies in and out every step, captured per "
+                   "slot as a CUDA graph and replayed, steps rotating over independent slots on their own "
+                   "streams (e2e.eager: the same calls issued from Python every step)"),
         "clocks": clocks,
     }
     if producers is not None:
