@@ -20,6 +20,12 @@
  *   - All tensor pointers are DEVICE pointers unless a comment says "host". The caller owns
  *     every buffer; the library allocates nothing in these calls and keeps no per-call state.
  *   - Calls are asynchronous and ordered on `stream` (NULL = the legacy default stream).
+ *     Kernels are launched with programmatic stream serialisation: each may start while the
+ *     previous kernel on the stream finishes, and waits for it (griddepcontrol.wait) before
+ *     reading or writing anything an earlier kernel touches. Each also lets the next kernel start
+ *     early. A caller's kernel launched with the same attribute right after a dsa call must
+ *     therefore wait the same way (cudaGridDependencySynchronize) before reading its outputs.
+ *     Kernels launched without it see plain stream order.
  *   - Return value: DSA_OK, or an error code for arguments rejected on the host before any
  *     launch (nothing is launched then) or a failed launch. Errors found on the device
  *     (index or position out of range, a bounded wait that ran out) are recorded in a device
