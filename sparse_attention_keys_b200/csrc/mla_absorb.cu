@@ -154,7 +154,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&w_map);
       mbar_arrive_expect_tx(b_full, 4 * kRegion);
       for (int j = 0; j < 4; ++j) tma_load_3d(smem + qa::kOffB + j * kRegion, &w_map, b_full, 256 * n + 64 * j, 0, h);
-      for (int i = 0; i < my_tiles; ++i) {
+      // The two CTAs of a head (n = 0, 1) read the same q_nope tiles. Requested at the same moment
+      // both miss the L2; the second trails by the weight load, so its tiles come from the L2.
+      bool go = n == 0 || mbar_wait(b_full, 0, &abort_flag, p.status, DSA_SITE_ABSORB_W);
+      for (int i = 0; go && i < my_tiles; ++i) {
         const int s = i & 1;
         if (i >= 2 && !mbar_wait(&a_empty[s], ((i >> 1) + 1) & 1, &abort_flag, p.status, DSA_SITE_ABSORB_A_EMPTY))
           break;
@@ -196,12 +199,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* srow = smem + qa::kOffStage + r * qa::kRowBytes;
     for (int i = 0; i < my_tiles; ++i) {
       const int a = i & 1;
+      const int64_t t = (tile0 + i) * kRows + r;
+      if (i > 0) bulk_wait_read();                   // the previous row's copy has read the staging row
+      // the rotary part first: its loads do not depend on the MMAs and overlap them
+      if (n == 1 && t < p.rows) {
+        const int pos = __ldg(p.pos + t);
+        if (!rope_row(p.q_pe + (t * kHeadsA + h) * kRopeD, pos, p, reinterpret_cast<uint4*>(srow + 512)))
+          set_status(p.status, DSA_ERR_DEVICE_BOUNDS);
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[a], (i >> 1) & 1, &abort_flag, p.status,
                                              DSA_SITE_ABSORB_ACC_FULL)))
         break;
       tc_fence_after();
-      const int64_t t = (tile0 + i) * kRows + r;
-      if (i > 0) bulk_wait_read();                   // the previous row's copy has read the staging row
       const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + a * 256;
 #pragma unroll 1
       for (int c = 0; c < 8; c += 2) {
@@ -215,11 +224,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&acc_empty[a]);
       if (t < p.rows) {
-        if (n == 1) {
-          const int pos = __ldg(p.pos + t);
-          if (!rope_row(p.q_pe + (t * kHeadsA + h) * kRopeD, pos, p, reinterpret_cast<uint4*>(srow + 512)))
-            set_status(p.status, DSA_ERR_DEVICE_BOUNDS);
-        }
         fence_proxy_async_smem();
         bulk_store_s2g(p.out + (t * kHeadsA + h) * kQk + 256 * n, smem_u32(srow), n ? 640u : 512u);
         bulk_commit();
@@ -466,6 +470,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     const int quad = warp & 3, et = tid - 64;           // epilogue thread 0..127
     uint8_t* stage = smem + fr::kOffW;                   // rows of 1152 B over the consumed weights
+    // rotary inputs of this thread's (token, pair) entries, loaded while the MMAs run
+    constexpr int kPairsPerThread = fr::kMaxRows * 32 / 128;
+    uint32_t pe[kPairsPerThread];
+    float2 pcs[kPairsPerThread];
+    int pps[kPairsPerThread];
+#pragma unroll
+    for (int r = 0; r < kPairsPerThread; ++r) {
+      const int i = et + r * 128, t = i >> 5, pr = i & 31;
+      pps[r] = -1;
+      if (i < rows * 32) {
+        pps[r] = __ldg(p.pos + t);
+        pe[r] = __ldg(reinterpret_cast<const uint32_t*>(p.q_pe + ((int64_t)t * kHeadsA + h) * kRopeD) + pr);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kPairsPerThread; ++r) {
+      const int pr = (et + r * 128) & 31;
+      pcs[r] = make_float2(1.f, 0.f);
+      if (pps[r] >= 0 && pps[r] < p.max_pos)
+        pcs[r] = __ldg(reinterpret_cast<const float2*>(p.rope_cs + (int64_t)pps[r] * kRopeD) + pr);
+    }
     const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, &abort_flag, p.status, DSA_SITE_ABSORB_ACC_FULL));
     if (ok) {
       tc_fence_after();
@@ -481,14 +506,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // rotary part: thread = (token, pair)
-      for (int i = et; i < rows * 32; i += 128) {
-        const int t = i >> 5, pr = i & 31;
-        const int ps = __ldg(p.pos + t);
+#pragma unroll
+      for (int r = 0; r < kPairsPerThread; ++r) {
+        const int i = et + r * 128, t = i >> 5, pr = i & 31;
+        if (i >= rows * 32) continue;
         uint32_t o = 0u;
-        if (ps >= 0 && ps < p.max_pos) {
-          const uint32_t x = __ldg(reinterpret_cast<const uint32_t*>(p.q_pe + ((int64_t)t * kHeadsA + h) * kRopeD) + pr);
-          const float2 cs = __ldg(reinterpret_cast<const float2*>(p.rope_cs + (int64_t)ps * kRopeD) + pr);
-          const float a = __uint_as_float(x << 16), b = __uint_as_float(x & 0xFFFF0000u);
+        if (pps[r] >= 0 && pps[r] < p.max_pos) {
+          const float a = __uint_as_float(pe[r] << 16), b = __uint_as_float(pe[r] & 0xFFFF0000u);
+          const float2 cs = pcs[r];
           o = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)), __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
         } else if (pr == 0) {
           set_status(p.status, DSA_ERR_DEVICE_BOUNDS);
