@@ -217,9 +217,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   const int32_t* idx_row = p.idx + bt * p.k + slot0;
   const uint32_t v_ring = smem_u32(smem + kOffV), rest_ring = smem_u32(smem + kOffRest);
 
-  // Start the Q reads before the set-up barrier: each head's features 0..319 into L2 (softmax
-  // warps, staged into TMEM below). No kernel of the stream that may still be running writes Q;
-  // the indices come from the preceding kernel and are read after grid_dep_wait.
+  // Before the set-up barrier, hint each head's features 0..319 into L2 (softmax warps, staged into
+  // TMEM below). A prefetch is only a hint, so it is safe even if the preceding kernel is still
+  // writing Q; every actual read of Q, and of the indices, comes after grid_dep_wait.
   if (warp < kSoftmaxWarps && ntiles > 0) {
     const char* qrow = reinterpret_cast<const char*>(p.q + (bt * kHeads + tid) * kDqk);
 #pragma unroll
@@ -286,13 +286,13 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // gather warp w copies keys 8w..8w+7 of each tile; for every key, lane L copies the 16-byte
     // chunks L (block L/8), L+32 (block 4+L/8) and, for L < 8, L+64 (the rotary block)
     const int w = warp - kGatherWarp;
+    grid_dep_wait();                                 // Q and the indices may come from the preceding kernel
     if (w == 0 && lane == 0 && ntiles > 0) {
       prefetch_tensormap(&q_map);
       mbar_arrive_expect_tx(q_full, kQBytes);
       for (int r = kQTmemRegions; r < kRegions; ++r)
         tma_load_2d(q_sm + (r - kQTmemRegions) * kQRegion, &q_map, q_full, 64 * r, (int32_t)(bt * kHeads));
     }
-    grid_dep_wait();                                 // the indices come from the preceding kernel
     const uint16_t* kv_b = PAGED ? p.kv : p.kv + (int64_t)b * p.S_max * kDqk;
     const int32_t* pages = PAGED ? p.block_table + (int64_t)b * p.max_pages : nullptr;
     const uint32_t blk = (uint32_t)(lane >> 3) * kKvRegion;      // block of chunks L and L+32 in its ring slot
@@ -369,6 +369,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // ------------------------------------------------------------------ softmax warps (thread = head)
     const int h = tid;
     const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
+    grid_dep_wait();                                 // Q, the indices (earlier kernels); outputs written below
     // Q features 0..319 of head h -> TMEM as bf16 pairs (feature f in column f/2)
     if (ntiles > 0) {
       // two batches of loads, each fully in flight before its TMEM stores (which order memory)
@@ -398,7 +399,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       tc_fence_before();
       mbar_arrive(q_full);
     }
-    grid_dep_wait();                                 // indices (preceding kernel); outputs written below
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     // slot j * 32 + lane of the next tile (paged: also the slot two tiles ahead and the next tile's page id)

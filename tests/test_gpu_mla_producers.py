@@ -119,13 +119,16 @@ def test_mla_layer_absorbed_equals_unabsorbed(table_dev):
     dsa.dsa_mla_kv_entry(P.bf16_dev(cache_src.kv), P.bf16_dev(cache_src.k_pe), P.to_dev(kpos), table_dev,
                          P.to_dev(np.arange(S, dtype=np.int64)), cache)
     wkv_b, w_uk, w_uv = _weights(inp)
-    q = dsa.dsa_mla_q_absorb(P.bf16_dev(inp.q_nope), P.bf16_dev(inp.q_pe), P.to_dev(inp.pos), table_dev, w_uk)
     idx = np.full((1, T, k), -1, np.int32)
     for t in range(T):
         n = int(inp.pos[t]) + 1
         m = min(n, k)
         idx[0, t, :m] = rng.choice(n, m, replace=False)
-    o, _ = dsa.dsa_sparse_mla(q.view(1, T, 128, 576), cache.view(1, S, 576), P.to_dev(idx))
+    # every input on the device first, so that q absorption and sparse MLA are adjacent kernels on
+    # the stream: sparse MLA must not read q before the absorption has finished writing it
+    idx_dev, q_nope, q_pe, pos = P.to_dev(idx), P.bf16_dev(inp.q_nope), P.bf16_dev(inp.q_pe), P.to_dev(inp.pos)
+    q = dsa.dsa_mla_q_absorb(q_nope, q_pe, pos, table_dev, w_uk)
+    o, _ = dsa.dsa_sparse_mla(q.view(1, T, 128, 576), cache.view(1, S, 576), idx_dev)
     x = dsa.dsa_mla_out_absorb(o.view(T, 128, 512), w_uv)
     assert _status() == 0
     got = x.float().cpu().numpy()
