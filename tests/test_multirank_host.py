@@ -51,3 +51,43 @@ def test_two_rank_weak_scaling_plumbing():
     assert u0 == u1 == 1024                              # same shapes on every replica
     assert x0 != x1                                      # but independent data
     assert v0 == pytest.approx(1024 * 10 * 2 / 1.5)
+
+
+def _failing_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import time
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        # the failing rank: leaves between steps, before the timing reduction, without a collective
+        raise SystemExit(3)
+    import bench
+    t0 = time.time()
+    try:
+        bench.max_over_ranks([1.0, 2.0], world, "cpu")
+        q.put(("no error", time.time() - t0))
+    except Exception as e:                               # the lost peer surfaces as an error
+        q.put((type(e).__name__, time.time() - t0))
+    finally:
+        try:
+            dist.destroy_process_group()
+        except Exception:
+            pass
+
+
+def test_a_lost_rank_ends_the_reduction_with_an_error():
+    """Failure detection on the host: when a rank leaves, the surviving rank's max-over-ranks
+    reduction ends with an error (the process group's short timeout or the closed connection)
+    instead of waiting for ever."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert procs[1].exitcode == 3
+    what, waited = q.get(timeout=5)
+    assert what != "no error"
+    assert waited < 60
