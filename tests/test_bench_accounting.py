@@ -39,3 +39,14 @@ def test_producer_units():
     assert u["q_absorb"]["flops"] == 8 * 128 * 128 * 512 * 2
     assert u["out_absorb"]["bytes"] == 8 * 128 * (512 + 128) * 2 + w
     assert u["out_absorb"]["flops"] == u["q_absorb"]["flops"]
+
+
+def test_prefill_oracle_unit_counts_its_causal_pairs():
+    from oracle import dsa_oracle as O
+    wl = DI.Workload("p", batch=1, queries=64, s_max=64, topk=16, decode=False, with_mla=True)
+    inp = DI.make_inputs(wl)
+    table = O.rope_table(128)
+    caches = O.index_keys(inp.idx_k, np.arange(64)[None, :], table)
+    assert bench.oracle_prefill_rows(inp, 16, table, caches) == sum(t + 1 for t in range(16, 16 + bench.PREFILL_CHUNK))
+    units = bench._oracle_units(inp)
+    assert units[0] == ("rows", 0) and units[-1] == ("rows", 64 - bench.PREFILL_CHUNK)
