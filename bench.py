@@ -390,7 +390,8 @@ def run_ours(args, rank, world, local_rank):
     # enough slots rotate that their data exceeds twice the L2: no slot finds its own data resident.
     n_slots = 2
     if st.flush_writes:
-        n_slots = max(2, math.ceil(2 * L2_BYTES / max(1, st.input_bytes)) + 1)
+        n_slots = min(16, max(2, math.ceil(2 * L2_BYTES / max(1, st.input_bytes)) + 1))
+    slots_exceed_l2 = n_slots * st.input_bytes > 2 * L2_BYTES
     slots = [st] + [Step(inp, dev, flush_buffers=False) for _ in range(n_slots - 1)]
     streams = [torch.cuda.Stream() for _ in slots]
 
@@ -487,6 +488,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": weak_scaling_value(units["pairs"], args.steps, world, t_e2e), "unit": UNIT, "h2d_bytes_per_step": st.bytes_h2d(),
                 "d2h_bytes_per_step": st.bytes_d2h(), "ms_per_step": t_e2e / args.steps * 1e3,
                 "pipelined_slots": n_slots,
+                "slots_data_exceeds_2x_l2": slots_exceed_l2,
                 "eager": {"value": weak_scaling_value(units["pairs"], args.steps, world, t_e2e_eager),
                           "ms_per_step": t_e2e_eager / args.steps * 1e3}},
         "gpu_launches": st.launches_per_step * args.steps,
