@@ -435,10 +435,3 @@ def paged_gather(pool, block_table, page_size: int, seq_len) -> np.ndarray:
                 raise IndexError(f"sequence {b} position {s}: page id {page} outside the pool")
             out[b, s] = pool[page * page_size + s % page_size]
     return out
-
-
-def f64_to_bf16_bits(x) -> np.ndarray:
-    """Round float64 to bf16 (via the nearest fp32; the double rounding is far below the 2e-2 bar)."""
-    f = np.asarray(x, dtype=np.float32)
-    u = f.view(np.uint32).astype(np.uint64)
-    return ((u + (((u >> 16) & 1) + 0x7FFF)) >> 16).astype(np.uint16)

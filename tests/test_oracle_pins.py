@@ -206,20 +206,25 @@ def test_scores_two_head_golden_example():
         assert top[0, 0].tolist() == case["top2"]
 
 
-def _brute_scores(q8, qs, w, k8, ks, q_pos, kv_len, sm):
+def _brute_scores(q8, qs, w, k8, ks, q_pos, kv_len, sm, magnitude=False):
+    """Triple loop over (query, key, head) of the score; with magnitude=True the same sum with
+    every folded head weight replaced by its absolute value (the error scale of an accumulation
+    of mixed-sign terms)."""
     B, T, H, D = q8.shape
     S = k8.shape[1]
-    out = np.full((B, T, S), -np.inf)
+    out = np.full((B, T, S), -np.inf) if not magnitude else np.zeros((B, T, S))
     dec = {c: float(O.e4m3_decode(c)) for c in range(256)}
     for b in range(B):
         for t in range(T):
-            for s in range(min(q_pos[b][t] + 1, kv_len[b])):
+            n = min(q_pos[b][t] + 1, kv_len[b]) if not magnitude else S
+            for s in range(n):
                 tot = 0.0
                 for j in range(H):
                     dot = 0.0
                     for i in range(D):
                         dot += dec[int(q8[b, t, j, i])] * dec[int(k8[b, s, i])]
-                    tot += float(w[b, t, j]) * H ** -0.5 * float(qs[b, t, j]) * sm * max(dot, 0.0)
+                    wj = float(w[b, t, j]) * H ** -0.5 * float(qs[b, t, j]) * sm
+                    tot += (abs(wj) if magnitude else wj) * max(dot, 0.0)
                 out[b, t, s] = tot * float(ks[b, s])
     return out
 
@@ -241,6 +246,78 @@ def test_scores_bruteforce_small():
     assert np.array_equal(np.isinf(got), np.isinf(want))
     fin = np.isfinite(want)
     assert np.allclose(got[fin], want[fin], rtol=1e-12, atol=1e-12)
+
+
+def test_score_magnitude_bruteforce_mixed_sign_weights():
+    """index_score_magnitude (the denominator of the score parity bar) against the triple loop with
+    |w'_j|: a dropped abs, a wrong factor of the weight fold or a missing k_scale fails here."""
+    rng = np.random.default_rng(16)
+    B, T, H, S, D = 2, 2, 5, 7, 128
+    q8 = rng.integers(0, 256, (B, T, H, D)).astype(np.uint8)
+    k8 = rng.integers(0, 256, (B, S, D)).astype(np.uint8)
+    q8[(q8 & 0x7F) == 0x7F] = 0x21
+    k8[(k8 & 0x7F) == 0x7F] = 0x21
+    qs = rng.uniform(0.01, 1, (B, T, H)).astype(np.float32)
+    ks = rng.uniform(0.01, 1, (B, S)).astype(np.float32)
+    w = rng.standard_normal((B, T, H)).astype(np.float32)
+    w[0, 0, :3] = [-2.0, 1.5, -0.25]                     # mixed signs on purpose
+    q_pos, kv_len = [[3, 6], [6, 2]], [7, 5]
+    got = O.index_score_magnitude(q8, qs, w, k8, ks, q_pos, kv_len, softmax_scale=0.3)
+    want = _brute_scores(q8, qs, w, k8, ks, q_pos, kv_len, 0.3, magnitude=True)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12)
+    # it bounds the score, and equals it where every weight is positive
+    sc = O.index_scores(q8, qs, w, k8, ks, q_pos, kv_len, softmax_scale=0.3)
+    fin = np.isfinite(sc)
+    assert np.all(np.abs(sc[fin]) <= got[fin] * (1 + 1e-12))
+    pos_w = np.abs(w)
+    sc_pos = O.index_scores(q8, qs, pos_w, k8, ks, q_pos, kv_len, softmax_scale=0.3)
+    fin = np.isfinite(sc_pos)
+    assert np.allclose(sc_pos[fin], got[fin], rtol=1e-12, atol=0)
+    # with some weight negative somewhere the magnitude is strictly larger for some entry
+    assert np.any(got[fin] > np.abs(sc[fin]) * (1 + 1e-9))
+
+
+def test_gemm_abs_terms_explicit_loops():
+    """gemm_abs_terms (the error scale of the absorption parity bars) against explicit loops on
+    the two contractions the producers use, with mixed-sign operands."""
+    rng = np.random.default_rng(17)
+    T, H, D, C = 2, 3, 4, 5
+    a = rng.standard_normal((T, H, D))
+    w = rng.standard_normal((H, D, C))
+    got = O.gemm_abs_terms(a, w, "thd,hdc->thc")
+    for t in range(T):
+        for h in range(H):
+            for c in range(C):
+                want = sum(abs(a[t, h, d]) * abs(w[h, d, c]) for d in range(D))
+                assert math.isclose(got[t, h, c], want, rel_tol=1e-13)
+    o = rng.standard_normal((T, H, C))
+    got = O.gemm_abs_terms(o, w, "thc,hdc->thd")
+    for t in range(T):
+        for h in range(H):
+            for d in range(D):
+                want = sum(abs(o[t, h, c]) * abs(w[h, d, c]) for c in range(C))
+                assert math.isclose(got[t, h, d], want, rel_tol=1e-13)
+    # it is never below the magnitude of the contraction itself
+    assert np.all(got >= np.abs(np.einsum("thc,hdc->thd", o, w)) - 1e-12)
+
+
+def test_bf16_decode_every_bit_pattern_against_torch():
+    """bf16_to_f64 (which decodes every bf16 input of the MLA oracle) against torch's bf16 -> fp64
+    conversion over all 65,536 bit patterns, and on closed-form values of the format."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    mine = O.bf16_to_f64(bits)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(mine[ok], ref[ok])
+    assert np.array_equal(np.signbit(mine[ok]), np.signbit(ref[ok]))
+    # closed forms: 1 sign, 8 exponent bits (bias 127), 7 mantissa bits
+    assert O.bf16_to_f64(np.uint16(0x3F80)) == 1.0
+    assert O.bf16_to_f64(np.uint16(0xC000)) == -2.0
+    assert O.bf16_to_f64(np.uint16(0x3FC0)) == 1.5
+    assert O.bf16_to_f64(np.uint16(0x0001)) == 2.0 ** -133          # smallest subnormal
+    assert O.bf16_to_f64(np.uint16(0x7F7F)) == (2 - 2.0 ** -7) * 2.0 ** 127
+    assert np.isinf(O.bf16_to_f64(np.uint16(0x7F80))) and np.isnan(O.bf16_to_f64(np.uint16(0x7FC0)))
 
 
 def test_scores_single_head_is_relu_matmul():
