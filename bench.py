@@ -386,8 +386,9 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end through the public API with host buffers: every step copies its inputs host ->
     # device from pinned memory, runs the calls and reads its results back. Steps rotate over
     # independent slots (device state, pinned buffers, a stream each), so one step's copies overlap
-    # another's kernels, as a serving loop would run them. When the step's inputs fit in the L2,
-    # enough slots rotate that their data exceeds twice the L2: no slot finds its own data resident.
+    # another's kernels, as a serving loop would run them. When the step's inputs fit in the L2, up
+    # to 16 slots rotate (enough that their data exceeds twice the L2 where 16 suffice);
+    # e2e.slots_data_exceeds_2x_l2 records whether it did.
     n_slots = 2
     if st.flush_writes:
         n_slots = min(16, max(2, math.ceil(2 * L2_BYTES / max(1, st.input_bytes)) + 1))

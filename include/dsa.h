@@ -192,8 +192,11 @@ DSA_API int dsa_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t*
  *     library keeps until the process exits.
  *   - A shape whose scratch need (dsa_sparse_mla_workspace_size) exceeds that array is rejected
  *     with DSA_ERR_WORKSPACE before any launch.
- *   - The first call on each device looks up the array's device address (a one-time set-up with
- *     that device current); make that first call before any stream capture.
+ *   - The first call on each device looks up the array's device address with that device current
+ *     (again after the device's context is re-created, e.g. by cudaDeviceReset); make that first
+ *     call before any stream capture.
+ *   - Argument checks and errors are those of dsa_sparse_mla, which this call forwards to with
+ *     the fixed array as its workspace.
  *   - Every call shares the one array and it keeps the last call's contents (nothing in it needs
  *     to start at zero: each call overwrites all the scratch it reads). Calls whose work overlaps
  *     on the GPU (different streams, or different host threads on one device) race on it:

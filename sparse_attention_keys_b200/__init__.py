@@ -236,6 +236,27 @@ def dsa_topk(scores, q_pos, kv_len, k: int, idx=None, flags: int = 0, stream=Non
     return idx
 
 
+def _mla_shapes(q, kv, idx, out, lse, kv_name="kv"):
+    """Shape and device checks of the sparse-MLA arguments (before any pointer reaches the library,
+    so a mismatched buffer raises here instead of being written out of bounds):
+    q [B,T,128,576], kv [...,576], idx [B,T,k], out [B,T,128,512], lse [B,T,128] or None."""
+    if q.dim() != 4 or tuple(q.shape[2:]) != (128, 576):
+        raise ValueError(f"q must be [B, T, 128, 576], got {tuple(q.shape)}")
+    B, T = int(q.shape[0]), int(q.shape[1])
+    if kv.shape[-1] != 576:
+        raise ValueError(f"{kv_name} rows must have 576 features, got {tuple(kv.shape)}")
+    if idx.dim() != 3 or tuple(idx.shape[:2]) != (B, T) or idx.shape[2] < 1:
+        raise ValueError(f"idx must be [B={B}, T={T}, k>=1], got {tuple(idx.shape)}")
+    if out is not None and tuple(out.shape) != (B, T, 128, 512):
+        raise ValueError(f"out must be [{B}, {T}, 128, 512], got {tuple(out.shape)}")
+    if lse is not None and tuple(lse.shape) != (B, T, 128):
+        raise ValueError(f"lse must be [{B}, {T}, 128], got {tuple(lse.shape)}")
+    for t, n in ((kv, kv_name), (idx, "idx"), (out, "out"), (lse, "lse")):
+        if t is not None and t.device != q.device:
+            raise ValueError(f"{n} is on {t.device}, q on {q.device}: all tensors must be on one device")
+    return B, T, int(idx.shape[2])
+
+
 def dsa_sparse_mla_workspace_size(B: int, T: int, k: int) -> int:
     return int(_lib.dsa_sparse_mla_workspace_size(int(B), int(T), int(k)))
 
@@ -246,18 +267,27 @@ def dsa_sparse_mla(q, kv, idx, softmax_scale: float = MLA_SOFTMAX_SCALE, out=Non
     _need(q, torch.bfloat16, "q")
     _need(kv, torch.bfloat16, "kv")
     _need(idx, torch.int32, "idx")
-    B, T = q.shape[0], q.shape[1]
+    if out is not None:
+        _need(out, torch.bfloat16, "out")
+    if lse is not None:
+        _need(lse, torch.float32, "lse")
+    if kv.dim() != 3 or kv.shape[0] != q.shape[0]:
+        raise ValueError(f"kv must be [B, S_max, 576], got {tuple(kv.shape)}")
+    B, T, k = _mla_shapes(q, kv, idx, out, lse)
     S = kv.shape[1]
-    k = idx.shape[-1]
     if out is None:
         out = torch.empty((B, T, 128, 512), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((B, T, 128), dtype=torch.float32, device=q.device)
     ws_bytes = dsa_sparse_mla_workspace_size(B, T, k)
+    if workspace is not None:
+        _need(workspace, workspace.dtype, "workspace")
+        if workspace.device != q.device:
+            raise ValueError("workspace must be on q's device")
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     rc = _lib.dsa_sparse_mla(_ptr(q), _ptr(kv), _ptr(idx), B, T, S, int(k), float(softmax_scale), _ptr(out),
-                             _ptr(lse), _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                             _ptr(lse), _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
                              _stream(stream))
     _check(rc, "dsa_sparse_mla")
     return out, lse
@@ -271,8 +301,13 @@ def dsa_sparse_mla_paged(q, kv_pool, block_table, page_size: int, idx, softmax_s
     _need(kv_pool, torch.bfloat16, "kv_pool")
     _need(block_table, torch.int32, "block_table")
     _need(idx, torch.int32, "idx")
-    B, T = q.shape[0], q.shape[1]
-    k = idx.shape[-1]
+    if out is not None:
+        _need(out, torch.bfloat16, "out")
+    if lse is not None:
+        _need(lse, torch.float32, "lse")
+    B, T, k = _mla_shapes(q, kv_pool, idx, out, lse, kv_name="kv_pool")
+    if block_table.dim() != 2 or block_table.shape[0] != B or block_table.device != q.device:
+        raise ValueError(f"block_table must be [B={B}, max_pages] on q's device, got {tuple(block_table.shape)}")
     max_pages = block_table.shape[1]
     num_pages = kv_pool.shape[0] // int(page_size)
     if out is None:
@@ -284,7 +319,8 @@ def dsa_sparse_mla_paged(q, kv_pool, block_table, page_size: int, idx, softmax_s
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     rc = _lib.dsa_sparse_mla_paged(_ptr(q), _ptr(kv_pool), num_pages, _ptr(block_table), max_pages, int(page_size),
                                    _ptr(idx), B, T, int(k), float(softmax_scale), _ptr(out), _ptr(lse),
-                                   _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
+                                   _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                   _stream(stream))
     _check(rc, "dsa_sparse_mla_paged")
     return out, lse
 
@@ -360,7 +396,9 @@ def dsa_sparse_mla_noalloc(q, kv, idx, out, lse=None, softmax_scale: float = MLA
     _need(out, torch.bfloat16, "out")
     if lse is not None:
         _need(lse, torch.float32, "lse")
-    B, T = q.shape[0], q.shape[1]
+    if kv.dim() != 3 or kv.shape[0] != q.shape[0]:
+        raise ValueError(f"kv must be [B, S_max, 576], got {tuple(kv.shape)}")
+    B, T, _ = _mla_shapes(q, kv, idx, out, lse)
     rc = _lib.dsa_sparse_mla_noalloc(_ptr(q), _ptr(kv), _ptr(idx), B, T, kv.shape[1], int(idx.shape[-1]),
                                      float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream))
     _check(rc, "dsa_sparse_mla_noalloc")

@@ -369,6 +369,16 @@ __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.w
 
 // Host-side launch helpers shared by the entry points (defined in dsa_abi.cu).
 namespace dsa_host {
+// Nonzero id of the CUDA context current on this thread (0 if none or it cannot be queried). A
+// device's primary context gets a new id when it is re-created (e.g. after cudaDeviceReset), and
+// device addresses and kernel attributes set up in the old one no longer hold.
+uint64_t current_context_id();
+constexpr int kMaxSetupDevices = 64;
+// Per-device set-up bookkeeping: `seen` has kMaxSetupDevices entries holding the context id each
+// device was last set up in. needs_setup() is true when the current device's context differs
+// (or cannot be identified); mark_setup() records the current context after the set-up succeeds.
+bool needs_setup(uint64_t* seen, int* dev_out);
+void mark_setup(uint64_t* seen);
 int* status_word();                 // device address of this device's status word (nullptr on error)
 int check_launch();                 // DSA_OK or DSA_ERR_CUDA after a launch
 bool aligned16(const void* p);

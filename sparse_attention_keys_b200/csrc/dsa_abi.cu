@@ -32,8 +32,34 @@ __global__ void selftest_wait_kernel(int* status) {
 
 constexpr int kMaxDevices = 64;
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// The driver's context queries, looked up once through the runtime (the library does not link
+// libcuda directly).
+struct ContextQueries {
+  CtxGetCurrentFn get_current = nullptr;
+  CtxGetIdFn get_id = nullptr;
+};
+const ContextQueries& context_queries() {
+  static ContextQueries q;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult r;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &r) == cudaSuccess &&
+        r == cudaDriverEntryPointSuccess)
+      q.get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &r) == cudaSuccess &&
+        r == cudaDriverEntryPointSuccess)
+      q.get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  return q;
+}
+
 struct DeviceCache {
-  bool init = false;
+  uint64_t ctx = 0;            // id of the context the addresses below belong to (0: not set up)
   bool supported = false;
   int sms = 0;
   int* status = nullptr;
@@ -42,13 +68,16 @@ struct DeviceCache {
 DeviceCache g_dev[kMaxDevices];
 std::mutex g_mu;
 
+// The status word's device address belongs to the context it was looked up in: when the device's
+// context is re-created (for instance after cudaDeviceReset) it is looked up again.
 DeviceCache* device_cache() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   DeviceCache& c = g_dev[dev];
-  if (!c.init) {
+  const uint64_t ctx = dsa_host::current_context_id();
+  if (c.ctx == 0 || c.ctx != ctx) {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!c.init) {
+    if (c.ctx == 0 || c.ctx != ctx) {
       cudaDeviceProp prop;
       if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return nullptr;
       c.supported = prop.major == 10 && prop.minor == 0;
@@ -56,7 +85,7 @@ DeviceCache* device_cache() {
       void* addr = nullptr;
       if (cudaGetSymbolAddress(&addr, g_dsa_status) != cudaSuccess) return nullptr;
       c.status = static_cast<int*>(addr);
-      c.init = true;
+      c.ctx = dsa_host::current_context_id();     // the lookup made the device's context current
     }
   }
   return &c;
@@ -92,6 +121,31 @@ EncodeTiledFn encode_fn() {
 }  // namespace
 
 namespace dsa_host {
+
+uint64_t current_context_id() {
+  const ContextQueries& q = context_queries();
+  if (!q.get_current || !q.get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (q.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (q.get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return (uint64_t)id + 1;
+}
+
+bool needs_setup(uint64_t* seen, int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  if (dev_out) *dev_out = dev;
+  if (dev < 0 || dev >= kMaxDevices) return true;
+  const uint64_t ctx = current_context_id();
+  return ctx == 0 || seen[dev] != ctx;
+}
+
+void mark_setup(uint64_t* seen) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return;
+  seen[dev] = current_context_id();
+}
 
 int* status_word() {
   DeviceCache* c = device_cache();

@@ -316,10 +316,10 @@ static int launch_scores_nq(const uint8_t* q8, const uint8_t* k8, const ScoresPa
   const int tiles_max = (base.S_max + kKeysPerTile - 1) / kKeysPerTile;
   const int64_t units = (int64_t)base.B * p.groups;
   // one wave: as many CTAs as fit on the device at once (key splits share a query group's tiles)
-  static int occupancy[64] = {0};
+  static uint64_t configured[dsa_host::kMaxSetupDevices] = {};
+  static int occupancy[dsa_host::kMaxSetupDevices] = {};
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && occupancy[dev] == 0) {
+  if (dsa_host::needs_setup(configured, &dev) && dev < dsa_host::kMaxSetupDevices) {
     // all of the unified L1 / shared storage as shared memory, so that as many CTAs as the shared
     // memory allows are resident
     if (cudaFuncSetAttribute(index_scores_kernel<NQ, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -331,8 +331,10 @@ static int launch_scores_nq(const uint8_t* q8, const uint8_t* k8, const ScoresPa
                                                       Cfg::kSmemBytes, Cfg::kTmemCols);
     if (per_sm < 1) return DSA_ERR_CUDA;
     occupancy[dev] = per_sm;
+    dsa_host::mark_setup(configured);
   }
-  const int64_t target = (int64_t)(dev < 64 ? occupancy[dev] : 1) * dsa_host::device_sm_count();
+  const int64_t target =
+      (int64_t)(dev < dsa_host::kMaxSetupDevices ? std::max(1, occupancy[dev]) : 1) * dsa_host::device_sm_count();
   int ksplit = (int)std::max<int64_t>(1, target / units);
   ksplit = max(1, min(ksplit, tiles_max));
   p.ksplit = ksplit;
@@ -340,7 +342,7 @@ static int launch_scores_nq(const uint8_t* q8, const uint8_t* k8, const ScoresPa
   p.ksplit = (tiles_max + p.tiles_per_split - 1) / p.tiles_per_split;
   const int64_t grid = units * p.ksplit;
   if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;
-  if (dev >= 64 && cudaFuncSetAttribute(index_scores_kernel<NQ, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (dev >= dsa_host::kMaxSetupDevices && cudaFuncSetAttribute(index_scores_kernel<NQ, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         Cfg::kSmemBytes) != cudaSuccess)
     return DSA_ERR_CUDA;
   return dsa_host::launch(index_scores_kernel<NQ, PAGED>, dim3((unsigned)grid), dim3(threads_for(NQ)),

@@ -690,14 +690,12 @@ int launch_mla_q_absorb(const uint16_t* q_nope, const uint16_t* q_pe, const int3
       !dsa_host::encode_tensor_map_3d(&w_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (void*)w_uk, w_dims, w_str, w_box,
                                       CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
-  static bool configured[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
+  static uint64_t configured[dsa_host::kMaxSetupDevices] = {};
+  if (dsa_host::needs_setup(configured, nullptr)) {
     if (!configure((const void*)q_absorb_kernel, qa::kSmemBytes) ||
         !configure((const void*)q_absorb_few_kernel, fr::kSmemBytes))
       return DSA_ERR_CUDA;
-    configured[dev] = true;
+    dsa_host::mark_setup(configured);
   }
   const int64_t ntiles = (rows + kRows - 1) / kRows;
   AbsorbParams p{};
@@ -737,14 +735,12 @@ int launch_mla_out_absorb(const uint16_t* o, const uint16_t* w_uv, int64_t w_hea
       !dsa_host::encode_tensor_map_3d(&w_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (void*)w_uv, w_dims, w_str, w_box,
                                       CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
-  static bool configured[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
+  static uint64_t configured[dsa_host::kMaxSetupDevices] = {};
+  if (dsa_host::needs_setup(configured, nullptr)) {
     if (!configure((const void*)out_absorb_kernel, oa::kSmemBytes) ||
         !configure((const void*)out_absorb_few_kernel, fr::kSmemBytes))
       return DSA_ERR_CUDA;
-    configured[dev] = true;
+    dsa_host::mark_setup(configured);
   }
   const int64_t ntiles = (rows + kRows - 1) / kRows;
   AbsorbParams p{};

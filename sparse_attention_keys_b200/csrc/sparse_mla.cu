@@ -629,14 +629,12 @@ static int launch_mla(const uint16_t* q, MlaParams p, cudaStream_t stream, void*
     p.part_o = static_cast<float*>(workspace);
     p.part_ml = p.part_o + (size_t)BT * s.nsplit * kHeads * kDv;
   }
-  static bool configured[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
+  static uint64_t configured[dsa_host::kMaxSetupDevices] = {};
+  if (dsa_host::needs_setup(configured, nullptr)) {
     if (cudaFuncSetAttribute(sparse_mla_kernel<PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
         cudaSuccess)
       return DSA_ERR_CUDA;
-    configured[dev] = true;
+    dsa_host::mark_setup(configured);
   }
   const int64_t grid = BT * s.nsplit * 2;          // two CTAs (output-feature halves) per (query, split)
   if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;

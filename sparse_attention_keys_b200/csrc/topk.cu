@@ -391,12 +391,21 @@ int launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int
   // candidate positions on the first radix digit: a quarter of the longest row (at least 256)
   const int cand_cap = std::max(256, ((max_row + 3) & ~3) / 4 / 4 * 4);
   const size_t smem = (size_t)(kHistBins + ((max_row + 3) & ~3) + cand_cap) * sizeof(uint32_t) + (size_t)sort_n * 8;
-  static int configured_smem = 0;
-  if ((int)smem > configured_smem) {
+  // the largest dynamic shared memory set so far, per device, in the context it was set in
+  static uint64_t configured[dsa_host::kMaxSetupDevices] = {};
+  static int configured_smem[dsa_host::kMaxSetupDevices] = {};
+  int dev = 0;
+  const bool fresh = dsa_host::needs_setup(configured, &dev);
+  const bool tracked = dev >= 0 && dev < dsa_host::kMaxSetupDevices;
+  if (fresh || !tracked || (int)smem > configured_smem[dev]) {
     if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
       return DSA_ERR_CUDA;
-    configured_smem = (int)smem;
+    if (tracked) {
+      if (fresh) configured_smem[dev] = 0;
+      configured_smem[dev] = std::max(configured_smem[dev], (int)smem);
+      dsa_host::mark_setup(configured);
+    }
   }
   return dsa_host::launch(topk_kernel, dim3((unsigned)rows), dim3(kTopkThreads), smem, stream, scores, ld, q_pos,
                           kv_len, T, k, max_row, cand_cap, flags, sort_n, idx, status);

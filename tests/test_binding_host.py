@@ -46,3 +46,31 @@ def test_noncontiguous_inputs_are_rejected(dsa):
 def test_status_strings_cover_every_site(dsa):
     assert all(isinstance(v, str) and v for v in dsa.SITE_NAMES.values())
     assert {0x41, 0x42, 0x43, 0x44, 0x45} <= set(dsa.SITE_NAMES)
+
+
+def test_sparse_mla_shape_checks(dsa):
+    """Mismatched sparse-MLA buffers raise before any pointer reaches the library (checked on host
+    tensors: the shape rules do not depend on the device)."""
+    bf = torch.bfloat16
+    q = torch.zeros(2, 3, 128, 576, dtype=bf)
+    kv = torch.zeros(2, 64, 576, dtype=bf)
+    idx = torch.zeros(2, 3, 16, dtype=torch.int32)
+    out = torch.zeros(2, 3, 128, 512, dtype=bf)
+    lse = torch.zeros(2, 3, 128)
+    assert dsa._mla_shapes(q, kv, idx, out, lse) == (2, 3, 16)
+    assert dsa._mla_shapes(q, kv, idx, None, None) == (2, 3, 16)
+    bad = [
+        (torch.zeros(2, 3, 64, 576, dtype=bf), kv, idx, out, lse),        # q heads
+        (torch.zeros(2, 3, 128, 512, dtype=bf), kv, idx, out, lse),       # q width
+        (q, torch.zeros(2, 64, 512, dtype=bf), idx, out, lse),            # kv width
+        (q, kv, torch.zeros(2, 2, 16, dtype=torch.int32), out, lse),      # idx queries
+        (q, kv, torch.zeros(3, 3, 16, dtype=torch.int32), out, lse),      # idx batch
+        (q, kv, idx, torch.zeros(2, 3, 128, 256, dtype=bf), lse),         # out too small
+        (q, kv, idx, torch.zeros(2, 2, 128, 512, dtype=bf), lse),         # out queries
+        (q, kv, idx, out, torch.zeros(2, 3, 64)),                         # lse heads
+    ]
+    for args in bad:
+        with pytest.raises(ValueError):
+            dsa._mla_shapes(*args)
+    with pytest.raises(ValueError):                                         # not on one device
+        dsa._mla_shapes(q, kv.to("meta"), idx, out, lse)

@@ -53,6 +53,28 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
         assert np.all(np.abs(nl - rl) <= P.LSE_ATOL)
 
 
+def test_noalloc_matches_on_a_multi_query_shape():
+    """Several queries per sequence (T = 4): the split-KV partials are laid out per (query, split),
+    so this exercises a scratch layout the one-query decode shapes do not."""
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    B, T, S, k = 1, 4, 4096, 2048
+    need = dsa.dsa_sparse_mla_workspace_size(B, T, k)
+    assert 0 < need <= dsa.dsa_sparse_mla_noalloc_scratch_bytes()
+    rng = np.random.default_rng(78)
+    q = P.bf16_dev(DI.bf16_bits_from_f32(rng.standard_normal((B, T, 128, 576), np.float32)))
+    kv = P.bf16_dev(DI.bf16_bits_from_f32(rng.standard_normal((B, S, 576), np.float32)))
+    idx = np.full((B, T, k), -1, np.int32)
+    for t, n in enumerate((S, 3000, 2048, 700)):              # full, partial and short rows
+        m = min(n, k)
+        idx[0, t, :m] = np.sort(rng.choice(n, m, replace=False))
+    for call in range(2):
+        ro, rl, no, nl = _ref_and_noalloc(q, kv, P.to_dev(idx))
+        assert np.all(np.abs(no - ro) <= P.MLA_ATOL), np.max(np.abs(no - ro))
+        assert np.all(np.abs(nl - rl) <= P.LSE_ATOL)
+        idx[0, 1, 1500:] = -1                                  # the second call changes a row
+
+
 def test_noalloc_rejects_shape_beyond_its_scratch():
     if not torch.cuda.is_available():
         pytest.skip("no GPU")
