@@ -1,6 +1,7 @@
 """Benchmark of the DSA hot path: one step = one pass of the whole path over one batch.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode_b8] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode_b64] [--extra prefill_16384]
+                    [--impl ours|reference]
 
 A decode step runs, through the C ABI: dsa_index_keys on the new keys (written into the
 resident FP8 K-cache) and on the queries, dsa_index_scores, dsa_topk and dsa_sparse_mla. A
@@ -17,8 +18,10 @@ The end-to-end figure (`e2e`) goes through the public API with host buffers: eac
 inputs host -> device from pinned memory and reads its results back, and the steps rotate over
 independent slots on their own streams so that copies overlap kernels. Each slot's copies and
 calls are captured once as a CUDA graph and replayed; `e2e.eager` issues them from Python every step.
-Under torchrun each rank runs its own replica of the workload (independent sequences, no
-collective on the data path): weak scaling.
+With --gpus N each of N ranks (one process per GPU; started here under torch.distributed.run when
+the script is not already a rank) runs its own replica of the workload (independent sequences, no
+collective on the data path): weak scaling. The default line also times the 16384-token prefill
+(--extra) on the same GPU, for the FP8 index scores and the long-row top-k.
 
 The reference arm (--impl reference) times the CPU oracle on the host cores on a bounded sample
 of the same workload.
@@ -64,13 +67,20 @@ def work_units(inp):
         "pairs": pairs,
         "queries": BT,
         "selected": sel,
-        # per kernel: bytes read + written that the operation cannot avoid
+        # per kernel, the algorithmic unit of the measurement rules times the units of one launch:
+        # index scores 132 B of K-cache per (query, key) pair; top-k 4 B read per visible score and
+        # 4 B written per index; sparse MLA 1152 B gathered per (query, selected key)
         "index_keys_bytes": (BT * 64 + new_keys) * (512 + 132) + (BT + new_keys) * 4,
-        "index_scores_bytes": pairs * (132 + 4) + BT * 64 * (128 + 4 + 4),
+        "index_scores_bytes": pairs * 132,
         "index_scores_flops": pairs * 64 * 128 * 2,
         "topk_bytes": pairs * 4 + BT * k * 4,
-        "sparse_mla_bytes": sel * 1152 + BT * 128 * (576 + 512) * 2 + BT * k * 4,
+        "sparse_mla_bytes": sel * 1152,
         "sparse_mla_flops": sel * 128 * (576 + 512) * 2,
+        # further bytes each launch moves beyond those units (reported beside, not in `achieved`):
+        # the scores written and the queries/weights read by the index scores; the queries, outputs
+        # and indices of the sparse MLA
+        "index_scores_other_bytes": pairs * 4 + BT * 64 * (128 + 4 + 4),
+        "sparse_mla_other_bytes": BT * 128 * (576 + 512) * 2 + BT * k * 4,
     }
 
 
@@ -172,6 +182,7 @@ class Step:
         import torch
         import sparse_attention_keys_b200 as dsa
         self.dsa, self.torch, self.inp = dsa, torch, inp
+        self.dev_index = device.index if device.index is not None else torch.cuda.current_device()
         wl = inp.workload
         B, T = inp.q_pos.shape
         S = wl.s_max
@@ -308,32 +319,14 @@ def check_status(dsa, stage):
                            f"{dsa.dsa_get_error_detail()}")
 
 
-def run_ours(args, rank, world, local_rank):
+def time_device(st, args, barrier, sample_clocks=True):
+    """Device time of `args.steps` steps of `st` with inputs resident in HBM. The step is captured
+    as a CUDA graph and replayed, so no host launch gaps are timed. A second graph of the same
+    step holds an event pair around each ABI call and is replayed after every timed step for the
+    per-kernel durations: event nodes lengthen a replay by a few microseconds each, so they stay
+    out of the step time. Returns (seconds for all steps, {call: seconds per step}, clocks)."""
     import torch
-    import torch.distributed as tdist
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    inp = DI.make_inputs(args.workload, seed=rank)
-    units = work_units(inp)
-    st = Step(inp, dev)
-    import sparse_attention_keys_b200 as dsa
 
-    for _ in range(args.warmup):
-        st.l2_flush()
-        st.run()
-    torch.cuda.synchronize()
-    check_status(dsa, "warm-up")
-
-    def barrier():
-        if world > 1:
-            tdist.barrier()
-        torch.cuda.synchronize()
-
-    # ---- device-timed region (inputs resident in HBM). The step is captured as a CUDA graph and
-    # replayed, so no host launch gaps are timed. A second graph of the same step holds an event
-    # pair around each ABI call and is replayed after every timed step for the per-kernel
-    # durations: event nodes lengthen a replay by a few microseconds each, so they stay out of
-    # the step time.
     def capture(fn):
         g = torch.cuda.CUDAGraph()
         cap_stream = torch.cuda.Stream()
@@ -351,10 +344,13 @@ def run_ours(args, rank, world, local_rank):
     graph = capture(st.run)
     graph_k = capture(lambda: st.run(kev))
     steps = []
-    with ClockSampler(local_rank) as clk:
+    clk = ClockSampler(st.dev_index) if sample_clocks else None
+    if clk is not None:
+        clk.__enter__()
+    try:
         # the sampler polls every 20 ms: keep the GPU under the same load for ~0.5 s before the
         # timed steps so that the samples taken while they run see steady-state clocks
-        t_end = time.perf_counter() + 0.5
+        t_end = time.perf_counter() + (0.5 if sample_clocks else 0.05)
         while time.perf_counter() < t_end:
             st.l2_flush()
             graph.replay()
@@ -377,10 +373,66 @@ def run_ours(args, rank, world, local_rank):
             for n, v in kev.items():
                 per_kernel_sum[n] += sum(a.elapsed_time(b) for a, b in v)
         barrier()
-    clocks = clk.summary()
+    finally:
+        if clk is not None:
+            clk.__exit__(None, None, None)
+    clocks = clk.summary() if clk is not None else None
     t_dev = sum(s.elapsed_time(e) for s, e in steps) / 1e3          # seconds
     per_kernel = {n: v / args.steps / 1e3 for n, v in per_kernel_sum.items()}
     del graph, graph_k
+    return t_dev, per_kernel, clocks
+
+
+def extra_workload(name, args, dev, peaks):
+    """A second workload timed in the same run (device time only, one GPU): the step's throughput
+    and the roofline of each of its kernels. The default decode line adds the 16384-token prefill
+    here, whose index scores are the FP8 tensor-core half of the metric."""
+    import torch
+    import sparse_attention_keys_b200 as dsa
+    inp = DI.make_inputs(name, seed=0)
+    units = work_units(inp)
+    st = Step(inp, dev)
+    for _ in range(args.warmup):
+        st.l2_flush()
+        st.run()
+    torch.cuda.synchronize()
+    check_status(dsa, f"{name} warm-up")
+    t_dev, per_kernel, _ = time_device(st, args, torch.cuda.synchronize, sample_clocks=False)
+    check_status(dsa, f"{name} graph replays")
+    out = {"workload": name, "desc": inp.workload.note, "steps": args.steps,
+           "ms_per_step": t_dev / args.steps * 1e3, "value": units["pairs"] * args.steps / t_dev, "unit": UNIT,
+           "pairs_per_step": units["pairs"], "l2": st.l2_policy(),
+           "kernel_ms": {n: v * 1e3 for n, v in per_kernel.items()},
+           "roofline": {n: roofline_entry(n, v, units, peaks, args, workload=name) for n, v in per_kernel.items()
+                        if f"{n}_bytes" in units}}
+    del st
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as tdist
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    inp = DI.make_inputs(args.workload, seed=rank)
+    units = work_units(inp)
+    st = Step(inp, dev)
+    import sparse_attention_keys_b200 as dsa
+
+    for _ in range(args.warmup):
+        st.l2_flush()
+        st.run()
+    torch.cuda.synchronize()
+    check_status(dsa, "warm-up")
+
+    def barrier():
+        if world > 1:
+            tdist.barrier()
+        torch.cuda.synchronize()
+
+    # ---- device-timed region (inputs resident in HBM)
+    t_dev, per_kernel, clocks = time_device(st, args, barrier, sample_clocks=True)
     check_status(dsa, "graph replays")
 
     # ---- end to end through the public API with host buffers: every step copies its inputs host ->
@@ -504,6 +556,12 @@ def run_ours(args, rank, world, local_rank):
         line["mla_producers"] = producer_rooflines(producers, peaks)
     if paged is not None:
         line["paged_caches"] = paged_rooflines(paged, units, peaks, args)
+    extras = [w for w in (args.extra or "").split(",") if w and w != args.workload]
+    if world == 1 and extras:
+        del st, slots
+        torch.cuda.empty_cache()
+        for name in extras:
+            line[name] = extra_workload(name, args, dev, peaks)
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_budget)
     return line
@@ -641,12 +699,13 @@ def producer_rooflines(t, peaks):
     return res
 
 
-def roofline_entry(name, seconds, units, peaks, args):
+def roofline_entry(name, seconds, units, peaks, args, workload=None):
     """Roofline of one kernel. Prefill shares one cache among all queries, so its index scores
     (e4m3) and sparse MLA (bf16) are bound by the tensor cores; decode kernels stream their own
     cache rows and are bound by HBM."""
-    traffic = load_traffic(name, args.workload)
-    prefill = not DI.WORKLOADS[args.workload].decode
+    workload = workload or args.workload
+    traffic = load_traffic(name, workload)
+    prefill = not DI.WORKLOADS[workload].decode
     if prefill and name in ("index_scores", "sparse_mla"):
         flops = units[f"{name}_flops"]
         if name == "index_scores":
@@ -657,12 +716,16 @@ def roofline_entry(name, seconds, units, peaks, args):
             src = f"{peaks['source']} bf16_tflops"
         ach = flops / seconds / 1e12
         return {"kernel": name, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": ach / peak, "traffic": traffic, "peak_source": src, "algorithmic_flops": flops}
+                "frac": ach / peak, "traffic": traffic, "peak_source": src, "algorithmic_flops": flops,
+                "kernel_us": seconds * 1e6}
     nbytes = units[f"{name}_bytes"]
     ach = nbytes / seconds / 1e9
-    return {"kernel": name, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": ach / peaks["hbm_gbs"], "traffic": traffic, "peak_source": f"{peaks['source']} hbm_gbs",
-            "algorithmic_bytes": nbytes}
+    entry = {"kernel": name, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+             "frac": ach / peaks["hbm_gbs"], "traffic": traffic, "peak_source": f"{peaks['source']} hbm_gbs",
+             "algorithmic_bytes": nbytes, "kernel_us": seconds * 1e6}
+    if f"{name}_other_bytes" in units:
+        entry["other_bytes"] = units[f"{name}_other_bytes"]
+    return entry
 
 
 def load_traffic(kernel, workload):
@@ -827,12 +890,24 @@ def run_reference(args, rank, world):
     }
 
 
+def launch_command(n_gpus, argv):
+    """The command that runs this script as `n_gpus` ranks on this node (rendezvous on 127.0.0.1)."""
+    import socket
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        port = sock.getsockname()[1]
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n_gpus}",
+            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="decode_b8", choices=sorted(DI.WORKLOADS))
+    ap.add_argument("--workload", default="decode_b64", choices=sorted(DI.WORKLOADS))
+    ap.add_argument("--extra", default="prefill_16384",
+                    help="comma-separated workloads also timed (device time, one GPU) in the same run; '' for none")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-producers", action="store_true", help="skip timing the MLA producer calls")
@@ -840,9 +915,17 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # one process per GPU: start the ranks here (torch.distributed.run on this node)
+        os.execv(sys.executable, launch_command(args.gpus, sys.argv[1:]))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}: launch one rank per GPU", file=sys.stderr)
+        sys.exit(2)
     if args.impl == "reference":
         line = run_reference(args, rank, world)
     else:

@@ -9,8 +9,9 @@ Tolerances (written here once, used by every test):
 * index scores: |I_gpu - I_ref| <= 1e-3 * max(|I_ref|, M) with M = k_scale * sum_j |w'_j| ReLU(dot_j)
   (the relative 1e-3 bar, measured against the magnitude of the terms that were summed, since
   mixed-sign head weights can cancel a score to near 0).
-* top-k: bit-exact on identical fp32 inputs; against oracle scores only slots whose score is
-  within the score tolerance of the k-th largest may differ.
+* top-k: bit-exact on identical fp32 inputs; against oracle scores (on identical quantised inputs)
+  only positions whose score lies within twice the score tolerance of the k-th largest may differ
+  (the derivation is in check_topk_near_ties).
 * sparse MLA: 2e-2 absolute on the bf16 outputs; lse 1e-3 absolute.
 """
 import numpy as np
@@ -79,18 +80,25 @@ def check_scores(gpu, ref, mag, nvalid):
         assert np.all(err <= lim), f"row {t}: worst {np.max(err / lim):.3g} x tolerance"
 
 
-def check_topk_near_ties(idx_gpu, idx_ref, scores_ref, mag_ref, k, band=1.0):
-    """Selected sets may differ only where the scores are within `band` x the score tolerance of
-    the k-th value, and in at most 1% of the slots."""
+def check_topk_near_ties(idx_gpu, idx_ref, scores_ref, mag_ref, k):
+    """Selected sets may differ only at near-ties.
+
+    Both selections come from scores that agree within the score tolerance tol_x =
+    SCORE_RTOL * max(|I_x|, M_x) (check_scores). If the GPU keeps x and drops y where the oracle
+    keeps y and drops x, then I_ref(x) + tol_x >= I_gpu(x) >= I_gpu(y) >= I_ref(y) - tol_y, and the
+    oracle's k-th score theta lies between I_ref(x) and I_ref(y). The two sets have equal sizes,
+    so every element of their symmetric difference D pairs with one on the other side, and
+    |I_ref(x) - theta| <= 2 * max_{j in D} tol_j for every x in D. That bound, and nothing looser,
+    is what is checked: the sets are equal except at scores that tie within the tolerance."""
     for r in range(idx_ref.shape[0]):
         a = set(int(i) for i in idx_gpu[r] if i >= 0)
         b = set(int(i) for i in idx_ref[r] if i >= 0)
-        assert len(a) == len(b)
+        assert len(a) == len(b), (r, len(a), len(b))
         if a == b:
             continue
-        assert len(a ^ b) <= max(2, len(b) // 50), (r, len(a ^ b))
-        row = scores_ref[r]
-        kth = min(row[i] for i in b)
-        for i in a ^ b:
-            tol = band * SCORE_RTOL * (max(abs(row[i]), mag_ref[r][i]) + abs(kth))
-            assert abs(row[i] - kth) <= tol, (r, i, row[i], kth)
+        row, mag = scores_ref[r], mag_ref[r]
+        theta = min(row[i] for i in b)
+        d = a ^ b
+        tol_d = max(SCORE_RTOL * max(abs(row[i]), mag[i]) for i in d)
+        for i in d:
+            assert abs(row[i] - theta) <= 2.0 * tol_d, (r, i, row[i], theta, tol_d)

@@ -12,9 +12,15 @@ def test_decode_pairs_are_the_visible_keys():
     assert u["pairs"] == 1024 and u["queries"] == 1 and u["selected"] == 256
     assert u["index_scores_flops"] == 1024 * 64 * 128 * 2
     assert u["topk_bytes"] == 1024 * 4 + 256 * 4
-    # selected latent rows + the query's q and output rows + its indices
-    assert u["sparse_mla_bytes"] == 256 * 1152 + 128 * (576 + 512) * 2 + 256 * 4
+    # the measurement unit: 1152 B gathered per (query, selected key); the query's q and output
+    # rows and its indices are reported beside it
+    assert u["sparse_mla_bytes"] == 256 * 1152
+    assert u["sparse_mla_other_bytes"] == 128 * (576 + 512) * 2 + 256 * 4
     assert u["sparse_mla_flops"] == 256 * 128 * (576 + 512) * 2
+    # index scores: 132 B of K-cache per (query, key) pair; the scores written and the query
+    # codes, scales and weights read are beside it
+    assert u["index_scores_bytes"] == 1024 * 132
+    assert u["index_scores_other_bytes"] == 1024 * 4 + 64 * (128 + 4 + 4)
 
 
 def test_decode_b8_pairs_sum_the_context_lengths():
@@ -50,3 +56,12 @@ def test_prefill_oracle_unit_counts_its_causal_pairs():
     assert bench.oracle_prefill_rows(inp, 16, table, caches) == sum(t + 1 for t in range(16, 16 + bench.PREFILL_CHUNK))
     units = bench._oracle_units(inp)
     assert units[0] == ("rows", 0) and units[-1] == ("rows", 64 - bench.PREFILL_CHUNK)
+
+
+def test_decode_b64_units_follow_the_measurement_rules():
+    inp = DI.make_inputs(DI.Workload("d", batch=64, queries=1, s_max=64, topk=16, decode=True,
+                                     kv_len_range=(64, 64), with_mla=False))
+    u = bench.work_units(inp)
+    assert u["pairs"] == 64 * 64 and u["selected"] == 64 * 16
+    assert u["sparse_mla_bytes"] == 64 * 16 * 1152
+    assert u["index_scores_bytes"] == 64 * 64 * 132

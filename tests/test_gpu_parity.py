@@ -81,6 +81,31 @@ def test_index_keys_cache_write(table_dev):
     assert np.all(c[untouched] == 0xAB) and np.all(s[untouched] == -1.0)
 
 
+def test_index_keys_full_prefill_16384_launch(table_dev):
+    """The benchmark's 16384-token prefill launches: all 16384 keys (1% of them scaled x8 before
+    RoPE and quantisation) written into the K-cache, and all 16384 x 64 query blocks. Every key row
+    is checked; query blocks on sampled rows: the first, the hot-key positions, the middle and the
+    last positions up to 16383."""
+    inp = DI.make_inputs("prefill_16384")
+    S = inp.idx_k.shape[1]
+    cache = torch.zeros((1, S, 128), dtype=torch.uint8, device="cuda")
+    cscale = torch.zeros((1, S), dtype=torch.float32, device="cuda")
+    dsa.dsa_index_keys(P.to_dev(inp.idx_k.reshape(S, 128)), P.to_dev(np.arange(S, dtype=np.int32)), table_dev,
+                       out_fp8=cache, out_scale=cscale, dst_row=P.to_dev(np.arange(S, dtype=np.int64)))
+    q8, qs = dsa.dsa_index_keys(P.to_dev(inp.idx_q.reshape(S, 64, 128)), P.to_dev(inp.q_pos.reshape(-1)), table_dev)
+    assert _status() == 0
+    hot = inp.hot_rows
+    assert hot is not None and len(hot) == 164
+    g_cache, g_scale = cache.cpu().numpy()[0], cscale.cpu().numpy()[0]
+    P.check_codes(g_cache, g_scale, inp.idx_k[0], np.arange(S), TABLE)
+    # the hot rows' scales are ~8x the others' (amax grows with the row)
+    cold = np.setdiff1d(np.arange(S), hot)
+    assert np.median(g_scale[hot]) > 6 * np.median(g_scale[cold])
+    rows = sorted(set([0, 1, 127, 128, 8191, 16381, 16382, 16383] + [int(r) for r in hot[:4]]))
+    g_q8, g_qs = q8.cpu().numpy(), qs.cpu().numpy()
+    P.check_codes(g_q8[rows], g_qs[rows], inp.idx_q[0, rows], np.array(rows)[:, None], TABLE)
+
+
 def test_index_keys_position_out_of_range_sets_status(table_dev):
     x = torch.zeros((4, 128), dtype=torch.float32, device="cuda")
     pos = torch.tensor([0, 1, 20000, 3], dtype=torch.int32, device="cuda")
@@ -258,24 +283,33 @@ def test_topk_longest_row_and_overlong_row(table_dev):
     assert _status() == 5
 
 
-@pytest.mark.parametrize("name", ["prefill_4096", "decode_b64"])
+@pytest.mark.parametrize("name", ["prefill_4096", "prefill_16384", "decode_b64"])
 def test_topk_full_size_on_oracle_scores(table_dev, name):
-    """Full launch on fp32 scores made by the oracle; sampled rows checked bit-exact."""
+    """Full launch on fp32 scores made by the oracle; sampled rows checked bit-exact. The 16384-token
+    prefill rows are up to 16384 wide and include the rows of the x8 hot keys."""
     inp = DI.make_inputs(name, with_mla=False)
     B, T = inp.idx_q.shape[:2]
-    rows = [(0, t) for t in (0, 5, 2046, 2047, 2048, 3000, T - 1) if t < T] if name.startswith("prefill") \
-        else [(b, 0) for b in (0, 31, 63)]
+    if name.startswith("prefill"):
+        cand = [0, 5, 2046, 2047, 2048, 3000, T // 2 + 1, T - 2, T - 1]
+        if inp.hot_rows is not None:
+            cand += [int(r) for r in inp.hot_rows[-2:]]
+        rows = [(0, t) for t in sorted(set(cand)) if t < T]
+    else:
+        rows = [(b, 0) for b in (0, 31, 63)]
     q8, qs, k8, ks = _quantised(inp, q_rows=rows, k_seqs=sorted(set(b for b, _ in rows)))
     ld = inp.idx_k.shape[1]
-    sc = np.random.default_rng(1).standard_normal((B, T, ld)).astype(np.float32)   # background rows
+    gen = torch.Generator(device="cuda").manual_seed(1)
+    sc_dev = torch.randn((B, T, ld), generator=gen, device="cuda", dtype=torch.float32)   # background rows
+    sc = {}
     for b, t in rows:
         sl = (slice(b, b + 1), slice(t, t + 1))
         r = O.index_scores(q8[sl], qs[sl], inp.idx_w[sl], k8[b:b + 1], ks[b:b + 1], inp.q_pos[sl], inp.kv_len[b:b + 1])
         sc[b, t] = r[0, 0].astype(np.float32)
-    got = _gpu_topk(sc, inp.q_pos, inp.kv_len, inp.workload.topk)
+        sc_dev[b, t] = torch.from_numpy(sc[b, t]).cuda()
+    got = dsa.dsa_topk(sc_dev, P.to_dev(inp.q_pos), P.to_dev(inp.kv_len), inp.workload.topk).cpu().numpy()
     assert _status() == 0
     for b, t in rows:
-        want = O.topk_indices(sc[b:b + 1, t:t + 1].astype(np.float64), inp.q_pos[b:b + 1, t:t + 1],
+        want = O.topk_indices(sc[b, t][None, None].astype(np.float64), inp.q_pos[b:b + 1, t:t + 1],
                               inp.kv_len[b:b + 1], inp.workload.topk)
         assert np.array_equal(got[b, t], want[0, 0]), (b, t)
 
@@ -358,45 +392,80 @@ def test_sparse_mla_full_size_sampled(table_dev, name):
 
 
 # ----------------------------------------------------------------------------------- whole path
-@pytest.mark.parametrize("name", ["tiny_decode", "decode_b8"])
+E2E_ROWS = {
+    "prefill_4096": [(0, t) for t in (0, 1, 127, 2047, 2048, 2049, 3001, 4095)],
+    "decode_b64": [(b, 0) for b in (0, 17, 40, 63)],
+}
+
+
+@pytest.mark.parametrize("name", ["tiny_decode", "decode_b8", "prefill_4096", "decode_b64"])
 def test_pipeline_end_to_end(table_dev, name):
-    """index_keys (cache + queries) -> scores -> top-k -> sparse MLA, all through the C ABI, against
-    the oracle chain. Selections may differ only at near-ties; attention is checked on the GPU's
-    own selection through the oracle."""
+    """index_keys (cache + queries) -> scores -> top-k -> sparse MLA, all through the C ABI in the
+    order and launch configuration the benchmark's step uses, at the workload's full size.
+
+    Checked link by link against the oracle, on every row of the small workloads and on sampled
+    rows of the large ones: the GPU's codes and scales against the oracle's quantiser; the GPU's
+    scores against the oracle's scores on those same codes (identical quantised inputs); the
+    selection against the GPU's own score buffer (bit-exact, both output orders) and against the
+    oracle's selection on the oracle's scores (equal except at near-ties); the attention output of
+    the GPU's selection against the oracle's."""
     inp = DI.make_inputs(name)
     B, S = inp.idx_k.shape[:2]
     T = inp.q_pos.shape[1]
     k = inp.workload.topk
+    rows = E2E_ROWS.get(name, [(b, t) for b in range(B) for t in range(T)])
+    seqs = sorted(set(b for b, _ in rows))
     cache = torch.zeros((B, S, 128), dtype=torch.uint8, device="cuda")
     cscale = torch.zeros((B, S), dtype=torch.float32, device="cuda")
     kx = P.to_dev(inp.idx_k.reshape(B * S, 128))
     kpos = P.to_dev(np.tile(np.arange(S, dtype=np.int32), B))
     dst = P.to_dev(np.arange(B * S, dtype=np.int64))
     dsa.dsa_index_keys(kx, kpos, table_dev, out_fp8=cache, out_scale=cscale, dst_row=dst)
+    del kx, kpos, dst
     q8, qs = dsa.dsa_index_keys(P.to_dev(inp.idx_q.reshape(B * T, 64, 128)), P.to_dev(inp.q_pos.reshape(-1)),
                                 table_dev)
     q8 = q8.view(B, T, 64, 128)
     qs = qs.view(B, T, 64)
-    sc = dsa.dsa_index_scores(q8, qs, P.to_dev(inp.idx_w), cache, cscale, P.to_dev(inp.q_pos), P.to_dev(inp.kv_len))
+    ld = (S + 3) // 4 * 4
+    sc = dsa.dsa_index_scores(q8, qs, P.to_dev(inp.idx_w), cache, cscale, P.to_dev(inp.q_pos), P.to_dev(inp.kv_len),
+                              ld=ld)
     idx = dsa.dsa_topk(sc, P.to_dev(inp.q_pos), P.to_dev(inp.kv_len), k)
     out, lse = dsa.dsa_sparse_mla(P.bf16_dev(inp.mla_q), P.bf16_dev(inp.mla_kv), idx)
+    gs = dsa.dsa_topk(sc, P.to_dev(inp.q_pos), P.to_dev(inp.kv_len), k, flags=dsa.DSA_SORTED)
     assert _status() == 0
-    # oracle chain
-    oq8, oqs, ok8, oks = _quantised(inp)
-    ref = O.index_scores(oq8, oqs, inp.idx_w, ok8, oks, inp.q_pos, inp.kv_len)
-    mag = O.index_score_magnitude(oq8, oqs, inp.idx_w, ok8, oks, inp.q_pos, inp.kv_len)
-    ref_idx = O.topk_indices(ref, inp.q_pos, inp.kv_len, k)
-    gidx = idx.cpu().numpy()
-    # the GPU's own codes may sit one step from the oracle's at e4m3 rounding boundaries, which
-    # moves a score by a small fraction of its term magnitude: swaps are allowed only there
-    P.check_topk_near_ties(gidx.reshape(B * T, k), ref_idx.reshape(B * T, k), ref.reshape(B * T, -1),
-                           mag.reshape(B * T, -1), k, band=20.0)
-    # on the GPU's own score buffer the selection is bit-exact, in both output orders
-    own = sc.cpu().numpy().astype(np.float64)
-    assert np.array_equal(gidx, O.topk_indices(own, inp.q_pos, inp.kv_len, k))
-    gs = dsa.dsa_topk(sc, P.to_dev(inp.q_pos), P.to_dev(inp.kv_len), k, flags=dsa.DSA_SORTED).cpu().numpy()
-    assert np.array_equal(gs, O.topk_indices(own, inp.q_pos, inp.kv_len, k, sorted_by_score=True))
-    _check_mla(out.float().cpu().numpy(), lse.cpu().numpy(), inp.mla_q, inp.mla_kv, gidx)
+    # 1. the GPU's codes against the oracle's quantiser
+    g_cache = cache.cpu().numpy()
+    g_cscale = cscale.cpu().numpy()
+    for b in seqs:
+        n = int(inp.kv_len[b])
+        P.check_codes(g_cache[b, :n], g_cscale[b, :n], inp.idx_k[b, :n], np.arange(n), TABLE)
+    g_q8 = np.stack([q8[b, t].cpu().numpy() for b, t in rows])
+    g_qs = np.stack([qs[b, t].cpu().numpy() for b, t in rows])
+    P.check_codes(g_q8, g_qs, np.stack([inp.idx_q[b, t] for b, t in rows]),
+                  np.array([inp.q_pos[b, t] for b, t in rows])[:, None], TABLE)
+    g_idx = idx.cpu().numpy()
+    g_sorted = gs.cpu().numpy()
+    g_out = out.float().cpu().numpy()
+    g_lse = lse.cpu().numpy()
+    for j, (b, t) in enumerate(rows):
+        qsl = (slice(b, b + 1), slice(t, t + 1))
+        args = (g_q8[j][None, None], g_qs[j][None, None], inp.idx_w[qsl], g_cache[b:b + 1], g_cscale[b:b + 1],
+                inp.q_pos[qsl], inp.kv_len[b:b + 1])
+        # 2. scores on identical quantised inputs
+        ref = O.index_scores(*args)
+        mag = O.index_score_magnitude(*args)
+        nv = O.valid_len(inp.q_pos[qsl], inp.kv_len[b:b + 1])
+        own = sc[b, t].cpu().numpy()[None]
+        P.check_scores(own, ref[0], mag[0], nv[0])
+        # 3. the selection: bit-exact on the GPU's own scores, near-ties only against the oracle's
+        own64 = own[None].astype(np.float64)
+        assert np.array_equal(g_idx[b, t], O.topk_indices(own64, inp.q_pos[qsl], inp.kv_len[b:b + 1], k)[0, 0])
+        assert np.array_equal(g_sorted[b, t],
+                              O.topk_indices(own64, inp.q_pos[qsl], inp.kv_len[b:b + 1], k, sorted_by_score=True)[0, 0])
+        ref_idx = O.topk_indices(ref, inp.q_pos[qsl], inp.kv_len[b:b + 1], k)
+        P.check_topk_near_ties(g_idx[b, t][None], ref_idx[0], ref[0], mag[0], k)
+        # 4. attention over the GPU's selection
+        _check_mla(g_out[qsl], g_lse[qsl], inp.mla_q[qsl], inp.mla_kv[b:b + 1], g_idx[qsl])
 
 
 def test_pipeline_degenerate_sequences(table_dev):

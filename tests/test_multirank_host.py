@@ -91,3 +91,30 @@ def test_a_lost_rank_ends_the_reduction_with_an_error():
     what, waited = q.get(timeout=5)
     assert what != "no error"
     assert waited < 60
+
+
+def test_gpus_flag_starts_one_rank_per_gpu():
+    """`bench.py --gpus N` outside a launcher re-executes itself as N ranks under
+    torch.distributed.run (rendezvous on 127.0.0.1); checked with the reference arm, which needs
+    no GPU: rank 0 prints the line with n_gpus = N."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--workload", "tiny_decode", "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=600, env=env, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1 and lines[0]["n_gpus"] == 2 and lines[0]["impl"] == "reference"
+
+
+def test_gpus_flag_must_match_the_launched_world():
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--workload", "tiny_decode"],
+                       capture_output=True, text=True, timeout=300, env=env, cwd=root)
+    assert r.returncode == 2 and "WORLD_SIZE=1" in r.stderr
