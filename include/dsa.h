@@ -280,6 +280,28 @@ DSA_API int dsa_mla_out_absorb(const uint16_t* o, const uint16_t* w_uv, int64_t 
 DSA_API size_t dsa_sparse_mla_workspace_size(int B, int T, int k);
 
 /*
+ * dsa_sparse_mla_heads - dsa_sparse_mla over a head shard: the query heads of one rank when the
+ * 128 attention heads are split across ranks ("RoPE coefficients" page, MLA init excerpt: each
+ * rank keeps n_local_heads = n_heads / world_size heads; the selected indices are the same on
+ * every rank, which the Indexer.forward excerpt of "Rotate first features" broadcasts from rank 0).
+ *   heads  64 (a two-way split) or 128 (the whole set: the same as dsa_sparse_mla)
+ *   q      bf16 [B][T][heads][576];  out bf16 [B][T][heads][512];  lse fp32 [B][T][heads] or NULL
+ *   kv, idx, softmax_scale, workspace: as dsa_sparse_mla, the workspace sized by
+ *          dsa_sparse_mla_heads_workspace_size(B, T, k, heads)
+ * The result for head h of the shard is that of dsa_sparse_mla for the same query row. A 64-head
+ * shard runs one CTA per (query, key split) instead of a pair: its score rows fill half the TMEM
+ * lanes, and the other half accumulates the second half of the output features.
+ * Returns DSA_ERR_INVALID_ARG for any other head count; errors otherwise as dsa_sparse_mla.
+ */
+DSA_API int dsa_sparse_mla_heads(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
+                                 int B, int T, int S_max, int k, int heads, float softmax_scale,
+                                 uint16_t* out, float* lse, void* workspace, size_t ws_bytes,
+                                 dsa_stream_t stream);
+
+/* Bytes of device scratch dsa_sparse_mla_heads needs (0 when none, or for an invalid shape). */
+DSA_API size_t dsa_sparse_mla_heads_workspace_size(int B, int T, int k, int heads);
+
+/*
  * dsa_get_device_status - synchronises `stream`, returns the first error recorded by a kernel
  * since the last call (DSA_OK if none) and clears it. DSA_ERR_CUDA if the sync itself fails.
  */

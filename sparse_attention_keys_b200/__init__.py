@@ -15,7 +15,8 @@ import torch
 __all__ = [
     "DsaError", "lib", "lib_path", "DSA_HADAMARD", "DSA_FILL_MASKED", "DSA_SORTED", "DSA_F32", "DSA_BF16", "INDEXER_SOFTMAX_SCALE",
     "MLA_SOFTMAX_SCALE", "dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk",
-    "dsa_sparse_mla", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_noalloc",
+    "dsa_sparse_mla", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_noalloc", "dsa_sparse_mla_heads",
+    "dsa_sparse_mla_heads_workspace_size",
     "dsa_index_scores_paged", "dsa_sparse_mla_paged", "dsa_mla_q_absorb", "dsa_mla_kv_entry",
     "dsa_mla_out_absorb",
     "dsa_sparse_mla_noalloc_scratch_bytes", "dsa_get_device_status", "dsa_get_error_detail",
@@ -64,6 +65,9 @@ def _load():
     L.dsa_topk.argtypes = [vp, i64, vp, vp, i32, i32, i32, u32, vp, vp]
     L.dsa_sparse_mla.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
     L.dsa_sparse_mla_workspace_size.argtypes = [i32, i32, i32]
+    L.dsa_sparse_mla_heads.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
+    L.dsa_sparse_mla_heads_workspace_size.argtypes = [i32, i32, i32, i32]
+    L.dsa_sparse_mla_heads_workspace_size.restype = sz
     L.dsa_index_scores_paged.argtypes = [vp, vp, vp, vp, vp, i64, vp, i32, i32, vp, vp, i32, i32, f32, vp, i64, u32,
                                          vp]
     L.dsa_sparse_mla_paged.argtypes = [vp, vp, i64, vp, i32, i32, vp, i32, i32, i32, f32, vp, vp, vp, sz, vp]
@@ -82,6 +86,7 @@ def _load():
     L.dsa_device_supported.argtypes = []
     L.dsa_version.restype = ctypes.c_char_p
     for f in ("dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk", "dsa_sparse_mla",
+              "dsa_sparse_mla_heads",
               "dsa_sparse_mla_noalloc", "dsa_get_device_status", "dsa_get_error_detail",
               "dsa_selftest_wait_timeout", "dsa_device_supported"):
         getattr(L, f).restype = ctypes.c_int
@@ -236,21 +241,21 @@ def dsa_topk(scores, q_pos, kv_len, k: int, idx=None, flags: int = 0, stream=Non
     return idx
 
 
-def _mla_shapes(q, kv, idx, out, lse, kv_name="kv"):
+def _mla_shapes(q, kv, idx, out, lse, kv_name="kv", heads=128):
     """Shape and device checks of the sparse-MLA arguments (before any pointer reaches the library,
     so a mismatched buffer raises here instead of being written out of bounds):
-    q [B,T,128,576], kv [...,576], idx [B,T,k], out [B,T,128,512], lse [B,T,128] or None."""
-    if q.dim() != 4 or tuple(q.shape[2:]) != (128, 576):
-        raise ValueError(f"q must be [B, T, 128, 576], got {tuple(q.shape)}")
+    q [B,T,H,576], kv [...,576], idx [B,T,k], out [B,T,H,512], lse [B,T,H] or None (H = heads)."""
+    if q.dim() != 4 or tuple(q.shape[2:]) != (heads, 576):
+        raise ValueError(f"q must be [B, T, {heads}, 576], got {tuple(q.shape)}")
     B, T = int(q.shape[0]), int(q.shape[1])
     if kv.shape[-1] != 576:
         raise ValueError(f"{kv_name} rows must have 576 features, got {tuple(kv.shape)}")
     if idx.dim() != 3 or tuple(idx.shape[:2]) != (B, T) or idx.shape[2] < 1:
         raise ValueError(f"idx must be [B={B}, T={T}, k>=1], got {tuple(idx.shape)}")
-    if out is not None and tuple(out.shape) != (B, T, 128, 512):
-        raise ValueError(f"out must be [{B}, {T}, 128, 512], got {tuple(out.shape)}")
-    if lse is not None and tuple(lse.shape) != (B, T, 128):
-        raise ValueError(f"lse must be [{B}, {T}, 128], got {tuple(lse.shape)}")
+    if out is not None and tuple(out.shape) != (B, T, heads, 512):
+        raise ValueError(f"out must be [{B}, {T}, {heads}, 512], got {tuple(out.shape)}")
+    if lse is not None and tuple(lse.shape) != (B, T, heads):
+        raise ValueError(f"lse must be [{B}, {T}, {heads}], got {tuple(lse.shape)}")
     for t, n in ((kv, kv_name), (idx, "idx"), (out, "out"), (lse, "lse")):
         if t is not None and t.device != q.device:
             raise ValueError(f"{n} is on {t.device}, q on {q.device}: all tensors must be on one device")
@@ -290,6 +295,42 @@ def dsa_sparse_mla(q, kv, idx, softmax_scale: float = MLA_SOFTMAX_SCALE, out=Non
                              _ptr(lse), _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
                              _stream(stream))
     _check(rc, "dsa_sparse_mla")
+    return out, lse
+
+
+def dsa_sparse_mla_heads_workspace_size(B: int, T: int, k: int, heads: int) -> int:
+    return int(_lib.dsa_sparse_mla_heads_workspace_size(int(B), int(T), int(k), int(heads)))
+
+
+def dsa_sparse_mla_heads(q, kv, idx, softmax_scale: float = MLA_SOFTMAX_SCALE, out=None, lse=None, workspace=None,
+                         want_lse: bool = True, stream=None):
+    """dsa_sparse_mla over a head shard: q bf16 [B,T,H,576] with H = 64 (half of the heads, as one
+    rank of a two-way head split holds) or 128 -> (out bf16 [B,T,H,512], lse fp32 [B,T,H])."""
+    _need(q, torch.bfloat16, "q")
+    _need(kv, torch.bfloat16, "kv")
+    _need(idx, torch.int32, "idx")
+    if out is not None:
+        _need(out, torch.bfloat16, "out")
+    if lse is not None:
+        _need(lse, torch.float32, "lse")
+    heads = int(q.shape[2]) if q.dim() == 4 else -1
+    if heads not in (64, 128):
+        raise ValueError(f"q must hold 64 or 128 heads, got {tuple(q.shape)}")
+    if kv.dim() != 3 or kv.shape[0] != q.shape[0]:
+        raise ValueError(f"kv must be [B, S_max, 576], got {tuple(kv.shape)}")
+    B, T, k = _mla_shapes(q, kv, idx, out, lse, heads=heads)
+    if out is None:
+        out = torch.empty((B, T, heads, 512), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, T, heads), dtype=torch.float32, device=q.device)
+    ws_bytes = dsa_sparse_mla_heads_workspace_size(B, T, k, heads)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    rc = _lib.dsa_sparse_mla_heads(_ptr(q), _ptr(kv), _ptr(idx), B, T, kv.shape[1], int(k), heads,
+                                   float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+                                   0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                   _stream(stream))
+    _check(rc, "dsa_sparse_mla_heads")
     return out, lse
 
 

@@ -312,12 +312,17 @@ int dsa_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int32_
 
 size_t dsa_sparse_mla_workspace_size(int B, int T, int k) {
   if (B < 1 || T < 1 || k < 1) return 0;
-  return dsa::sparse_mla_workspace_size(B, T, k);
+  return dsa::sparse_mla_workspace_size(B, T, k, DSA_MLA_HEADS);
 }
 
-int dsa_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T, int S_max,
-                   int k, float softmax_scale, uint16_t* out, float* lse, void* workspace,
-                   size_t ws_bytes, dsa_stream_t stream) {
+size_t dsa_sparse_mla_heads_workspace_size(int B, int T, int k, int heads) {
+  if (B < 1 || T < 1 || k < 1 || (heads != 64 && heads != DSA_MLA_HEADS)) return 0;
+  return dsa::sparse_mla_workspace_size(B, T, k, heads);
+}
+
+static int sparse_mla_checked(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T, int S_max,
+                              int k, int heads, float softmax_scale, uint16_t* out, float* lse, void* workspace,
+                              size_t ws_bytes, dsa_stream_t stream) {
   if (B < 1 || T < 1 || S_max < 1 || k < 1 || !(softmax_scale > 0.f) || !isfinite(softmax_scale))
     return DSA_ERR_INVALID_ARG;
   if ((int64_t)B * T * 2 * 1024 > 0x7fffffffLL) return DSA_ERR_INVALID_ARG;
@@ -329,8 +334,22 @@ int dsa_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, in
   int* status;
   int rc = prologue(&status);
   if (rc != DSA_OK) return rc;
-  return dsa::launch_sparse_mla(q, kv, idx, B, T, S_max, k, softmax_scale, out, lse, workspace, ws_bytes,
+  return dsa::launch_sparse_mla(q, kv, idx, B, T, S_max, k, heads, softmax_scale, out, lse, workspace, ws_bytes,
                                 (cudaStream_t)stream, status);
+}
+
+int dsa_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T, int S_max,
+                   int k, float softmax_scale, uint16_t* out, float* lse, void* workspace,
+                   size_t ws_bytes, dsa_stream_t stream) {
+  return sparse_mla_checked(q, kv, idx, B, T, S_max, k, DSA_MLA_HEADS, softmax_scale, out, lse, workspace, ws_bytes,
+                            stream);
+}
+
+int dsa_sparse_mla_heads(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T, int S_max, int k,
+                         int heads, float softmax_scale, uint16_t* out, float* lse, void* workspace, size_t ws_bytes,
+                         dsa_stream_t stream) {
+  if (heads != 64 && heads != DSA_MLA_HEADS) return DSA_ERR_INVALID_ARG;
+  return sparse_mla_checked(q, kv, idx, B, T, S_max, k, heads, softmax_scale, out, lse, workspace, ws_bytes, stream);
 }
 
 static bool weights_ok(const uint16_t* w, int64_t w_head_stride) {

@@ -25,7 +25,7 @@ int launch_index_scores_paged(const uint8_t* q8, const float* q_scale, const flo
 int launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int32_t* kv_len, int B,
                 int T, int k, uint32_t flags, int32_t* idx, cudaStream_t stream, int* status);
 
-size_t sparse_mla_workspace_size(int B, int T, int k);
+size_t sparse_mla_workspace_size(int B, int T, int k, int heads);
 int launch_sparse_mla_paged(const uint16_t* q, const uint16_t* kv_pool, int64_t num_pages,
                             const int32_t* block_table, int max_pages, int page_size, const int32_t* idx, int B,
                             int T, int k, float softmax_scale, uint16_t* out, float* lse, void* workspace,
@@ -39,7 +39,7 @@ int launch_mla_kv_entry(const uint16_t* kv, const uint16_t* k_pe, const int32_t*
 int launch_mla_out_absorb(const uint16_t* o, const uint16_t* w_uv, int64_t w_head_stride, int64_t rows,
                           uint16_t* out, cudaStream_t stream, int* status);
 int launch_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T,
-                      int S_max, int k, float softmax_scale, uint16_t* out, float* lse,
+                      int S_max, int k, int heads, float softmax_scale, uint16_t* out, float* lse,
                       void* workspace, size_t ws_bytes, cudaStream_t stream, int* status);
 
 }  // namespace dsa

@@ -50,27 +50,40 @@ namespace dsa {
 
 namespace {
 
-constexpr int kHeads = 128;
+constexpr int kHeads = 128;                        // TMEM lanes = MMA M
 constexpr int kDqk = 576;
 constexpr int kDv = 512;
 constexpr int kKeys = 32;                          // selected keys per tile (N of Q K^T)
 constexpr int kRegions = 9;                        // 576 features = 9 blocks of 64 (128 B), 128B swizzle
-constexpr int kVRegions = 4;                       // the blocks of this CTA's 256 output features
-constexpr int kRestRegions = kRegions - kVRegions; // the other half's 4 latent blocks + the rotary one
 constexpr int kQTmemRegions = 5;                   // Q features 0..319 live in TMEM
 constexpr int kQRegion = kHeads * 128;             // 16 KB
 constexpr int kQBytes = (kRegions - kQTmemRegions) * kQRegion;   // 64 KB: features 320..575
 constexpr int kKvRegion = kKeys * 128;             // 4 KB: one 64-feature block of a tile
-constexpr int kVSlotBytes = kVRegions * kKvRegion;        // 16 KB
-constexpr int kRestSlotBytes = kRestRegions * kKvRegion;  // 20 KB
-constexpr int kVSlots = 5, kRestSlots = 4, kSBufs = 3;
-constexpr int kOffQ = 0;
-constexpr int kOffV = kOffQ + kQBytes;
-constexpr int kOffRest = kOffV + kVSlots * kVSlotBytes;
-constexpr int kOffBar = kOffRest + kRestSlots * kRestSlotBytes;
-constexpr int kSmemBytes = 1024 + kOffBar + 256;
+
+// Shared-memory rings for the two layouts. 128 heads (a CTA pair per (query, split)): the "V ring"
+// holds the four 64-feature blocks of this CTA's output half, the "rest ring" the other half's
+// four and the rotary block. 64 heads (one CTA per (query, split), the head-parallel shard): the V
+// ring holds all eight latent blocks, the rest ring the rotary block.
+template <int HEADS>
+struct MlaCfg {
+  static_assert(HEADS == 128 || HEADS == 64, "128 heads, or a 64-head shard");
+  static constexpr int kVRegions = HEADS == 128 ? 4 : 8;
+  static constexpr int kRestRegions = kRegions - kVRegions;
+  static constexpr int kVSlotBytes = kVRegions * kKvRegion;
+  static constexpr int kRestSlotBytes = kRestRegions * kKvRegion;
+  static constexpr int kVSlots = HEADS == 128 ? 5 : 4;
+  static constexpr int kRestSlots = 4;
+  static constexpr int kOffV = kQBytes;
+  static constexpr int kOffRest = kOffV + kVSlots * kVSlotBytes;
+  static constexpr int kOffBar = kOffRest + kRestSlots * kRestSlotBytes;
+  static constexpr int kSmemBytes = 1024 + kOffBar + 256;
+  static constexpr int kCtasPerUnit = HEADS == 128 ? 2 : 1;   // CTAs per (query, split)
+};
+constexpr int kSBufs = 3;
 constexpr int kStageRow = 256 + 4;                 // floats per staged output row (1040 B: conflict-free)
-static_assert(kOffV + kHeads * kStageRow * 4 <= kOffBar, "output staging fits in the KV rings");
+static_assert(MlaCfg<128>::kOffV + kHeads * kStageRow * 4 <= MlaCfg<128>::kOffBar, "output staging fits");
+static_assert(MlaCfg<64>::kOffV + kHeads * kStageRow * 4 <= MlaCfg<64>::kOffBar, "output staging fits");
+static_assert(MlaCfg<128>::kSmemBytes <= 232448 && MlaCfg<64>::kSmemBytes <= 232448, "shared memory per CTA");
 constexpr int kSoftmaxWarps = 4, kPvWarp = 4, kGatherWarp = 5, kGatherWarps = 4, kQkWarp = 9, kQkWarps = kSBufs;
 constexpr int kMlaThreads = (kSoftmaxWarps + 1 + kGatherWarps + kQkWarps) * 32;
 constexpr int kMaxSlots = 2048;                    // selected slots per CTA (split chunk cap)
@@ -82,9 +95,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 // any magnitude), l below 2^43 and O far from the fp32 range, and a rescale, which stalls the
 // warp that does it while the other softmax warps wait at the next barrier, becomes rare.
 constexpr float kRescaleThreshold = 32.0f;         // log2 units
-static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 static_assert(kTmemQ + kQTmemRegions * 32 == kTmemCols, "TMEM budget");
-static_assert(kTmemQ <= kTmemCols, "TMEM budget");
 
 struct MlaSplit {
   int nsplit;
@@ -94,7 +105,7 @@ struct MlaSplit {
 // Key splits per query. Each CTA pays a fixed pipeline fill (about four tiles' time: Q staging and
 // the first gather) and the splits need a merge pass, so the count minimises an estimate in tile
 // units: waves x (tiles per CTA + fill) + merge, with waves = ceil(CTAs / SMs).
-MlaSplit choose_split(int64_t BT, int k, int sms) {
+MlaSplit choose_split(int64_t BT, int k, int sms, int ctas_per_unit, int heads) {
   constexpr double kFillTiles = 4.0, kMergeTiles = 2.0;
   constexpr double kMergeTilesPerMB = 0.15;          // partials written + read, ~1.2 us per tile at HBM rate
   const int n_min = (k + kMaxSlots - 1) / kMaxSlots;  // a split holds at most kMaxSlots slots
@@ -105,10 +116,10 @@ MlaSplit choose_split(int64_t BT, int k, int sms) {
     int chunk = (k + n - 1) / n;
     chunk = (chunk + kKeys - 1) / kKeys * kKeys;     // <= kMaxSlots, a multiple of kKeys
     const int nsplit = (k + chunk - 1) / chunk;
-    const int64_t ctas = BT * 2 * nsplit;
+    const int64_t ctas = BT * ctas_per_unit * nsplit;
     const double waves = (double)((ctas + sms - 1) / sms);
     double cost = waves * (chunk / kKeys + kFillTiles);
-    if (nsplit > 1) cost += kMergeTiles + kMergeTilesPerMB * (double)BT * nsplit * kHeads * kDv * 8 / 1e6;
+    if (nsplit > 1) cost += kMergeTiles + kMergeTilesPerMB * (double)BT * nsplit * heads * kDv * 8 / 1e6;
     if (cost < best_cost) {
       best_cost = cost;
       best.nsplit = nsplit;
@@ -135,12 +146,13 @@ struct MlaParams {
   const uint16_t* kv;
   const int32_t* idx;
   int B, T, S_max, k;
+  int heads;                 // query heads per row of q / out / lse (128, or a 64-head shard)
   int nsplit, chunk;
   float scale_log2;          // softmax_scale * log2(e)
   uint16_t* out;
   float* lse;
-  float* part_o;             // [BT][nsplit][128][512]   (nsplit > 1)
-  float* part_ml;            // [BT][nsplit][128][2]     running max (log2 domain), sum
+  float* part_o;             // [BT][nsplit][heads][512]   (nsplit > 1)
+  float* part_ml;            // [BT][nsplit][heads][2]     running max (log2 domain), sum
   int* status;
   // paged latent cache: kv is a pool of num_pages pages of page_size rows, and logical position v of
   // sequence b lives in row block_table[b][v / page_size] * page_size + v % page_size
@@ -161,18 +173,20 @@ __device__ __forceinline__ int kv_row(const MlaParams& p, int v, int pg) {
   return PAGED ? (pg << p.page_shift) + (v & (p.page_size - 1)) : v;
 }
 
-// Q K^T of one 32-key tile: 20 K-steps with Q from TMEM, then 16 with Q from shared memory. HALF
-// fixes which ring holds each 64-feature block, so every B descriptor is a base plus a constant.
-// *_lo: low descriptor words (start address >> 4 in bits 0-13) of the shared-memory bases; hi: the
-// common high word of the K-major 128B-swizzle descriptors.
-template <int HALF>
+// Q K^T of one 32-key tile: 20 K-steps with Q from TMEM, then 16 with Q from shared memory. LAYOUT
+// fixes which ring holds each 64-feature block (0 / 1: the output half of a CTA of a 128-head pair;
+// 2: the 64-head shard, latent blocks in the V ring and the rotary block in the rest ring), so every
+// B descriptor is a base plus a constant. *_lo: low descriptor words (start address >> 4 in bits
+// 0-13) of the shared-memory bases; hi: the common high word of the K-major 128B-swizzle descriptors.
+template <int LAYOUT>
 __device__ __forceinline__ void issue_qk_tile(uint32_t d, uint32_t tq, uint32_t q_lo, uint32_t v_lo, uint32_t r_lo,
                                               uint32_t hi, uint32_t idesc) {
 #pragma unroll
   for (int r = 0; r < kRegions; ++r) {
-    const bool in_v = r < 8 && (r >> 2) == HALF;
-    const uint32_t kb = in_v ? v_lo + (uint32_t)(((r & 3) * kKvRegion) >> 4)
-                             : r_lo + (uint32_t)(((r == 8 ? 4 : (r & 3)) * kKvRegion) >> 4);
+    const bool in_v = LAYOUT == 2 ? r < 8 : (r < 8 && (r >> 2) == LAYOUT);
+    const int v_blk = LAYOUT == 2 ? r : (r & 3);
+    const int r_blk = LAYOUT == 2 ? 0 : (r == 8 ? 4 : (r & 3));
+    const uint32_t kb = in_v ? v_lo + (uint32_t)((v_blk * kKvRegion) >> 4) : r_lo + (uint32_t)((r_blk * kKvRegion) >> 4);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       const int ks = 4 * r + kk;
@@ -187,12 +201,22 @@ __device__ __forceinline__ void issue_qk_tile(uint32_t d, uint32_t tq, uint32_t 
   }
 }
 
-template <bool PAGED>
+// HEADS = 128: two CTAs per (query, key split), CTA c owning output features [256c, 256c + 256).
+// HEADS = 64 (a head-parallel shard of the 128 heads): one CTA per (query, key split). TMEM lanes
+// 64..127 hold a copy of heads 0..63 (their Q rows are staged twice, so Q K^T writes every score
+// row twice), and P V runs block-diagonally: lanes 0..63 write P into the first 16 columns of the
+// score buffer and zeros into the last 16, lanes 64..127 the reverse, and four MMAs accumulate
+// P V[:, 0:256] into lanes 0..63 and P V[:, 256:512] into lanes 64..127 of the same 256 O columns.
+template <bool PAGED, int HEADS>
 __global__ void __launch_bounds__(kMlaThreads, 1)
     sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) {
+  using Cfg = MlaCfg<HEADS>;
+  constexpr int kVRegions = Cfg::kVRegions, kVSlots = Cfg::kVSlots, kRestSlots = Cfg::kRestSlots;
+  constexpr int kVSlotBytes = Cfg::kVSlotBytes, kRestSlotBytes = Cfg::kRestSlotBytes;
+  constexpr int kOffV = Cfg::kOffV, kOffRest = Cfg::kOffRest, kOffBar = Cfg::kOffBar;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_sm = smem + kOffQ;
+  uint8_t* q_sm = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* kv_full = bars;                         // [kRestSlots] gather (cp.async) -> Q K^T issuer
   uint64_t* rest_empty = bars + kRestSlots;         // [kRestSlots] Q K^T done -> gather
@@ -206,8 +230,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int half = blockIdx.x & 1;             // output features [256*half, 256*half + 256)
-  const int unit = blockIdx.x >> 1;
+  // 128 heads: this CTA's output features [256*half, 256*half + 256); 64 heads: one CTA per unit
+  const int half = HEADS == 128 ? (int)(blockIdx.x & 1) : 0;
+  const int unit = HEADS == 128 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int q_head = tid & (HEADS - 1);        // softmax thread: the query head of its TMEM lane
   const int split = unit % p.nsplit;
   const int64_t bt = unit / p.nsplit;
   const int b = (int)(bt / p.T);
@@ -221,7 +247,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   // TMEM below). A prefetch is only a hint, so it is safe even if the preceding kernel is still
   // writing Q; every actual read of Q, and of the indices, comes after grid_dep_wait.
   if (warp < kSoftmaxWarps && ntiles > 0) {
-    const char* qrow = reinterpret_cast<const char*>(p.q + (bt * kHeads + tid) * kDqk);
+    const char* qrow = reinterpret_cast<const char*>(p.q + (bt * HEADS + q_head) * kDqk);
 #pragma unroll
     for (int i = 0; i < kQTmemRegions; ++i) asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + 128 * i));
   }
@@ -275,7 +301,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         tc_fence_after();
         const uint32_t v_lo = v_lo0 + (uint32_t)(((j % kVSlots) * kVSlotBytes) >> 4);
         const uint32_t r_lo = r_lo0 + (uint32_t)(((j % kRestSlots) * kRestSlotBytes) >> 4);
-        if (half == 0) issue_qk_tile<0>(d, tq, q_lo, v_lo, r_lo, hi, idesc_s);
+        if (HEADS == 64) issue_qk_tile<2>(d, tq, q_lo, v_lo, r_lo, hi, idesc_s);
+        else if (half == 0) issue_qk_tile<0>(d, tq, q_lo, v_lo, r_lo, hi, idesc_s);
         else issue_qk_tile<1>(d, tq, q_lo, v_lo, r_lo, hi, idesc_s);
         mma_commit(&s_full[e]);
         mma_commit(&rest_empty[j % kRestSlots]);
@@ -290,8 +317,12 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     if (w == 0 && lane == 0 && ntiles > 0) {
       prefetch_tensormap(&q_map);
       mbar_arrive_expect_tx(q_full, kQBytes);
-      for (int r = kQTmemRegions; r < kRegions; ++r)
-        tma_load_2d(q_sm + (r - kQTmemRegions) * kQRegion, &q_map, q_full, 64 * r, (int32_t)(bt * kHeads));
+      for (int r = kQTmemRegions; r < kRegions; ++r) {
+        uint8_t* dst = q_sm + (r - kQTmemRegions) * kQRegion;
+        tma_load_2d(dst, &q_map, q_full, 64 * r, (int32_t)(bt * HEADS));
+        // 64 heads: the same 64 rows again into rows 64..127 (8 KB on: whole 8-row swizzle atoms)
+        if (HEADS == 64) tma_load_2d(dst + 64 * 128, &q_map, q_full, 64 * r, (int32_t)(bt * HEADS));
+      }
     }
     const uint16_t* kv_b = PAGED ? p.kv : p.kv + (int64_t)b * p.S_max * kDqk;
     const int32_t* pages = PAGED ? p.block_table + (int64_t)b * p.max_pages : nullptr;
@@ -330,9 +361,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         break;
       const uint32_t v_slot = v_ring + (j % kVSlots) * kVSlotBytes;
       const uint32_t r_slot = rest_ring + (j % kRestSlots) * kRestSlotBytes;
-      const uint32_t d0 = (half == 0 ? v_slot : r_slot) + blk;           // latent block L/8
-      const uint32_t d1 = (half == 1 ? v_slot : r_slot) + blk;           // latent block 4 + L/8
-      const uint32_t d2 = r_slot + 4 * kKvRegion;                        // rotary block
+      // latent blocks L/8 and 4 + L/8, and the rotary block
+      const uint32_t d0 = HEADS == 64 ? v_slot + blk : (half == 0 ? v_slot : r_slot) + blk;
+      const uint32_t d1 = HEADS == 64 ? v_slot + 4 * kKvRegion + blk : (half == 1 ? v_slot : r_slot) + blk;
+      const uint32_t d2 = HEADS == 64 ? r_slot : r_slot + 4 * kKvRegion;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const int row = __shfl_sync(0xffffffffu, row_cur, kk);
@@ -360,6 +392,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         if (j == 0) mma_f16_ts_lo<0>(tmem + kTmemO, a, v_lo, hi, idesc_pv);
         else mma_f16_ts_lo<1>(tmem + kTmemO, a, v_lo, hi, idesc_pv);
         mma_f16_ts_lo<1>(tmem + kTmemO, a + 8, v_lo + (2048 >> 4), hi, idesc_pv);    // keys 16..31
+        if (HEADS == 64) {       // the block-diagonal second half: P of lanes 64..127 times V[:, 256:512]
+          mma_f16_ts_lo<1>(tmem + kTmemO, a + 16, v_lo + ((4 * kKvRegion) >> 4), hi, idesc_pv);
+          mma_f16_ts_lo<1>(tmem + kTmemO, a + 24, v_lo + ((4 * kKvRegion + 2048) >> 4), hi, idesc_pv);
+        }
         mma_commit(&pv_done[j % kSBufs]);
         mma_commit(&v_empty[j % kVSlots]);
       }
@@ -373,7 +409,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // Q features 0..319 of head h -> TMEM as bf16 pairs (feature f in column f/2)
     if (ntiles > 0) {
       // two batches of loads, each fully in flight before its TMEM stores (which order memory)
-      const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (bt * kHeads + h) * kDqk);
+      const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (bt * HEADS + q_head) * kDqk);
       auto stage = [&](int c0, int nc) {
         uint4 v[3 * 8];
 #pragma unroll
@@ -478,7 +514,18 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         }
       }
       m = m_new;
-      tmem_st16(t_row + s_col, pk);              // P over the scores it came from
+      if (HEADS == 128) {
+        tmem_st16(t_row + s_col, pk);            // P over the scores it came from
+      } else {                                   // the block-diagonal P of the 64-head shard
+        uint32_t pz[2 * (kKeys / 2)];
+        const bool low = warp < 2;               // lanes 0..63
+#pragma unroll
+        for (int i = 0; i < kKeys / 2; ++i) {
+          pz[i] = low ? pk[i] : 0u;
+          pz[kKeys / 2 + i] = low ? 0u : pk[i];
+        }
+        tmem_st32(t_row + s_col, pz);
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[j % kSBufs]);
@@ -491,6 +538,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // partial of a key split) in the now idle KV rings, then one bulk copy (TMA engine) per row
     // writes it out: the row is contiguous in global memory.
     const bool final_out = p.nsplit == 1;
+    // 128 heads: lane h is head h, features of this CTA's half; 64 heads: lane h is head h mod 64,
+    // features [256 * (h / 64), + 256)
+    const int o_half = HEADS == 128 ? half : (h >> 6);
     const float scale = final_out ? (l > 0.f ? 1.f / l : 0.f) : 1.f;
     uint8_t* srow = smem + kOffV + h * kStageRow * 4;
 #pragma unroll 1
@@ -526,13 +576,13 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     }
     fence_proxy_async_smem();                          // the row's generic writes -> the bulk copy's reads
     if (final_out) {
-      bulk_store_s2g(p.out + (bt * kHeads + h) * kDv + 256 * half, smem_u32(srow), 256 * 2);
-      if (p.lse && half == 0)
-        p.lse[bt * kHeads + h] = l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+      bulk_store_s2g(p.out + (bt * HEADS + q_head) * kDv + 256 * o_half, smem_u32(srow), 256 * 2);
+      if (p.lse && o_half == 0)
+        p.lse[bt * HEADS + q_head] = l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
     } else {
-      const int64_t prow = (bt * p.nsplit + split) * kHeads + h;
-      bulk_store_s2g(p.part_o + prow * kDv + 256 * half, smem_u32(srow), 256 * 4);
-      if (half == 0) *reinterpret_cast<float2*>(p.part_ml + prow * 2) = make_float2(m, l);
+      const int64_t prow = (bt * p.nsplit + split) * HEADS + q_head;
+      bulk_store_s2g(p.part_o + prow * kDv + 256 * o_half, smem_u32(srow), 256 * 4);
+      if (o_half == 0) *reinterpret_cast<float2*>(p.part_ml + prow * 2) = make_float2(m, l);
     }
     bulk_commit();
     bulk_wait_all();                                   // shared memory stays valid until the copy is done
@@ -555,10 +605,10 @@ __global__ void __launch_bounds__(256) sparse_mla_combine_kernel(const MlaParams
   grid_dep_wait();                                   // the partials come from the preceding kernel
   grid_dep_launch();
   if (wid >= rows) return;
-  const int64_t bt = wid / kHeads;
-  const int head = (int)(wid - bt * kHeads);
+  const int64_t bt = wid / p.heads;
+  const int head = (int)(wid - bt * p.heads);
   const float2* ml = reinterpret_cast<const float2*>(p.part_ml);
-  auto ml_of = [&](int s) { return __ldg(ml + (bt * p.nsplit + s) * kHeads + head); };
+  auto ml_of = [&](int s) { return __ldg(ml + (bt * p.nsplit + s) * p.heads + head); };
   float m_all = -INFINITY;
   for (int s = lane; s < p.nsplit; s += 32) m_all = fmaxf(m_all, ml_of(s).x);
 #pragma unroll
@@ -584,7 +634,7 @@ __global__ void __launch_bounds__(256) sparse_mla_combine_kernel(const MlaParams
       if (s < p.nsplit) {
         wgt[u] = weight(ml_of(s).x);
         const float4* src =
-            reinterpret_cast<const float4*>(p.part_o + ((bt * p.nsplit + s) * kHeads + head) * kDv + lane * 16);
+            reinterpret_cast<const float4*>(p.part_o + ((bt * p.nsplit + s) * p.heads + head) * kDv + lane * 16);
 #pragma unroll
         for (int i = 0; i < 4; ++i) v[u][i] = __ldcs(src + i);
       }
@@ -603,60 +653,68 @@ __global__ void __launch_bounds__(256) sparse_mla_combine_kernel(const MlaParams
   uint32_t packed[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) packed[i] = pack_bf16(acc[2 * i] * inv, acc[2 * i + 1] * inv);
-  uint4* dst = reinterpret_cast<uint4*>(p.out + (bt * kHeads + head) * kDv + lane * 16);
+  uint4* dst = reinterpret_cast<uint4*>(p.out + (bt * p.heads + head) * kDv + lane * 16);
   dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
   dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
   if (p.lse && lane == 0)
-    p.lse[bt * kHeads + head] = l_all > 0.f ? (m_all + log2f(l_all)) * 0.6931471805599453f : -INFINITY;
+    p.lse[bt * p.heads + head] = l_all > 0.f ? (m_all + log2f(l_all)) * 0.6931471805599453f : -INFINITY;
 }
 
-size_t sparse_mla_workspace_size(int B, int T, int k) {
+static MlaSplit split_for(int64_t BT, int k, int heads) {
+  return choose_split(BT, k, dsa_host::device_sm_count(), heads == 128 ? MlaCfg<128>::kCtasPerUnit : MlaCfg<64>::kCtasPerUnit,
+                      heads);
+}
+
+size_t sparse_mla_workspace_size(int B, int T, int k, int heads) {
   const int64_t BT = (int64_t)B * T;
-  const MlaSplit s = choose_split(BT, k, dsa_host::device_sm_count());
+  const MlaSplit s = split_for(BT, k, heads);
   if (s.nsplit <= 1) return 0;
-  return (size_t)BT * s.nsplit * kHeads * (kDv + 2) * sizeof(float);
+  return (size_t)BT * s.nsplit * heads * (kDv + 2) * sizeof(float);
 }
 
-template <bool PAGED>
+template <bool PAGED, int HEADS>
 static int launch_mla(const uint16_t* q, MlaParams p, cudaStream_t stream, void* workspace, size_t ws_bytes) {
+  using Cfg = MlaCfg<HEADS>;
   const int64_t BT = (int64_t)p.B * p.T;
   if (BT == 0) return DSA_OK;
-  const MlaSplit s = choose_split(BT, p.k, dsa_host::device_sm_count());
+  p.heads = HEADS;
+  const MlaSplit s = split_for(BT, p.k, HEADS);
   p.nsplit = s.nsplit; p.chunk = s.chunk;
   if (s.nsplit > 1) {
-    const size_t need = (size_t)BT * s.nsplit * kHeads * (kDv + 2) * sizeof(float);
+    const size_t need = (size_t)BT * s.nsplit * HEADS * (kDv + 2) * sizeof(float);
     if (workspace == nullptr || ws_bytes < need) return DSA_ERR_WORKSPACE;
     p.part_o = static_cast<float*>(workspace);
-    p.part_ml = p.part_o + (size_t)BT * s.nsplit * kHeads * kDv;
+    p.part_ml = p.part_o + (size_t)BT * s.nsplit * HEADS * kDv;
   }
   static uint64_t configured[dsa_host::kMaxSetupDevices] = {};
   if (dsa_host::needs_setup(configured, nullptr)) {
-    if (cudaFuncSetAttribute(sparse_mla_kernel<PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(sparse_mla_kernel<PAGED, HEADS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::kSmemBytes) != cudaSuccess)
       return DSA_ERR_CUDA;
     dsa_host::mark_setup(configured);
   }
-  const int64_t grid = BT * s.nsplit * 2;          // two CTAs (output-feature halves) per (query, split)
+  const int64_t grid = BT * s.nsplit * Cfg::kCtasPerUnit;
   if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;
-  CUtensorMap q_map;
+  CUtensorMap q_map;                               // Q rows of HEADS heads, boxes of 64 features
   if (!dsa_host::encode_tensor_map_2d(&q_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (void*)q, kDqk,
-                                      (uint64_t)BT * kHeads, kDqk * 2, 64, kHeads, CU_TENSOR_MAP_SWIZZLE_128B))
+                                      (uint64_t)BT * HEADS, kDqk * 2, 64, HEADS, CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
-  int rc = dsa_host::launch(sparse_mla_kernel<PAGED>, dim3((unsigned)grid), dim3(kMlaThreads), kSmemBytes, stream,
-                            q_map, p);
+  int rc = dsa_host::launch(sparse_mla_kernel<PAGED, HEADS>, dim3((unsigned)grid), dim3(kMlaThreads), Cfg::kSmemBytes,
+                            stream, q_map, p);
   if (rc != DSA_OK || s.nsplit == 1) return rc;
-  const int64_t rows = BT * kHeads;
+  const int64_t rows = BT * HEADS;
   return dsa_host::launch(sparse_mla_combine_kernel, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, stream, p, rows);
 }
 
 int launch_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T,
-                      int S_max, int k, float softmax_scale, uint16_t* out, float* lse,
+                      int S_max, int k, int heads, float softmax_scale, uint16_t* out, float* lse,
                       void* workspace, size_t ws_bytes, cudaStream_t stream, int* status) {
   MlaParams p{};
   p.q = q; p.kv = kv; p.idx = idx; p.B = B; p.T = T; p.S_max = S_max; p.k = k;
   p.scale_log2 = softmax_scale * kLog2e;
   p.out = out; p.lse = lse; p.status = status;
-  return launch_mla<false>(q, p, stream, workspace, ws_bytes);
+  if (heads == 64) return launch_mla<false, 64>(q, p, stream, workspace, ws_bytes);
+  return launch_mla<false, 128>(q, p, stream, workspace, ws_bytes);
 }
 
 int launch_sparse_mla_paged(const uint16_t* q, const uint16_t* kv_pool, int64_t num_pages,
@@ -669,7 +727,7 @@ int launch_sparse_mla_paged(const uint16_t* q, const uint16_t* kv_pool, int64_t 
   p.out = out; p.lse = lse; p.status = status;
   p.block_table = block_table; p.max_pages = max_pages; p.page_size = page_size; p.num_pages = num_pages;
   p.page_shift = __builtin_ctz((unsigned)page_size);
-  return launch_mla<true>(q, p, stream, workspace, ws_bytes);
+  return launch_mla<true, 128>(q, p, stream, workspace, ws_bytes);
 }
 
 }  // namespace dsa

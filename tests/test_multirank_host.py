@@ -118,3 +118,64 @@ def test_gpus_flag_must_match_the_launched_world():
     r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--workload", "tiny_decode"],
                        capture_output=True, text=True, timeout=300, env=env, cwd=root)
     assert r.returncode == 2 and "WORLD_SIZE=1" in r.stderr
+
+
+def _head_parallel_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import numpy as np
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import importlib.util
+        root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+        spec = importlib.util.spec_from_file_location(
+            "head_parallel", os.path.join(root, "sparse_attention_keys_b200", "head_parallel.py"))
+        hp = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(hp)            # the plumbing alone: no CUDA library on this host
+        import dsa_inputs as DI
+        from oracle import dsa_oracle as O
+        inp = DI.make_custom(2, 2, 96, 16, decode=False, seed=11)    # identical inputs on every rank
+        # only the source rank has the indexer's selection; the others hold garbage until the broadcast
+        if rank == 0:
+            rng = np.random.default_rng(5)
+            idx_np = np.stack([np.stack([np.sort(rng.choice(96, 16, replace=False)) for _ in range(2)])
+                               for _ in range(2)]).astype(np.int32)
+        else:
+            idx_np = np.full((2, 2, 16), 12345, np.int32)
+        idx = torch.from_numpy(idx_np.copy())
+        sl = hp.head_shard(rank, world)
+
+        def oracle_attend(q_local, kv, idx_t):
+            return O.sparse_mla(q_local, kv, idx_t.numpy())
+
+        out, lse = hp.sparse_mla_head_parallel(np.ascontiguousarray(inp.mla_q[:, :, sl]), inp.mla_kv, idx,
+                                               attend=oracle_attend)
+        q.put((rank, sl.start, sl.stop, idx.numpy().copy(), out, lse))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_parallel_plumbing_two_ranks():
+    """Two gloo ranks: rank 0's selected indices reach rank 1 through the broadcast, each rank
+    attends with its 64 heads (the oracle stands in for the kernel on CPU), and the two shards
+    put together are the 128-head result."""
+    import numpy as np
+    import dsa_inputs as DI
+    from oracle import dsa_oracle as O
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_head_parallel_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted([q.get(timeout=300) for _ in range(2)], key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    (r0, a0, b0, idx0, out0, lse0), (r1, a1, b1, idx1, out1, lse1) = res
+    assert (a0, b0, a1, b1) == (0, 64, 64, 128)
+    assert np.array_equal(idx0, idx1) and not np.any(idx1 == 12345)
+    inp = DI.make_custom(2, 2, 96, 16, decode=False, seed=11)
+    full, full_lse = O.sparse_mla(inp.mla_q, inp.mla_kv, idx0)
+    assert np.array_equal(np.concatenate([out0, out1], axis=2), full)
+    assert np.array_equal(np.concatenate([lse0, lse1], axis=2), full_lse)
