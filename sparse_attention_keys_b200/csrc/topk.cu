@@ -379,6 +379,348 @@ __global__ void __launch_bounds__(kTopkThreads, 4) topk_kernel(const float* __re
   }
 }
 
+// ------------------------------------------------------------------------------------------------
+// Register-resident variant, for rows of at most kRegRowMax keys (every workload of the pages'
+// model: max_seq_len is 16384). The row is read with coalesced 16-byte loads and transposed through
+// shared memory so that thread t holds the KPT order keys of positions [t*KPT, t*KPT+KPT) in
+// registers. Every later step works on per-thread bit masks over those keys (bit i: position
+// t*KPT + i), with branch-free per-key loops:
+//   - digit 1 (key bits 31..21) is histogrammed over every key, digit 2 (bits 20..10) over the
+//     keys on digit 1 only;
+//   - the few keys left on the first 22 bits go to a short shared-memory list, where one step finds
+//     the k-th largest key exactly (ties by position) and marks each listed key above or equal to
+//     it in per-thread mask words (a radix pass over bits 9..0 does this instead if the list would
+//     overflow);
+//   - one block scan of packed (above, equal) counts orders the selection by position (each thread's
+//     run is contiguous), and the positions are staged in shared memory and leave in coalesced
+//     16-byte stores.
+constexpr int kRegThreads = 512;
+constexpr int kRegWarps = kRegThreads / 32;
+constexpr int kRegRowMax = 16384;
+constexpr int kListCap = 256;                               // keys on the first 22 bits picked directly
+// shared words: h1 (2048) | h2 (2048) | h3 (1024) | above / equal masks (512 + 512) | list keys,
+// positions (kListCap each) | a region for the transposed row, later the staged output
+constexpr int kRegFixedWords = 2048 + 2048 + 1024 + 2 * kRegThreads + 2 * kListCap;
+__host__ __device__ constexpr int reg_row_words(int kpt) { return kpt * kRegThreads / 32 * 36; }
+
+// hist[bin] += 1 when `pred`, as one predicated shared-memory reduction (no branch, no return value).
+__device__ __forceinline__ void hist_inc_if(uint32_t* hist, uint32_t bin, bool pred) {
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t@p red.shared.add.u32 [%0], 1;\n\t}" ::"r"(
+                   smem_u32(hist + bin)),
+               "r"((uint32_t)pred)
+               : "memory");
+}
+
+// dst[0] = v when `pred` (a predicated shared-memory store).
+__device__ __forceinline__ void st_shared_if(int32_t* dst, int32_t v, bool pred) {
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %2, 0;\n\t@p st.shared.s32 [%0], %1;\n\t}" ::"r"(smem_u32(dst)),
+               "r"(v), "r"((uint32_t)pred)
+               : "memory");
+}
+
+// Exclusive prefix, in thread order, of one value per thread of the CTA; *total gets the sum.
+// One barrier; `tot` (kRegWarps words) is written before it and read after it, so a call must not
+// reuse the `tot` of the previous call before another barrier.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tot, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const uint32_t o = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += o;
+  }
+  if (lane == 31) tot[warp] = incl;
+  __syncthreads();
+  const uint32_t wt = lane < kRegWarps ? tot[lane] : 0u;
+  uint32_t ws = wt;
+#pragma unroll
+  for (int d = 1; d < kRegWarps; d <<= 1) {
+    const uint32_t o = __shfl_up_sync(0xffffffffu, ws, d);
+    if (lane >= d) ws += o;
+  }
+  const uint32_t warp_before = __shfl_sync(0xffffffffu, ws - wt, warp);
+  *total = __shfl_sync(0xffffffffu, ws, kRegWarps - 1);
+  return warp_before + incl - v;
+}
+
+// The bin holding the target-th largest histogrammed key (bins scanned from the top; thread t
+// owns bins NB-1-t*C .. NB-C-t*C). Writes the bin to sel[0], the target's rank inside it (1-based)
+// to sel[1] and the bin's count to sel[2]; ends with a barrier.
+template <int NB>
+__device__ __forceinline__ void select_bin(const uint32_t* hist, uint32_t target, uint32_t* tot, uint32_t* sel) {
+  constexpr int C = NB / kRegThreads;
+  const int top = NB - 1 - (int)threadIdx.x * C;
+  uint32_t h[C];
+  uint32_t local = 0;
+#pragma unroll
+  for (int j = 0; j < C; ++j) {
+    h[j] = hist[top - j];
+    local += h[j];
+  }
+  uint32_t total;
+  uint32_t before = block_excl_scan(local, tot, &total);
+  if (before < target && target <= before + local) {
+#pragma unroll
+    for (int j = 0; j < C; ++j) {
+      if (before + h[j] >= target) {
+        sel[0] = (uint32_t)(top - j);
+        sel[1] = target - before;
+        sel[2] = h[j];
+        break;
+      }
+      before += h[j];
+    }
+  }
+  __syncthreads();
+}
+
+template <int KPT>
+__global__ void __launch_bounds__(kRegThreads, 2) topk_regs_kernel(const float* __restrict__ scores, int64_t ld,
+                                                                   const int32_t* __restrict__ q_pos,
+                                                                   const int32_t* __restrict__ kv_len, int T, int k,
+                                                                   uint32_t flags, int sort_n,
+                                                                   int32_t* __restrict__ idx, int* status) {
+  static_assert(KPT % 4 == 0 && KPT <= 32 && KPT * kRegThreads <= kRegRowMax, "keys per thread");
+  extern __shared__ __align__(16) uint32_t smem[];
+  uint32_t* h1 = smem;                                      // 2048 bins: key bits 31..21
+  uint32_t* h2 = smem + 2048;                               // 2048 bins: key bits 20..10
+  uint32_t* h3 = smem + 4096;                               // 1024 bins: key bits 9..0 (list overflow)
+  uint32_t* gt_words = smem + 5120;                         // per thread: its keys above the k-th (list keys)
+  uint32_t* eq_words = gt_words + kRegThreads;              //             and equal to it
+  uint32_t* list_key = eq_words + kRegThreads;              // keys on the first 22 bits of the k-th
+  int32_t* list_pos = reinterpret_cast<int32_t*>(list_key + kListCap);
+  uint32_t* region = smem + kRegFixedWords;                 // the transposed row, then the output
+  int32_t* stage = reinterpret_cast<int32_t*>(region);      // k positions, or
+  uint64_t* sbuf = reinterpret_cast<uint64_t*>(region);     // sort_n (score, position) keys
+  __shared__ uint32_t tots[4][kRegWarps];
+  __shared__ uint32_t sel[3];
+  __shared__ uint32_t n_list, thr_sh, need_sh;
+
+  const int64_t row = blockIdx.x;
+  const int b = (int)(row / T);
+  const int tid = threadIdx.x;
+  const bool sorted = (flags & DSA_SORTED) != 0;
+  grid_dep_wait();                                          // the scores come from the preceding kernel
+  grid_dep_launch();
+  int32_t* out = idx + row * (int64_t)k;
+  int n = min(q_pos[row] + 1, kv_len[b]);
+  if (n < 0) n = 0;
+  if (n <= k && !sorted) {                                  // everything visible is selected
+    for (int i = tid; i < k; i += kRegThreads) out[i] = i < n ? i : -1;
+    return;
+  }
+  if ((int64_t)n > ld) {                                    // the row buffer is shorter than the visible keys
+    if (tid == 0) set_status(status, DSA_ERR_DEVICE_BOUNDS);
+    for (int i = tid; i < k; i += kRegThreads) out[i] = -1;
+    return;
+  }
+  for (int i = tid; i < kRegFixedWords - 2 * kListCap; i += kRegThreads) smem[i] = 0u;
+  if (tid == 0) n_list = 0;
+
+  // coalesced 16-byte loads (ld is a multiple of 4, so a float4 that starts below n lies in the
+  // row), each written to the transposed layout: position p at word p + 4 (p / 32)
+  const float* src = scores + row * ld;
+  const int n4 = (n + 3) >> 2;
+#pragma unroll
+  for (int c = 0; c < KPT / 4; ++c) {
+    const int f = c * kRegThreads + tid;
+    if (f < n4) {
+      const float4 v = __ldcs(reinterpret_cast<const float4*>(src) + f);
+      *reinterpret_cast<float4*>(region + 4 * f + 4 * (f >> 3)) = v;
+    }
+  }
+  __syncthreads();
+  const int p0 = tid * KPT;
+  const int nv = max(0, min(KPT, n - p0));
+  uint32_t key[KPT];
+#pragma unroll
+  for (int c = 0; c < KPT / 4; ++c) {
+    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int pc = p0 + 4 * c;                              // at word pc + 4 (pc / 32)
+    if (4 * c < nv) f = *reinterpret_cast<const float4*>(region + pc + 4 * (pc >> 5));
+    key[4 * c] = order_key(f.x);
+    key[4 * c + 1] = order_key(f.y);
+    key[4 * c + 2] = order_key(f.z);
+    key[4 * c + 3] = order_key(f.w);
+  }
+  __syncthreads();                                          // the region is free again
+
+  if (n <= k) {                                             // DSA_SORTED with everything selected
+#pragma unroll
+    for (int i = 0; i < KPT; ++i)
+      if (i < nv) sbuf[p0 + i] = ((uint64_t)(~key[i]) << 32) | (uint32_t)(p0 + i);
+    for (int i = n + tid; i < sort_n; i += kRegThreads) sbuf[i] = ~0ull;
+    sort_and_write(sbuf, sort_n, n, k, out);
+    return;
+  }
+
+  const uint32_t valid = nv >= 32 ? 0xffffffffu : ((1u << nv) - 1u);
+  // digit 1 over every key (threads past the end of a short row skip the per-key work)
+  if (nv == KPT) {
+#pragma unroll
+    for (int i = 0; i < KPT; ++i) hist_inc_if(h1, key[i] >> 21, true);
+  } else if (nv > 0) {
+#pragma unroll
+    for (int i = 0; i < KPT; ++i) hist_inc_if(h1, key[i] >> 21, i < nv);
+  }
+  __syncthreads();
+  select_bin<2048>(h1, (uint32_t)k, tots[0], sel);
+  const uint32_t d1 = sel[0];
+  uint32_t rem = sel[1];
+  uint32_t m_gt = 0, m_on = 0;                              // above the k-th key / still undecided
+  if (nv > 0) {
+#pragma unroll
+    for (int i = 0; i < KPT; ++i) {
+      const uint32_t dg = key[i] >> 21;
+      m_gt |= (uint32_t)(dg > d1) << i;
+      m_on |= (uint32_t)(dg == d1) << i;
+    }
+    m_gt &= valid;
+    m_on &= valid;
+  }
+  // digit 2 over the keys on digit 1
+  if (m_on) {
+#pragma unroll
+    for (int i = 0; i < KPT; ++i) hist_inc_if(h2, (key[i] >> 10) & 2047u, (m_on >> i) & 1u);
+  }
+  __syncthreads();
+  select_bin<2048>(h2, rem, tots[1], sel);
+  const uint32_t pre22 = (d1 << 11) | sel[0];
+  rem = sel[1];
+  const uint32_t n_on = sel[2];                             // keys on the first 22 bits of the k-th
+  if (m_on) {
+    uint32_t m2 = 0, g2 = 0;
+#pragma unroll
+    for (int i = 0; i < KPT; ++i) {
+      const uint32_t pfx = key[i] >> 10;
+      g2 |= (uint32_t)(pfx > pre22) << i;
+      m2 |= (uint32_t)(pfx == pre22) << i;
+    }
+    m_gt |= g2 & m_on;
+    m_on &= m2;
+  }
+
+  uint32_t m_eq = 0;
+  if (n_on <= (uint32_t)kListCap) {
+    // the keys on the first 22 bits, into the list (positions in any order)
+    for (uint32_t m = m_on; m; m &= m - 1u) {
+      const int i = __ffs(m) - 1;
+      const uint32_t slot = atomicAdd(&n_list, 1u);
+      list_key[slot] = order_key(src[p0 + i]);
+      list_pos[slot] = p0 + i;
+    }
+    __syncthreads();
+    // the rem-th largest listed key (equal keys ranked by position): entry j's rank is the number
+    // of entries above it in (key descending, position ascending) order
+    const uint32_t nl = n_list;
+    if ((uint32_t)tid < nl) {
+      const uint32_t kj = list_key[tid];
+      const int pj = list_pos[tid];
+      uint32_t rank = 0;
+      for (uint32_t e = 0; e < nl; ++e) {
+        const uint32_t ke = list_key[e];
+        rank += (ke > kj || (ke == kj && list_pos[e] < pj)) ? 1u : 0u;
+      }
+      if (rank == rem - 1u) thr_sh = kj;
+    }
+    __syncthreads();
+    const uint32_t thr = thr_sh;
+    if ((uint32_t)tid < nl) {                               // mark the listed keys for their owners
+      const uint32_t kj = list_key[tid];
+      const int pj = list_pos[tid];
+      if (kj > thr) atomicOr(&gt_words[pj / KPT], 1u << (pj % KPT));
+      else if (kj == thr) atomicOr(&eq_words[pj / KPT], 1u << (pj % KPT));
+    }
+    if (tid == 0) {
+      uint32_t above = 0;
+      for (uint32_t e = 0; e < nl; ++e) above += list_key[e] > thr ? 1u : 0u;
+      need_sh = rem - above;                                // keys equal to the k-th that are selected
+    }
+    __syncthreads();
+    m_gt |= gt_words[tid];
+    m_eq = eq_words[tid];
+  } else {
+    // many keys share the first 22 bits: the last 10 bits by one more radix pass
+#pragma unroll
+    for (int i = 0; i < KPT; ++i) hist_inc_if(h3, key[i] & 1023u, (m_on >> i) & 1u);
+    __syncthreads();
+    select_bin<1024>(h3, rem, tots[2], sel);
+    const uint32_t thr = (pre22 << 10) | sel[0];
+    if (tid == 0) need_sh = sel[1];
+    uint32_t g3 = 0, e3 = 0;
+#pragma unroll
+    for (int i = 0; i < KPT; ++i) {
+      g3 |= (uint32_t)(key[i] > thr) << i;
+      e3 |= (uint32_t)(key[i] == thr) << i;
+    }
+    m_gt |= g3 & m_on;
+    m_eq = e3 & m_on;
+    __syncthreads();
+  }
+  const uint32_t need_eq = need_sh;
+
+  // compaction in position order: keys above the k-th, and the first need_eq equal to it
+  uint32_t total;
+  const uint32_t before = block_excl_scan(((uint32_t)__popc(m_gt) << 16) | (uint32_t)__popc(m_eq), tots[3], &total);
+  const uint32_t gb = before >> 16, eb = before & 0xFFFFu;
+  uint32_t m_sel = m_gt;
+  if (m_eq) {                                               // this thread's equal keys ranked eb, eb+1, ...
+    uint32_t m = m_eq;
+    for (uint32_t r = eb; m && r < need_eq; ++r) {
+      m_sel |= m & (0u - m);                                // lowest remaining equal key
+      m &= m - 1u;
+    }
+  }
+  const uint32_t base = gb + min(eb, need_eq);
+  if (sorted) {
+#pragma unroll
+    for (int i = 0; i < KPT; ++i)
+      if ((m_sel >> i) & 1u)
+        sbuf[base + (uint32_t)__popc(m_sel & ((1u << i) - 1u))] = ((uint64_t)(~key[i]) << 32) | (uint32_t)(p0 + i);
+    for (int i = k + tid; i < sort_n; i += kRegThreads) sbuf[i] = ~0ull;
+    sort_and_write(sbuf, sort_n, k, k, out);
+    return;
+  }
+  if (m_sel) {
+#pragma unroll
+    for (int i = 0; i < KPT; ++i)
+      st_shared_if(stage + base + (uint32_t)__popc(m_sel & ((1u << i) - 1u)), p0 + i, (m_sel >> i) & 1u);
+  }
+  __syncthreads();
+  if ((k & 3) == 0) {
+    const int4* s4 = reinterpret_cast<const int4*>(stage);
+    int4* o4 = reinterpret_cast<int4*>(out);
+    for (int i = tid; i < (k >> 2); i += kRegThreads) o4[i] = s4[i];
+  } else {
+    for (int i = tid; i < k; i += kRegThreads) out[i] = stage[i];
+  }
+}
+
+template <int KPT>
+static int launch_topk_regs(const float* scores, int64_t ld, const int32_t* q_pos, const int32_t* kv_len,
+                            int64_t rows, int T, int k, uint32_t flags, int sort_n, int32_t* idx,
+                            cudaStream_t stream, int* status) {
+  const size_t smem = (size_t)kRegFixedWords * 4 +
+                      std::max({(size_t)reg_row_words(KPT) * 4, (size_t)k * 4, (size_t)sort_n * 8});
+  static uint64_t configured[dsa_host::kMaxSetupDevices] = {};
+  static int configured_smem[dsa_host::kMaxSetupDevices] = {};
+  int dev = 0;
+  const bool fresh = dsa_host::needs_setup(configured, &dev);
+  const bool tracked = dev >= 0 && dev < dsa_host::kMaxSetupDevices;
+  if (smem > 48 * 1024 && (fresh || !tracked || (int)smem > configured_smem[dev])) {
+    if (cudaFuncSetAttribute(topk_regs_kernel<KPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return DSA_ERR_CUDA;
+    if (tracked) {
+      if (fresh) configured_smem[dev] = 0;
+      configured_smem[dev] = std::max(configured_smem[dev], (int)smem);
+      dsa_host::mark_setup(configured);
+    }
+  }
+  return dsa_host::launch(topk_regs_kernel<KPT>, dim3((unsigned)rows), dim3(kRegThreads), smem, stream, scores, ld,
+                          q_pos, kv_len, T, k, flags, sort_n, idx, status);
+}
+
 int launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int32_t* kv_len, int B,
                 int T, int k, uint32_t flags, int32_t* idx, cudaStream_t stream, int* status) {
   const int64_t rows = (int64_t)B * T;
@@ -388,6 +730,13 @@ int launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int
   if (flags & DSA_SORTED)
     for (sort_n = 1; sort_n < k; sort_n <<= 1) {
     }
+  // rows of at most 16384 keys: the register-resident kernel, sized to the longest row
+  if (max_row <= kRegThreads * 8)
+    return launch_topk_regs<8>(scores, ld, q_pos, kv_len, rows, T, k, flags, sort_n, idx, stream, status);
+  if (max_row <= kRegThreads * 16)
+    return launch_topk_regs<16>(scores, ld, q_pos, kv_len, rows, T, k, flags, sort_n, idx, stream, status);
+  if (max_row <= kRegThreads * 32)
+    return launch_topk_regs<32>(scores, ld, q_pos, kv_len, rows, T, k, flags, sort_n, idx, stream, status);
   // candidate positions on the first radix digit: a quarter of the longest row (at least 256)
   const int cand_cap = std::max(256, ((max_row + 3) & ~3) / 4 / 4 * 4);
   const size_t smem = (size_t)(kHistBins + ((max_row + 3) & ~3) + cand_cap) * sizeof(uint32_t) + (size_t)sort_n * 8;
