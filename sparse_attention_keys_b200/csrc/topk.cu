@@ -518,7 +518,8 @@ __global__ void __launch_bounds__(kRegThreads, 2) topk_regs_kernel(const float* 
   if (tid == 0) n_list = 0;
 
   // coalesced 16-byte loads (ld is a multiple of 4, so a float4 that starts below n lies in the
-  // row), each written to the transposed layout: position p at word p + 4 (p / 32)
+  // row), converted to order keys and written to the transposed layout: position p at word
+  // p + 4 (p / 32). The row stays there, readable by position, until the output is staged.
   const float* src = scores + row * ld;
   const int n4 = (n + 3) >> 2;
 #pragma unroll
@@ -526,26 +527,28 @@ __global__ void __launch_bounds__(kRegThreads, 2) topk_regs_kernel(const float* 
     const int f = c * kRegThreads + tid;
     if (f < n4) {
       const float4 v = __ldcs(reinterpret_cast<const float4*>(src) + f);
-      *reinterpret_cast<float4*>(region + 4 * f + 4 * (f >> 3)) = v;
+      *reinterpret_cast<uint4*>(region + 4 * f + 4 * (f >> 3)) =
+          make_uint4(order_key(v.x), order_key(v.y), order_key(v.z), order_key(v.w));
     }
   }
   __syncthreads();
+  auto key_at = [&](int pos) -> uint32_t { return region[pos + 4 * (pos >> 5)]; };
   const int p0 = tid * KPT;
   const int nv = max(0, min(KPT, n - p0));
   uint32_t key[KPT];
 #pragma unroll
   for (int c = 0; c < KPT / 4; ++c) {
-    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+    uint4 kk = make_uint4(0u, 0u, 0u, 0u);
     const int pc = p0 + 4 * c;                              // at word pc + 4 (pc / 32)
-    if (4 * c < nv) f = *reinterpret_cast<const float4*>(region + pc + 4 * (pc >> 5));
-    key[4 * c] = order_key(f.x);
-    key[4 * c + 1] = order_key(f.y);
-    key[4 * c + 2] = order_key(f.z);
-    key[4 * c + 3] = order_key(f.w);
+    if (4 * c < nv) kk = *reinterpret_cast<const uint4*>(region + pc + 4 * (pc >> 5));
+    key[4 * c] = kk.x;
+    key[4 * c + 1] = kk.y;
+    key[4 * c + 2] = kk.z;
+    key[4 * c + 3] = kk.w;
   }
-  __syncthreads();                                          // the region is free again
 
   if (n <= k) {                                             // DSA_SORTED with everything selected
+    __syncthreads();                                        // the region becomes the sort buffer
 #pragma unroll
     for (int i = 0; i < KPT; ++i)
       if (i < nv) sbuf[p0 + i] = ((uint64_t)(~key[i]) << 32) | (uint32_t)(p0 + i);
@@ -578,26 +581,22 @@ __global__ void __launch_bounds__(kRegThreads, 2) topk_regs_kernel(const float* 
     m_gt &= valid;
     m_on &= valid;
   }
-  // digit 2 over the keys on digit 1
-  if (m_on) {
-#pragma unroll
-    for (int i = 0; i < KPT; ++i) hist_inc_if(h2, (key[i] >> 10) & 2047u, (m_on >> i) & 1u);
-  }
+  // digit 2 over the keys on digit 1 (a few per thread: read back by position)
+  for (uint32_t m = m_on; m; m &= m - 1u) atomicAdd(&h2[(key_at(p0 + __ffs(m) - 1) >> 10) & 2047u], 1u);
   __syncthreads();
   select_bin<2048>(h2, rem, tots[1], sel);
   const uint32_t pre22 = (d1 << 11) | sel[0];
   rem = sel[1];
   const uint32_t n_on = sel[2];                             // keys on the first 22 bits of the k-th
-  if (m_on) {
-    uint32_t m2 = 0, g2 = 0;
-#pragma unroll
-    for (int i = 0; i < KPT; ++i) {
-      const uint32_t pfx = key[i] >> 10;
-      g2 |= (uint32_t)(pfx > pre22) << i;
+  {
+    uint32_t m2 = 0;
+    for (uint32_t m = m_on; m; m &= m - 1u) {
+      const int i = __ffs(m) - 1;
+      const uint32_t pfx = key_at(p0 + i) >> 10;
+      m_gt |= (uint32_t)(pfx > pre22) << i;
       m2 |= (uint32_t)(pfx == pre22) << i;
     }
-    m_gt |= g2 & m_on;
-    m_on &= m2;
+    m_on = m2;
   }
 
   uint32_t m_eq = 0;
@@ -606,7 +605,7 @@ __global__ void __launch_bounds__(kRegThreads, 2) topk_regs_kernel(const float* 
     for (uint32_t m = m_on; m; m &= m - 1u) {
       const int i = __ffs(m) - 1;
       const uint32_t slot = atomicAdd(&n_list, 1u);
-      list_key[slot] = order_key(src[p0 + i]);
+      list_key[slot] = key_at(p0 + i);
       list_pos[slot] = p0 + i;
     }
     __syncthreads();
