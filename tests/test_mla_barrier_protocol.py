@@ -1,13 +1,20 @@
-"""CPU model of the sparse-MLA exchange kernel's mbarrier protocol for the gathered key data.
+"""CPU model of the sparse-MLA kernel's mbarrier protocol for the gathered key data.
 
-The kernel has two data slots and three Q K^T issuers (issuer e takes pair-tiles e, e+3, ...), so
-the previous user of a slot's barrier phase is another issuer. An mbarrier parity wait returns as
-soon as the phase with that parity is complete relative to the barrier's current phase: on a
-barrier still one phase behind, the wait for parity P returns at once (the "preceding phase" has
-parity P). The model plays random interleavings of gathers completing, gathers being issued (only
-once Q K^T of the pair-tile two earlier has read the slot) and issuers waiting, with that parity
-rule, and checks that no Q K^T starts before its own gather has landed: true with the kernel's
-two-step wait (the slot's previous phase, then its own), false with a single wait.
+The kernel's three Q K^T issuers take the 32-key tiles round robin (issuer e: tiles e, e+3, ...),
+and the gather fills a ring of slots whose "full" barrier a later tile's issuer waits on with a
+parity wait. An mbarrier parity wait returns as soon as the phase with that parity is complete
+relative to the barrier's current phase, so on a barrier still one phase behind, a wait for the
+next phase returns at once. What keeps each issuer's wait on its own phase is the ordering around
+it. The model plays random interleavings of gathers landing (in order), gathers being issued (once
+the tile that last used the slot has been read) and issuers waiting, with that parity rule, and
+reports whether a Q K^T could start before its own tile's data has landed.
+
+- The kernel's configuration: four slots in the ring Q K^T reads for three issuers. A slot's previous
+  user is tile j - 4, which landed before tile j - 3, the issuer's own previous tile, whose data it
+  has already waited for: never early, with or without the issuer's wait for P V of tile j - 3.
+- Two slots with three issuers and a single wait (a layout tried while developing the kernel) does
+  start early; waiting first for the slot's previous phase closes it. The model shows the hazard is
+  real, so the slot count and the ordering are load-bearing.
 """
 import random
 
@@ -18,9 +25,9 @@ def _parity_complete(completed_phases: int, phase: int) -> bool:
     return (completed_phases & 1) != (phase & 1)
 
 
-def _run(ntiles: int, seed: int, two_step: bool) -> bool:
+def _run(ntiles, seed, slots, two_step=False, order_after_pv=True) -> bool:
     rnd = random.Random(seed)
-    kv_full = [0, 0]                       # completed phases per slot barrier
+    full = [0] * slots                     # completed phases per slot barrier
     issued = landed = 0                    # gathers issued / landed (they land in order)
     qk_done = [False] * ntiles
     stage = {}
@@ -30,25 +37,27 @@ def _run(ntiles: int, seed: int, two_step: bool) -> bool:
             return True
         r = rnd.random()
         if r < 0.3:
-            if issued < ntiles and (issued < 2 or qk_done[issued - 2]):
+            if issued < ntiles and (issued < slots or qk_done[issued - slots]):
                 issued += 1
         elif r < 0.6:
             if landed < issued:
-                kv_full[landed % 2] += 1
+                full[landed % slots] += 1
                 landed += 1
         else:
             e = rnd.randrange(3)
             if not todo[e]:
                 continue
             j = todo[e][0]
-            if j >= 3 and not qk_done[j - 3]:          # the issuer's wait for P V of pair-tile j - 3
+            # the issuer first waits for P V of tile j - 3 (modelled as that tile's Q K^T, which
+            # P V follows), whose data landed before tile j - 2's
+            if order_after_pv and j >= 3 and not qk_done[j - 3]:
                 continue
-            s = j % 2
-            if two_step and j >= 2 and stage.get(j, 0) == 0:
-                if _parity_complete(kv_full[s], j // 2 - 1):
+            s = j % slots
+            if two_step and j >= slots and stage.get(j, 0) == 0:
+                if _parity_complete(full[s], j // slots - 1):
                     stage[j] = 1
                 continue
-            if _parity_complete(kv_full[s], j // 2):
+            if _parity_complete(full[s], j // slots):
                 if landed <= j:                        # Q K^T would read a slot still being filled
                     return False
                 qk_done[j] = True
@@ -56,10 +65,14 @@ def _run(ntiles: int, seed: int, two_step: bool) -> bool:
     return True
 
 
-def test_two_step_wait_never_reads_early():
-    assert all(_run(n, seed, two_step=True) for n in range(1, 12) for seed in range(200))
+def test_kernel_configuration_never_reads_early():
+    assert all(_run(n, seed, slots=4) for n in range(1, 14) for seed in range(200))
 
 
-def test_single_wait_would_read_early():
-    # the model does reach the hazard the two-step wait removes
-    assert not all(_run(n, seed, two_step=False) for n in range(1, 12) for seed in range(200))
+def test_two_slots_need_the_two_step_wait():
+    assert not all(_run(n, seed, slots=2) for n in range(1, 12) for seed in range(200))
+    assert all(_run(n, seed, slots=2, two_step=True) for n in range(1, 12) for seed in range(200))
+
+
+def test_four_slots_are_ordered_by_the_issuers_own_waits():
+    assert all(_run(n, seed, slots=4, order_after_pv=False) for n in range(1, 14) for seed in range(200))
