@@ -89,13 +89,14 @@ __device__ void select_digit(const uint32_t* hist, int nb, uint32_t remaining, u
   __syncthreads();
 }
 
-// Ascending bitonic sort of buf[0, n) (n a power of two) by the CTA, then out[i] = the position in
-// the low word of buf[i] for i < count, and -1 for count <= i < k.
+// Ascending bitonic sort of buf[0, n) (n a power of two) by the CTA of NT threads, then out[i] = the
+// position in the low word of buf[i] for i < count, and -1 for count <= i < k.
+template <int NT = kTopkThreads>
 __device__ void sort_and_write(uint64_t* buf, int n, int count, int k, int32_t* out) {
   __syncthreads();
   for (int size = 2; size <= n; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < (n >> 1); i += kTopkThreads) {
+      for (int i = threadIdx.x; i < (n >> 1); i += NT) {
         const int lo = 2 * stride * (i / stride) + (i % stride), hi = lo + stride;
         const bool up = (lo & size) == 0;
         const uint64_t a = buf[lo], b = buf[hi];
@@ -104,7 +105,7 @@ __device__ void sort_and_write(uint64_t* buf, int n, int count, int k, int32_t* 
       __syncthreads();
     }
   }
-  for (int i = threadIdx.x; i < k; i += kTopkThreads) out[i] = i < count ? (int32_t)(uint32_t)buf[i] : -1;
+  for (int i = threadIdx.x; i < k; i += NT) out[i] = i < count ? (int32_t)(uint32_t)buf[i] : -1;
 }
 
 }  // namespace
@@ -394,14 +395,14 @@ __global__ void __launch_bounds__(kTopkThreads, 4) topk_kernel(const float* __re
 //   - one block scan of packed (above, equal) counts orders the selection by position (each thread's
 //     run is contiguous), and the positions are staged in shared memory and leave in coalesced
 //     16-byte stores.
-constexpr int kRegThreads = 512;
-constexpr int kRegWarps = kRegThreads / 32;
+// NT threads per CTA: 512 (two CTAs per SM, for launches with many rows) or 1024 (one per SM, for
+// launches with fewer rows than SMs, where each row's latency is the launch's).
 constexpr int kRegRowMax = 16384;
 constexpr int kListCap = 256;                               // keys on the first 22 bits picked directly
-// shared words: h1 (2048) | h2 (2048) | h3 (1024) | above / equal masks (512 + 512) | list keys,
+// shared words: h1 (2048) | h2 (2048) | h3 (1024) | above / equal masks (NT + NT) | list keys,
 // positions (kListCap each) | a region for the transposed row, later the staged output
-constexpr int kRegFixedWords = 2048 + 2048 + 1024 + 2 * kRegThreads + 2 * kListCap;
-__host__ __device__ constexpr int reg_row_words(int kpt) { return kpt * kRegThreads / 32 * 36; }
+__host__ __device__ constexpr int reg_fixed_words(int nt) { return 2048 + 2048 + 1024 + 2 * nt + 2 * kListCap; }
+__host__ __device__ constexpr int reg_row_words(int kpt, int nt) { return kpt * nt / 32 * 36; }
 
 // hist[bin] += 1 when `pred`, as one predicated shared-memory reduction (no branch, no return value).
 __device__ __forceinline__ void hist_inc_if(uint32_t* hist, uint32_t bin, bool pred) {
@@ -418,10 +419,12 @@ __device__ __forceinline__ void st_shared_if(int32_t* dst, int32_t v, bool pred)
                : "memory");
 }
 
-// Exclusive prefix, in thread order, of one value per thread of the CTA; *total gets the sum.
-// One barrier; `tot` (kRegWarps words) is written before it and read after it, so a call must not
-// reuse the `tot` of the previous call before another barrier.
+// Exclusive prefix, in thread order, of one value per thread of the CTA (NT threads); *total gets
+// the sum. One barrier; `tot` (NT / 32 words) is written before it and read after it, so a call
+// must not reuse the `tot` of the previous call before another barrier.
+template <int NT>
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tot, uint32_t* total) {
+  constexpr int kRegWarps = NT / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t incl = v;
 #pragma unroll
@@ -446,9 +449,10 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tot, u
 // The bin holding the target-th largest histogrammed key (bins scanned from the top; thread t
 // owns bins NB-1-t*C .. NB-C-t*C). Writes the bin to sel[0], the target's rank inside it (1-based)
 // to sel[1] and the bin's count to sel[2]; ends with a barrier.
-template <int NB>
+template <int NB, int NT>
 __device__ __forceinline__ void select_bin(const uint32_t* hist, uint32_t target, uint32_t* tot, uint32_t* sel) {
-  constexpr int C = NB / kRegThreads;
+  constexpr int C = NB / NT;
+  static_assert(C >= 1, "bins per thread");
   const int top = NB - 1 - (int)threadIdx.x * C;
   uint32_t h[C];
   uint32_t local = 0;
@@ -458,7 +462,7 @@ __device__ __forceinline__ void select_bin(const uint32_t* hist, uint32_t target
     local += h[j];
   }
   uint32_t total;
-  uint32_t before = block_excl_scan(local, tot, &total);
+  uint32_t before = block_excl_scan<NT>(local, tot, &total);
   if (before < target && target <= before + local) {
 #pragma unroll
     for (int j = 0; j < C; ++j) {
@@ -474,13 +478,14 @@ __device__ __forceinline__ void select_bin(const uint32_t* hist, uint32_t target
   __syncthreads();
 }
 
-template <int KPT>
-__global__ void __launch_bounds__(kRegThreads, 2) topk_regs_kernel(const float* __restrict__ scores, int64_t ld,
+template <int KPT, int NT>
+__global__ void __launch_bounds__(NT, 1024 / NT) topk_regs_kernel(const float* __restrict__ scores, int64_t ld,
                                                                    const int32_t* __restrict__ q_pos,
                                                                    const int32_t* __restrict__ kv_len, int T, int k,
                                                                    uint32_t flags, int sort_n,
                                                                    int32_t* __restrict__ idx, int* status) {
-  static_assert(KPT % 4 == 0 && KPT <= 32 && KPT * kRegThreads <= kRegRowMax, "keys per thread");
+  static_assert(KPT % 4 == 0 && KPT <= 32 && KPT * NT <= kRegRowMax, "keys per thread");
+  constexpr int kRegThreads = NT, kRegWarps = NT / 32, kRegFixedWords = reg_fixed_words(NT);
   extern __shared__ __align__(16) uint32_t smem[];
   uint32_t* h1 = smem;                                      // 2048 bins: key bits 31..21
   uint32_t* h2 = smem + 2048;                               // 2048 bins: key bits 20..10
@@ -553,7 +558,7 @@ __global__ void __launch_bounds__(kRegThreads, 2) topk_regs_kernel(const float* 
     for (int i = 0; i < KPT; ++i)
       if (i < nv) sbuf[p0 + i] = ((uint64_t)(~key[i]) << 32) | (uint32_t)(p0 + i);
     for (int i = n + tid; i < sort_n; i += kRegThreads) sbuf[i] = ~0ull;
-    sort_and_write(sbuf, sort_n, n, k, out);
+    sort_and_write<NT>(sbuf, sort_n, n, k, out);
     return;
   }
 
@@ -567,7 +572,7 @@ __global__ void __launch_bounds__(kRegThreads, 2) topk_regs_kernel(const float* 
     for (int i = 0; i < KPT; ++i) hist_inc_if(h1, key[i] >> 21, i < nv);
   }
   __syncthreads();
-  select_bin<2048>(h1, (uint32_t)k, tots[0], sel);
+  select_bin<2048, NT>(h1, (uint32_t)k, tots[0], sel);
   const uint32_t d1 = sel[0];
   uint32_t rem = sel[1];
   uint32_t m_gt = 0, m_on = 0;                              // above the k-th key / still undecided
@@ -584,7 +589,7 @@ __global__ void __launch_bounds__(kRegThreads, 2) topk_regs_kernel(const float* 
   // digit 2 over the keys on digit 1 (a few per thread: read back by position)
   for (uint32_t m = m_on; m; m &= m - 1u) atomicAdd(&h2[(key_at(p0 + __ffs(m) - 1) >> 10) & 2047u], 1u);
   __syncthreads();
-  select_bin<2048>(h2, rem, tots[1], sel);
+  select_bin<2048, NT>(h2, rem, tots[1], sel);
   const uint32_t pre22 = (d1 << 11) | sel[0];
   rem = sel[1];
   const uint32_t n_on = sel[2];                             // keys on the first 22 bits of the k-th
@@ -643,7 +648,7 @@ __global__ void __launch_bounds__(kRegThreads, 2) topk_regs_kernel(const float* 
 #pragma unroll
     for (int i = 0; i < KPT; ++i) hist_inc_if(h3, key[i] & 1023u, (m_on >> i) & 1u);
     __syncthreads();
-    select_bin<1024>(h3, rem, tots[2], sel);
+    select_bin<1024, NT>(h3, rem, tots[2], sel);
     const uint32_t thr = (pre22 << 10) | sel[0];
     if (tid == 0) need_sh = sel[1];
     uint32_t g3 = 0, e3 = 0;
@@ -660,7 +665,8 @@ __global__ void __launch_bounds__(kRegThreads, 2) topk_regs_kernel(const float* 
 
   // compaction in position order: keys above the k-th, and the first need_eq equal to it
   uint32_t total;
-  const uint32_t before = block_excl_scan(((uint32_t)__popc(m_gt) << 16) | (uint32_t)__popc(m_eq), tots[3], &total);
+  const uint32_t before =
+      block_excl_scan<NT>(((uint32_t)__popc(m_gt) << 16) | (uint32_t)__popc(m_eq), tots[3], &total);
   const uint32_t gb = before >> 16, eb = before & 0xFFFFu;
   uint32_t m_sel = m_gt;
   if (m_eq) {                                               // this thread's equal keys ranked eb, eb+1, ...
@@ -677,7 +683,7 @@ __global__ void __launch_bounds__(kRegThreads, 2) topk_regs_kernel(const float* 
       if ((m_sel >> i) & 1u)
         sbuf[base + (uint32_t)__popc(m_sel & ((1u << i) - 1u))] = ((uint64_t)(~key[i]) << 32) | (uint32_t)(p0 + i);
     for (int i = k + tid; i < sort_n; i += kRegThreads) sbuf[i] = ~0ull;
-    sort_and_write(sbuf, sort_n, k, k, out);
+    sort_and_write<NT>(sbuf, sort_n, k, k, out);
     return;
   }
   if (m_sel) {
@@ -695,19 +701,19 @@ __global__ void __launch_bounds__(kRegThreads, 2) topk_regs_kernel(const float* 
   }
 }
 
-template <int KPT>
+template <int KPT, int NT>
 static int launch_topk_regs(const float* scores, int64_t ld, const int32_t* q_pos, const int32_t* kv_len,
                             int64_t rows, int T, int k, uint32_t flags, int sort_n, int32_t* idx,
                             cudaStream_t stream, int* status) {
-  const size_t smem = (size_t)kRegFixedWords * 4 +
-                      std::max({(size_t)reg_row_words(KPT) * 4, (size_t)k * 4, (size_t)sort_n * 8});
+  const size_t smem = (size_t)reg_fixed_words(NT) * 4 +
+                      std::max({(size_t)reg_row_words(KPT, NT) * 4, (size_t)k * 4, (size_t)sort_n * 8});
   static uint64_t configured[dsa_host::kMaxSetupDevices] = {};
   static int configured_smem[dsa_host::kMaxSetupDevices] = {};
   int dev = 0;
   const bool fresh = dsa_host::needs_setup(configured, &dev);
   const bool tracked = dev >= 0 && dev < dsa_host::kMaxSetupDevices;
   if (smem > 48 * 1024 && (fresh || !tracked || (int)smem > configured_smem[dev])) {
-    if (cudaFuncSetAttribute(topk_regs_kernel<KPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+    if (cudaFuncSetAttribute(topk_regs_kernel<KPT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
       return DSA_ERR_CUDA;
     if (tracked) {
@@ -716,7 +722,7 @@ static int launch_topk_regs(const float* scores, int64_t ld, const int32_t* q_po
       dsa_host::mark_setup(configured);
     }
   }
-  return dsa_host::launch(topk_regs_kernel<KPT>, dim3((unsigned)rows), dim3(kRegThreads), smem, stream, scores, ld,
+  return dsa_host::launch(topk_regs_kernel<KPT, NT>, dim3((unsigned)rows), dim3(NT), smem, stream, scores, ld,
                           q_pos, kv_len, T, k, flags, sort_n, idx, status);
 }
 
@@ -729,13 +735,19 @@ int launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int
   if (flags & DSA_SORTED)
     for (sort_n = 1; sort_n < k; sort_n <<= 1) {
     }
-  // rows of at most 16384 keys: the register-resident kernel, sized to the longest row
-  if (max_row <= kRegThreads * 8)
-    return launch_topk_regs<8>(scores, ld, q_pos, kv_len, rows, T, k, flags, sort_n, idx, stream, status);
-  if (max_row <= kRegThreads * 16)
-    return launch_topk_regs<16>(scores, ld, q_pos, kv_len, rows, T, k, flags, sort_n, idx, stream, status);
-  if (max_row <= kRegThreads * 32)
-    return launch_topk_regs<32>(scores, ld, q_pos, kv_len, rows, T, k, flags, sort_n, idx, stream, status);
+  // rows of at most 16384 keys: the register-resident kernel, sized to the longest row; 1024 threads
+  // per row when the launch has fewer rows than SMs (each row's latency is then the launch's)
+  if (rows < dsa_host::device_sm_count() && max_row <= 1024 * 16) {
+    if (max_row <= 1024 * 8)
+      return launch_topk_regs<8, 1024>(scores, ld, q_pos, kv_len, rows, T, k, flags, sort_n, idx, stream, status);
+    return launch_topk_regs<16, 1024>(scores, ld, q_pos, kv_len, rows, T, k, flags, sort_n, idx, stream, status);
+  }
+  if (max_row <= 512 * 8)
+    return launch_topk_regs<8, 512>(scores, ld, q_pos, kv_len, rows, T, k, flags, sort_n, idx, stream, status);
+  if (max_row <= 512 * 16)
+    return launch_topk_regs<16, 512>(scores, ld, q_pos, kv_len, rows, T, k, flags, sort_n, idx, stream, status);
+  if (max_row <= 512 * 32)
+    return launch_topk_regs<32, 512>(scores, ld, q_pos, kv_len, rows, T, k, flags, sort_n, idx, stream, status);
   // candidate positions on the first radix digit: a quarter of the longest row (at least 256)
   const int cand_cap = std::max(256, ((max_row + 3) & ~3) / 4 / 4 * 4);
   const size_t smem = (size_t)(kHistBins + ((max_row + 3) & ~3) + cand_cap) * sizeof(uint32_t) + (size_t)sort_n * 8;
