@@ -556,7 +556,7 @@ def run_ours(args, rank, world, local_rank):
         line["mla_producers"] = producer_rooflines(producers, peaks)
     if paged is not None:
         line["paged_caches"] = paged_rooflines(paged, units, peaks, args)
-    extras = [w for w in (args.extra or "").split(",") if w and w != args.workload]
+    extras = [w for w in (args.extra or "").split(",") if w and w not in (args.workload, "none")]
     if world == 1 and extras:
         del st, slots
         torch.cuda.empty_cache()
@@ -907,7 +907,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="decode_b64", choices=sorted(DI.WORKLOADS))
     ap.add_argument("--extra", default="prefill_16384",
-                    help="comma-separated workloads also timed (device time, one GPU) in the same run; '' for none")
+                    help="comma-separated workloads also timed (device time, one GPU) in the same run; '' or 'none' for none")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-producers", action="store_true", help="skip timing the MLA producer calls")
