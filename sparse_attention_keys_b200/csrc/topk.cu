@@ -519,22 +519,26 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_regs_kernel(const float* _
     for (int i = tid; i < k; i += kRegThreads) out[i] = -1;
     return;
   }
-  for (int i = tid; i < kRegFixedWords - 2 * kListCap; i += kRegThreads) smem[i] = 0u;
-  if (tid == 0) n_list = 0;
-
   // coalesced 16-byte loads (ld is a multiple of 4, so a float4 that starts below n lies in the
   // row), converted to order keys and written to the transposed layout: position p at word
   // p + 4 (p / 32). The row stays there, readable by position, until the output is staged.
+  // All of a thread's loads are issued before the first store, so that their latencies overlap.
   const float* src = scores + row * ld;
   const int n4 = (n + 3) >> 2;
+  float4 ld4[KPT / 4];
 #pragma unroll
   for (int c = 0; c < KPT / 4; ++c) {
     const int f = c * kRegThreads + tid;
-    if (f < n4) {
-      const float4 v = __ldcs(reinterpret_cast<const float4*>(src) + f);
+    ld4[c] = f < n4 ? __ldcs(reinterpret_cast<const float4*>(src) + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int i = tid; i < kRegFixedWords - 2 * kListCap; i += kRegThreads) smem[i] = 0u;   // while they fly
+  if (tid == 0) n_list = 0;
+#pragma unroll
+  for (int c = 0; c < KPT / 4; ++c) {
+    const int f = c * kRegThreads + tid;
+    if (f < n4)
       *reinterpret_cast<uint4*>(region + 4 * f + 4 * (f >> 3)) =
-          make_uint4(order_key(v.x), order_key(v.y), order_key(v.z), order_key(v.w));
-    }
+          make_uint4(order_key(ld4[c].x), order_key(ld4[c].y), order_key(ld4[c].z), order_key(ld4[c].w));
   }
   __syncthreads();
   auto key_at = [&](int pos) -> uint32_t { return region[pos + 4 * (pos >> 5)]; };
