@@ -343,6 +343,20 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 // ------------------------------------------------------------------- programmatic dependent launch
 // Kernels are launched so that the next kernel on the stream may start while this one finishes.
+// (a0, a1) * (b0, b1) + c, lane by lane, as one paired fp32 FMA (each lane rounds as fmaf);
+// c and the result hold lane 0 in the low word.
+__device__ __forceinline__ uint64_t fma_f32x2(float a0, float a1, float b0, float b1, uint64_t c) {
+  uint64_t d;
+  asm("{\n\t.reg .b64 a, b;\n\tmov.b64 a, {%1, %2};\n\tmov.b64 b, {%3, %4};\n\t"
+      "fma.rn.f32x2 %0, a, b, %5;\n\t}"
+      : "=l"(d)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "l"(c));
+  return d;
+}
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
 // grid_dep_wait: block until the preceding kernel on the stream has completed and its writes are
 // visible (a no-op when the kernel was launched without the attribute). Every kernel calls it
 // before reading a buffer an earlier kernel of the stream writes, and before its own writes.

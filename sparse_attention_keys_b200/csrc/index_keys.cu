@@ -47,13 +47,15 @@ __global__ void __launch_bounds__(256) index_keys_kernel(const In* __restrict__ 
   if (blk >= blocks) return;
   const int64_t row = blk / heads;
   const int head = (int)(blk - row * heads);
+  // the three loads that do not depend on the position go out together, before the RoPE table
+  // load that does (a warp's only work is this one block, so its latency is the chain of loads)
+  const float4 v4 = load4<In>(x, blk, lane);
+  const int64_t dst = dst_row ? __ldg(dst_row + row) : -1;
   const int p = pos[row];
   if (p < 0 || p >= max_pos) {
     if (lane == 0) set_status(status, DSA_ERR_DEVICE_BOUNDS);
     return;
   }
-
-  const float4 v4 = load4<In>(x, blk, lane);
   float v[4] = {v4.x, v4.y, v4.z, v4.w};
 
   // RoPE on features 0..63: lanes 0-7 hold the first halves a_j (j = 4*lane + i), lanes 8-15
@@ -111,7 +113,7 @@ __global__ void __launch_bounds__(256) index_keys_kernel(const In* __restrict__ 
                                __NV_SATFINITE, __NV_E4M3);
   const uint32_t packed = (uint32_t)lo | ((uint32_t)hi << 16);
 
-  const int64_t out_blk = dst_row ? dst_row[row] * heads + head : blk;
+  const int64_t out_blk = dst_row ? dst * heads + head : blk;
   reinterpret_cast<uint32_t*>(out_fp8 + out_blk * 128)[lane] = packed;
   if (lane == 0) out_scale[out_blk] = scale;
 }

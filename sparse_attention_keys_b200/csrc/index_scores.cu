@@ -246,21 +246,25 @@ __global__ void __launch_bounds__(threads_for(NQ), 1)
           tmem_ld32(taddr, r0);
           tmem_ld32(taddr + 32, r1);
           tmem_ld_wait();
-          float acc[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+          // eight partial sums, as four packed pairs: head j accumulates into sum j mod 8 with one
+          // lane of a paired fma.rn.f32x2 (each lane rounds exactly as fmaf)
+          uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
           const float4* w4 = reinterpret_cast<const float4*>(&wq[q][0]);
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj) {
             const float4 wa = w4[2 * jj], wb = w4[2 * jj + 1];
             const float ww[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+            for (int u = 0; u < 8; u += 2) {
               const int j = 8 * jj + u;
-              const float v = __uint_as_float(j < 32 ? r0[j] : r1[j - 32]);
-              acc[u] = fmaf(ww[u], fmaxf(v, 0.f), acc[u]);
+              const float v0 = fmaxf(__uint_as_float(j < 32 ? r0[j] : r1[j - 32]), 0.f);
+              const float v1 = fmaxf(__uint_as_float(j + 1 < 32 ? r0[j + 1] : r1[j + 1 - 32]), 0.f);
+              acc2[u / 2] = fma_f32x2(ww[u], ww[u + 1], v0, v1, acc2[u / 2]);
             }
           }
+          float acc[8];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) unpack_f32x2(acc2[u], acc[2 * u], acc[2 * u + 1]);
           const float tot = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
           const int t = t0 + q;
           if (t < p.T) {
