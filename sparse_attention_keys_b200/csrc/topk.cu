@@ -690,7 +690,10 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_regs_kernel(const float* _
     sort_and_write<NT>(sbuf, sort_n, k, k, out);
     return;
   }
-  if (m_sel) {
+  if (4 * k <= n) {            // a sparse selection (row-uniform): visit only the selected keys
+    uint32_t r = base;
+    for (uint32_t m = m_sel; m; m &= m - 1u) stage[r++] = p0 + __ffs(m) - 1;
+  } else if (m_sel) {
 #pragma unroll
     for (int i = 0; i < KPT; ++i)
       st_shared_if(stage + base + (uint32_t)__popc(m_sel & ((1u << i) - 1u)), p0 + i, (m_sel >> i) & 1u);
