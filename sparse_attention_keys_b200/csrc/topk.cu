@@ -608,8 +608,12 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_regs_kernel(const float* _
     m_on = m2;
   }
 
-  uint32_t m_eq = 0;
-  if (n_on <= (uint32_t)kListCap) {
+  uint32_t m_eq = 0, need_eq = 0;
+  if (rem == n_on) {
+    // the k-th key is the smallest on its first 22 bits (always so when it is alone there): every
+    // key on them is selected, with no tie to break
+    m_gt |= m_on;
+  } else if (n_on <= (uint32_t)kListCap) {
     // the keys on the first 22 bits, into the list (positions in any order)
     for (uint32_t m = m_on; m; m &= m - 1u) {
       const int i = __ffs(m) - 1;
@@ -647,6 +651,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_regs_kernel(const float* _
     __syncthreads();
     m_gt |= gt_words[tid];
     m_eq = eq_words[tid];
+    need_eq = need_sh;
   } else {
     // many keys share the first 22 bits: the last 10 bits by one more radix pass
 #pragma unroll
@@ -664,8 +669,8 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_regs_kernel(const float* _
     m_gt |= g3 & m_on;
     m_eq = e3 & m_on;
     __syncthreads();
+    need_eq = need_sh;
   }
-  const uint32_t need_eq = need_sh;
 
   // compaction in position order: keys above the k-th, and the first need_eq equal to it
   uint32_t total;
