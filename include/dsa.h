@@ -160,6 +160,26 @@ DSA_API int dsa_topk(const float* scores, int64_t ld, const int32_t* q_pos, cons
              int B, int T, int k, uint32_t flags, int32_t* idx, dsa_stream_t stream);
 
 /*
+ * dsa_index_topk - the decode indexer fused with its top-k: the selection dsa_index_scores
+ * followed by dsa_topk would make (fp8_index, the causal mask and topk(min(index_topk, end_pos)) of
+ * Indexer.forward; [dense] S^I and top_2048), in one launch, without writing the scores anywhere.
+ *
+ *   q8, q_scale, w, k8, k_scale, q_pos, kv_len: as for dsa_index_scores (dense K-cache)
+ *   idx int32 [B][T][k] (output): the min(k, n_valid) visible positions with the largest scores,
+ *   in ascending order, then -1 up to k; ties go to the smaller position.
+ * The scores are the fp32 values dsa_index_scores computes, bit for bit, so idx equals
+ * dsa_topk(dsa_index_scores(...)) exactly. Each query's key tiles are scored by a thread-block
+ * cluster of up to 8 CTAs that merge their radix histograms in distributed shared memory.
+ * Constraints: as dsa_index_scores, plus 1 <= k and S_max <= 32768 (at most 32 key tiles of 128
+ * per CTA of the cluster). No workspace; flags are reserved (0).
+ */
+DSA_API int dsa_index_topk(const uint8_t* q8, const float* q_scale, const float* w,
+                   const uint8_t* k8, const float* k_scale,
+                   const int32_t* q_pos, const int32_t* kv_len,
+                   int B, int T, int S_max, float softmax_scale, int k, uint32_t flags,
+                   int32_t* idx, dsa_stream_t stream);
+
+/*
  * dsa_sparse_mla - sparse MQA-style latent attention over the selected positions
  * ([sim] MQA decode: scores over the latent and rotary parts, index mask, softmax, latent-
  * weighted sum; [dense] sparse attention steps S' = S m^2 / sqrt 192; the MLA prefill excerpt

@@ -14,7 +14,7 @@ import torch
 
 __all__ = [
     "DsaError", "lib", "lib_path", "DSA_HADAMARD", "DSA_FILL_MASKED", "DSA_SORTED", "DSA_F32", "DSA_BF16", "INDEXER_SOFTMAX_SCALE",
-    "MLA_SOFTMAX_SCALE", "dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk",
+    "MLA_SOFTMAX_SCALE", "dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk", "dsa_index_topk",
     "dsa_sparse_mla", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_noalloc", "dsa_sparse_mla_heads",
     "dsa_sparse_mla_heads_workspace_size",
     "dsa_index_scores_paged", "dsa_sparse_mla_paged", "dsa_mla_q_absorb", "dsa_mla_kv_entry",
@@ -63,6 +63,7 @@ def _load():
     L.dsa_index_keys.argtypes = [vp, i32, i64, i32, vp, vp, i32, u32, vp, vp, vp, vp]
     L.dsa_index_scores.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, f32, vp, i64, u32, vp]
     L.dsa_topk.argtypes = [vp, i64, vp, vp, i32, i32, i32, u32, vp, vp]
+    L.dsa_index_topk.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, f32, i32, u32, vp, vp]
     L.dsa_sparse_mla.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
     L.dsa_sparse_mla_workspace_size.argtypes = [i32, i32, i32]
     L.dsa_sparse_mla_heads.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
@@ -85,7 +86,7 @@ def _load():
     L.dsa_status_string.restype = ctypes.c_char_p
     L.dsa_device_supported.argtypes = []
     L.dsa_version.restype = ctypes.c_char_p
-    for f in ("dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk", "dsa_sparse_mla",
+    for f in ("dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk", "dsa_index_topk", "dsa_sparse_mla",
               "dsa_sparse_mla_heads",
               "dsa_sparse_mla_noalloc", "dsa_get_device_status", "dsa_get_error_detail",
               "dsa_selftest_wait_timeout", "dsa_device_supported"):
@@ -197,6 +198,38 @@ def dsa_index_scores(q8, q_scale, w, k8, k_scale, q_pos, kv_len, softmax_scale: 
                                _stream(stream))
     _check(rc, "dsa_index_scores")
     return scores
+
+
+def dsa_index_topk(q8, q_scale, w, k8, k_scale, q_pos, kv_len, k: int,
+                   softmax_scale: float = INDEXER_SOFTMAX_SCALE, idx=None, stream=None):
+    """The decode indexer fused with its top-k: the same idx int32 [B,T,k] as
+    dsa_topk(dsa_index_scores(...), q_pos, kv_len, k), in one launch and with no scores buffer.
+    Inputs as dsa_index_scores (dense K-cache, S <= 32768)."""
+    for t, dt, n in ((q8, torch.uint8, "q8"), (q_scale, torch.float32, "q_scale"), (w, torch.float32, "w"),
+                     (k8, torch.uint8, "k8"), (k_scale, torch.float32, "k_scale"), (q_pos, torch.int32, "q_pos"),
+                     (kv_len, torch.int32, "kv_len")):
+        _need(t, dt, n)
+    B, T = q8.shape[0], q8.shape[1]
+    S = k8.shape[1]
+    if tuple(q8.shape[2:]) != (64, 128) or tuple(q_scale.shape) != (B, T, 64) or tuple(w.shape) != (B, T, 64):
+        raise ValueError("q8 must be [B, T, 64, 128] with q_scale and w [B, T, 64]")
+    if k8.dim() != 3 or k8.shape[0] != B or k8.shape[2] != 128 or tuple(k_scale.shape) != (B, S):
+        raise ValueError("k8 must be [B, S, 128] with k_scale [B, S]")
+    if tuple(q_pos.shape) != (B, T) or tuple(kv_len.shape) != (B,):
+        raise ValueError("q_pos must be [B, T] and kv_len [B]")
+    if idx is None:
+        idx = torch.empty((B, T, int(k)), dtype=torch.int32, device=q8.device)
+    _need(idx, torch.int32, "idx")
+    if tuple(idx.shape) != (B, T, int(k)):
+        raise ValueError(f"idx must be [{B}, {T}, {int(k)}]")
+    for t, n in ((q_scale, "q_scale"), (w, "w"), (k8, "k8"), (k_scale, "k_scale"), (q_pos, "q_pos"),
+                 (kv_len, "kv_len"), (idx, "idx")):
+        if t.device != q8.device:
+            raise ValueError(f"{n} is on {t.device}, q8 on {q8.device}: all tensors must be on one device")
+    rc = _lib.dsa_index_topk(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale), _ptr(q_pos), _ptr(kv_len),
+                             B, T, S, float(softmax_scale), int(k), 0, _ptr(idx), _stream(stream))
+    _check(rc, "dsa_index_topk")
+    return idx
 
 
 def dsa_index_scores_paged(q8, q_scale, w, k8_pool, k_scale_pool, block_table, page_size: int, q_pos, kv_len,

@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libdsa.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["dsa_abi.cu", "index_keys.cu", "index_scores.cu", "topk.cu", "sparse_mla.cu", "sparse_mla_noalloc.cu", "mla_absorb.cu"]
+SOURCES = ["dsa_abi.cu", "index_keys.cu", "index_scores.cu", "index_topk.cu", "topk.cu", "sparse_mla.cu", "sparse_mla_noalloc.cu", "mla_absorb.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
               "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

@@ -295,6 +295,26 @@ int dsa_index_scores(const uint8_t* q8, const float* q_scale, const float* w, co
                                   scores, ld, flags, (cudaStream_t)stream, status);
 }
 
+int dsa_index_topk(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8,
+                   const float* k_scale, const int32_t* q_pos, const int32_t* kv_len, int B, int T, int S_max,
+                   float softmax_scale, int k, uint32_t flags, int32_t* idx, dsa_stream_t stream) {
+  if (B < 1 || T < 1 || S_max < 1 || S_max > DSA_TOPK_MAX_ROW || k < 1 || flags != 0 || !(softmax_scale > 0.f) ||
+      !isfinite(softmax_scale))
+    return DSA_ERR_INVALID_ARG;
+  if ((int64_t)B * T * 64 > 0x7fffffffLL || (int64_t)B * S_max > 0x7fffffffLL ||
+      (int64_t)B * T * 8 > 0x7fffffffLL)
+    return DSA_ERR_INVALID_ARG;
+  if (!q8 || !q_scale || !w || !k8 || !k_scale || !q_pos || !kv_len || !idx) return DSA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q8, q_scale, w, k8, k_scale, q_pos, kv_len, idx};
+  for (const void* p : ptrs)
+    if (!dsa_host::aligned16(p)) return DSA_ERR_INVALID_ARG;
+  int* status;
+  int rc = prologue(&status);
+  if (rc != DSA_OK) return rc;
+  return dsa::launch_index_topk(q8, q_scale, w, k8, k_scale, q_pos, kv_len, B, T, S_max, softmax_scale, k, idx,
+                                (cudaStream_t)stream, status);
+}
+
 int dsa_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int32_t* kv_len, int B, int T,
              int k, uint32_t flags, int32_t* idx, dsa_stream_t stream) {
   if (B < 1 || T < 1 || k < 1 || ld < 1 || (ld & 3) != 0 || (flags & ~DSA_SORTED) != 0) return DSA_ERR_INVALID_ARG;

@@ -11,6 +11,9 @@ int launch_index_keys(const void* x, int x_dtype, int64_t rows, int heads, const
                       const float* rope_cs, int max_pos, uint32_t flags, uint8_t* out_fp8,
                       float* out_scale, const int64_t* dst_row, cudaStream_t stream, int* status);
 
+int launch_index_topk(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8,
+                      const float* k_scale, const int32_t* q_pos, const int32_t* kv_len, int B, int T,
+                      int S_max, float softmax_scale, int k, int32_t* idx, cudaStream_t stream, int* status);
 int launch_index_scores(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8,
                         const float* k_scale, const int32_t* q_pos, const int32_t* kv_len, int B,
                         int T, int S_max, float softmax_scale, float* scores, int64_t ld,
