@@ -159,6 +159,28 @@ __device__ __forceinline__ void merge_hist(const uint32_t* h, uint32_t* s, int C
   cluster_barrier();
 }
 
+// A launch of `kernel` as a grid of thread-block clusters of `cluster_x` CTAs along x, with
+// programmatic stream serialization like every other launch of the library.
+template <typename... KArgs, typename... Args>
+int launch_clusters(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, int cluster_x,
+                    Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)cluster_x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
 }  // namespace
 
 template <int KPT>
@@ -490,12 +512,12 @@ int launch_index_topk(const uint8_t* q8, const float* q_scale, const float* w, c
                                       128, kTile, CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
   if (p.tps <= 8)
-    return dsa_host::launch_cluster(index_topk_kernel<8>, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, C,
+    return launch_clusters(index_topk_kernel<8>, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, C,
                                     qmap, kmap, p);
   if (p.tps <= 16)
-    return dsa_host::launch_cluster(index_topk_kernel<16>, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, C,
+    return launch_clusters(index_topk_kernel<16>, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, C,
                                     qmap, kmap, p);
-  return dsa_host::launch_cluster(index_topk_kernel<32>, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, C,
+  return launch_clusters(index_topk_kernel<32>, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, C,
                                   qmap, kmap, p);
 }
 
