@@ -295,8 +295,10 @@ class Step:
             d["kv_len"], scores=self.scores, ld=self.ld))
         rec("topk", lambda: dsa.dsa_topk(self.scores, d["q_pos"], d["kv_len"], self.k, idx=self.idx))
         if self.kv is not None:
+            # the MLA query is a step input (resident, or copied in from the host), never written by
+            # a kernel of the step: the sparse MLA may stage it while the top-k finishes
             rec("sparse_mla", lambda: dsa.dsa_sparse_mla(d["mq"], self.kv, self.idx, out=self.out, lse=self.lse,
-                                                         workspace=self.ws))
+                                                         workspace=self.ws, flags=dsa.DSA_Q_READY))
 
     def l2_flush(self, force=False):
         """Evict the step's data from the L2 (when the step's inputs fit in it, or `force`): write a

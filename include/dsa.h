@@ -78,6 +78,9 @@ typedef struct CUstream_st* dsa_stream_t; /* a cudaStream_t */
                                   indexer steps; rotate_activation in Indexer.forward)         */
 #define DSA_SORTED 0x4u        /* dsa_topk: order the selection by descending score, ties by
                                   ascending position (default: ascending position)           */
+#define DSA_Q_READY 0x8u       /* dsa_sparse_mla_ex: q is complete before the call (a host copy,
+                                  or written two or more kernels earlier): the kernel may stage
+                                  it while the preceding kernel on the stream finishes        */
 #define DSA_F32 0              /* dsa_index_keys input element types                           */
 #define DSA_BF16 1
 #define DSA_FILL_MASKED 0x2u   /* dsa_index_scores: write -inf at masked (s > pos) entries of
@@ -200,6 +203,17 @@ DSA_API int dsa_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t*
                    int B, int T, int S_max, int k, float softmax_scale,
                    uint16_t* out, float* lse, void* workspace, size_t ws_bytes,
                    dsa_stream_t stream);
+
+/*
+ * dsa_sparse_mla_ex - dsa_sparse_mla with flags: 0, or DSA_Q_READY when q is complete before the
+ * call (not written by the kernel launched right before on the stream). The kernel then loads q
+ * while that kernel finishes, and waits for it only before reading idx. Same arguments, results
+ * and errors as dsa_sparse_mla; other flag bits return DSA_ERR_INVALID_ARG.
+ */
+DSA_API int dsa_sparse_mla_ex(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
+                      int B, int T, int S_max, int k, float softmax_scale,
+                      uint16_t* out, float* lse, void* workspace, size_t ws_bytes,
+                      uint32_t flags, dsa_stream_t stream);
 
 /*
  * dsa_sparse_mla_noalloc - the same computation and arguments as dsa_sparse_mla, minus the

@@ -13,7 +13,7 @@ import os
 import torch
 
 __all__ = [
-    "DsaError", "lib", "lib_path", "DSA_HADAMARD", "DSA_FILL_MASKED", "DSA_SORTED", "DSA_F32", "DSA_BF16", "INDEXER_SOFTMAX_SCALE",
+    "DsaError", "lib", "lib_path", "DSA_HADAMARD", "DSA_FILL_MASKED", "DSA_SORTED", "DSA_Q_READY", "DSA_F32", "DSA_BF16", "INDEXER_SOFTMAX_SCALE",
     "MLA_SOFTMAX_SCALE", "dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk", "dsa_index_topk",
     "dsa_sparse_mla", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_noalloc", "dsa_sparse_mla_heads",
     "dsa_sparse_mla_heads_workspace_size",
@@ -28,6 +28,7 @@ DSA_OK = 0
 DSA_HADAMARD = 0x1
 DSA_FILL_MASKED = 0x2
 DSA_SORTED = 0x4
+DSA_Q_READY = 0x8
 DSA_F32 = 0
 DSA_BF16 = 1
 MAX_POS = 16384                 # max_seq_len of the model (ModelArgs)
@@ -65,6 +66,7 @@ def _load():
     L.dsa_topk.argtypes = [vp, i64, vp, vp, i32, i32, i32, u32, vp, vp]
     L.dsa_index_topk.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, f32, i32, u32, vp, vp]
     L.dsa_sparse_mla.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
+    L.dsa_sparse_mla_ex.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp, sz, u32, vp]
     L.dsa_sparse_mla_workspace_size.argtypes = [i32, i32, i32]
     L.dsa_sparse_mla_heads.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
     L.dsa_sparse_mla_heads_workspace_size.argtypes = [i32, i32, i32, i32]
@@ -87,6 +89,7 @@ def _load():
     L.dsa_device_supported.argtypes = []
     L.dsa_version.restype = ctypes.c_char_p
     for f in ("dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk", "dsa_index_topk", "dsa_sparse_mla",
+              "dsa_sparse_mla_ex",
               "dsa_sparse_mla_heads",
               "dsa_sparse_mla_noalloc", "dsa_get_device_status", "dsa_get_error_detail",
               "dsa_selftest_wait_timeout", "dsa_device_supported"):
@@ -300,8 +303,9 @@ def dsa_sparse_mla_workspace_size(B: int, T: int, k: int) -> int:
 
 
 def dsa_sparse_mla(q, kv, idx, softmax_scale: float = MLA_SOFTMAX_SCALE, out=None, lse=None, workspace=None,
-                   want_lse: bool = True, stream=None):
-    """q bf16 [B,T,128,576], kv bf16 [B,S,576], idx int32 [B,T,k] -> (out bf16 [B,T,128,512], lse fp32)."""
+                   want_lse: bool = True, flags: int = 0, stream=None):
+    """q bf16 [B,T,128,576], kv bf16 [B,S,576], idx int32 [B,T,k] -> (out bf16 [B,T,128,512], lse fp32).
+    flags = DSA_Q_READY when q is complete before the call (not written by the kernel right before)."""
     _need(q, torch.bfloat16, "q")
     _need(kv, torch.bfloat16, "kv")
     _need(idx, torch.int32, "idx")
@@ -324,9 +328,13 @@ def dsa_sparse_mla(q, kv, idx, softmax_scale: float = MLA_SOFTMAX_SCALE, out=Non
             raise ValueError("workspace must be on q's device")
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
-    rc = _lib.dsa_sparse_mla(_ptr(q), _ptr(kv), _ptr(idx), B, T, S, int(k), float(softmax_scale), _ptr(out),
-                             _ptr(lse), _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
-                             _stream(stream))
+    ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if flags:
+        rc = _lib.dsa_sparse_mla_ex(_ptr(q), _ptr(kv), _ptr(idx), B, T, S, int(k), float(softmax_scale), _ptr(out),
+                                    _ptr(lse), _ptr(workspace), ws_len, int(flags), _stream(stream))
+    else:
+        rc = _lib.dsa_sparse_mla(_ptr(q), _ptr(kv), _ptr(idx), B, T, S, int(k), float(softmax_scale), _ptr(out),
+                                 _ptr(lse), _ptr(workspace), ws_len, _stream(stream))
     _check(rc, "dsa_sparse_mla")
     return out, lse
 

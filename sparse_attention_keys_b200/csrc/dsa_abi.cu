@@ -342,7 +342,8 @@ size_t dsa_sparse_mla_heads_workspace_size(int B, int T, int k, int heads) {
 
 static int sparse_mla_checked(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T, int S_max,
                               int k, int heads, float softmax_scale, uint16_t* out, float* lse, void* workspace,
-                              size_t ws_bytes, dsa_stream_t stream) {
+                              size_t ws_bytes, dsa_stream_t stream, uint32_t flags = 0) {
+  if ((flags & ~DSA_Q_READY) != 0) return DSA_ERR_INVALID_ARG;
   if (B < 1 || T < 1 || S_max < 1 || k < 1 || !(softmax_scale > 0.f) || !isfinite(softmax_scale))
     return DSA_ERR_INVALID_ARG;
   if ((int64_t)B * T * 2 * 1024 > 0x7fffffffLL) return DSA_ERR_INVALID_ARG;
@@ -355,7 +356,7 @@ static int sparse_mla_checked(const uint16_t* q, const uint16_t* kv, const int32
   int rc = prologue(&status);
   if (rc != DSA_OK) return rc;
   return dsa::launch_sparse_mla(q, kv, idx, B, T, S_max, k, heads, softmax_scale, out, lse, workspace, ws_bytes,
-                                (cudaStream_t)stream, status);
+                                (flags & DSA_Q_READY) != 0, (cudaStream_t)stream, status);
 }
 
 int dsa_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T, int S_max,
@@ -363,6 +364,13 @@ int dsa_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, in
                    size_t ws_bytes, dsa_stream_t stream) {
   return sparse_mla_checked(q, kv, idx, B, T, S_max, k, DSA_MLA_HEADS, softmax_scale, out, lse, workspace, ws_bytes,
                             stream);
+}
+
+int dsa_sparse_mla_ex(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T, int S_max, int k,
+                      float softmax_scale, uint16_t* out, float* lse, void* workspace, size_t ws_bytes,
+                      uint32_t flags, dsa_stream_t stream) {
+  return sparse_mla_checked(q, kv, idx, B, T, S_max, k, DSA_MLA_HEADS, softmax_scale, out, lse, workspace, ws_bytes,
+                            stream, flags);
 }
 
 int dsa_sparse_mla_heads(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T, int S_max, int k,

@@ -43,6 +43,6 @@ int launch_mla_out_absorb(const uint16_t* o, const uint16_t* w_uv, int64_t w_hea
                           uint16_t* out, cudaStream_t stream, int* status);
 int launch_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T,
                       int S_max, int k, int heads, float softmax_scale, uint16_t* out, float* lse,
-                      void* workspace, size_t ws_bytes, cudaStream_t stream, int* status);
+                      void* workspace, size_t ws_bytes, bool q_ready, cudaStream_t stream, int* status);
 
 }  // namespace dsa

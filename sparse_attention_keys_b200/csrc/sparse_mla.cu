@@ -147,6 +147,7 @@ struct MlaParams {
   const int32_t* idx;
   int B, T, S_max, k;
   int heads;                 // query heads per row of q / out / lse (128, or a 64-head shard)
+  int q_ready;               // q is complete before the launch: it may be staged before the wait
   int nsplit, chunk;
   float scale_log2;          // softmax_scale * log2(e)
   uint16_t* out;
@@ -245,7 +246,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 
   // Before the set-up barrier, hint each head's features 0..319 into L2 (softmax warps, staged into
   // TMEM below). A prefetch is only a hint, so it is safe even if the preceding kernel is still
-  // writing Q; every actual read of Q, and of the indices, comes after grid_dep_wait.
+  // writing Q; every actual read of Q (unless the caller stated that Q is complete before the
+  // launch), and of the indices, comes after grid_dep_wait.
   if (warp < kSoftmaxWarps && ntiles > 0) {
     const char* qrow = reinterpret_cast<const char*>(p.q + (bt * HEADS + q_head) * kDqk);
 #pragma unroll
@@ -313,7 +315,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // gather warp w copies keys 8w..8w+7 of each tile; for every key, lane L copies the 16-byte
     // chunks L (block L/8), L+32 (block 4+L/8) and, for L < 8, L+64 (the rotary block)
     const int w = warp - kGatherWarp;
-    grid_dep_wait();                                 // Q and the indices may come from the preceding kernel
+    if (!p.q_ready) grid_dep_wait();                 // Q may come from the preceding kernel
     if (w == 0 && lane == 0 && ntiles > 0) {
       prefetch_tensormap(&q_map);
       mbar_arrive_expect_tx(q_full, kQBytes);
@@ -324,6 +326,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         if (HEADS == 64) tma_load_2d(dst + 64 * 128, &q_map, q_full, 64 * r, (int32_t)(bt * HEADS));
       }
     }
+    if (p.q_ready) grid_dep_wait();                  // the indices may come from the preceding kernel
     const uint16_t* kv_b = PAGED ? p.kv : p.kv + (int64_t)b * p.S_max * kDqk;
     const int32_t* pages = PAGED ? p.block_table + (int64_t)b * p.max_pages : nullptr;
     const uint32_t blk = (uint32_t)(lane >> 3) * kKvRegion;      // block of chunks L and L+32 in its ring slot
@@ -405,7 +408,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // ------------------------------------------------------------------ softmax warps (thread = head)
     const int h = tid;
     const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
-    grid_dep_wait();                                 // Q, the indices (earlier kernels); outputs written below
+    if (!p.q_ready) grid_dep_wait();                 // Q may come from the preceding kernel
     // Q features 0..319 of head h -> TMEM as bf16 pairs (feature f in column f/2)
     if (ntiles > 0) {
       // two batches of loads, each fully in flight before its TMEM stores (which order memory)
@@ -435,6 +438,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       tc_fence_before();
       mbar_arrive(q_full);
     }
+    if (p.q_ready) grid_dep_wait();                  // the indices (earlier kernels); outputs written below
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     // slot j * 32 + lane of the next tile (paged: also the slot two tiles ahead and the next tile's page id)
@@ -708,8 +712,9 @@ static int launch_mla(const uint16_t* q, MlaParams p, cudaStream_t stream, void*
 
 int launch_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T,
                       int S_max, int k, int heads, float softmax_scale, uint16_t* out, float* lse,
-                      void* workspace, size_t ws_bytes, cudaStream_t stream, int* status) {
+                      void* workspace, size_t ws_bytes, bool q_ready, cudaStream_t stream, int* status) {
   MlaParams p{};
+  p.q_ready = q_ready ? 1 : 0;
   p.q = q; p.kv = kv; p.idx = idx; p.B = B; p.T = T; p.S_max = S_max; p.k = k;
   p.scale_log2 = softmax_scale * kLog2e;
   p.out = out; p.lse = lse; p.status = status;

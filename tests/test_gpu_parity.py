@@ -356,6 +356,29 @@ def test_sparse_mla_small_ragged(table_dev):
     assert np.all(got[1, 0] == 0) and np.all(np.isneginf(lse[1, 0]))
 
 
+def test_sparse_mla_q_ready_flag(table_dev):
+    """DSA_Q_READY only moves when the kernel loads q (before it waits for the preceding kernel):
+    the outputs are bitwise those of the plain call, on a split-KV shape and a single-split one,
+    with the indices written by a kernel right before. Other flag bits are rejected."""
+    rng = np.random.default_rng(41)
+    for B, T, S, k in ((2, 3, 300, 64), (4, 1, 3000, 2048)):
+        inp = DI.make_custom(B, T, S, k, decode=(T == 1), seed=8 + B)
+        q_pos = np.minimum(np.tile(np.arange(T, dtype=np.int32) * 37 + S - T * 37, (B, 1)), S - 1)
+        idx = _random_idx(rng, B, T, k, q_pos, inp.kv_len)
+        q, kv = P.bf16_dev(inp.mla_q), P.bf16_dev(inp.mla_kv)
+        idx_src = P.to_dev(idx)
+        idx_dev = torch.empty_like(idx_src)
+        idx_dev.copy_(idx_src)                            # a kernel on the stream writes the indices
+        o0, l0 = dsa.dsa_sparse_mla(q, kv, idx_dev)
+        idx_dev.zero_()
+        idx_dev.copy_(idx_src)
+        o1, l1 = dsa.dsa_sparse_mla(q, kv, idx_dev, flags=dsa.DSA_Q_READY)
+        assert _status() == 0
+        assert torch.equal(o0, o1) and torch.equal(l0, l1)
+    with pytest.raises(dsa.DsaError):
+        dsa.dsa_sparse_mla(q, kv, idx_dev, flags=0x10)
+
+
 def test_sparse_mla_full_context_equals_dense(table_dev):
     inp = DI.make_custom(1, 4, 200, 256, decode=False, seed=7)
     q_pos = np.array([[10, 99, 150, 199]], np.int32)
