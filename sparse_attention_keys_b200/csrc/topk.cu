@@ -422,6 +422,11 @@ __device__ __forceinline__ void st_shared_if(int32_t* dst, int32_t v, bool pred)
 // Exclusive prefix, in thread order, of one value per thread of the CTA (NT threads); *total gets
 // the sum. One barrier; `tot` (NT / 32 words) is written before it and read after it, so a call
 // must not reuse the `tot` of the previous call before another barrier.
+// Bulk prefetch of [p, p + bytes) into the L2 (p 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 template <int NT>
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tot, uint32_t* total) {
   constexpr int kRegWarps = NT / 32;
@@ -482,7 +487,7 @@ template <int KPT, int NT>
 __global__ void __launch_bounds__(NT, 1024 / NT) topk_regs_kernel(const float* __restrict__ scores, int64_t ld,
                                                                    const int32_t* __restrict__ q_pos,
                                                                    const int32_t* __restrict__ kv_len, int T, int k,
-                                                                   uint32_t flags, int sort_n,
+                                                                   uint32_t flags, int sort_n, int ahead,
                                                                    int32_t* __restrict__ idx, int* status) {
   static_assert(KPT % 4 == 0 && KPT <= 32 && KPT * NT <= kRegRowMax, "keys per thread");
   constexpr int kRegThreads = NT, kRegWarps = NT / 32, kRegFixedWords = reg_fixed_words(NT);
@@ -508,6 +513,19 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_regs_kernel(const float* _
   grid_dep_wait();                                          // the scores come from the preceding kernel
   grid_dep_launch();
   int32_t* out = idx + row * (int64_t)k;
+  // The row that the CTA taking a slot `ahead` launches later will read goes into the L2 now
+  // (rows are dispatched in order, and a slot frees about one row's time later), so that its load
+  // phase reads the L2 instead of waiting on DRAM.
+  if (ahead > 0 && tid < 32 && row + ahead < (int64_t)gridDim.x) {
+    const int64_t nrow = row + ahead;
+    const int nn = min(q_pos[nrow] + 1, kv_len[nrow / T]);
+    if ((nn > k || sorted) && nn > 0 && (int64_t)nn <= ld) {
+      const uint32_t bytes = (uint32_t)((nn + 3) >> 2) * 16u;
+      const char* base = reinterpret_cast<const char*>(scores + nrow * ld);
+      for (uint32_t off = (uint32_t)tid * 4096u; off < bytes; off += 32u * 4096u)
+        prefetch_l2(base + off, min(4096u, bytes - off));
+    }
+  }
   int n = min(q_pos[row] + 1, kv_len[b]);
   if (n < 0) n = 0;
   if (n <= k && !sorted) {                                  // everything visible is selected
@@ -734,8 +752,16 @@ static int launch_topk_regs(const float* scores, int64_t ld, const int32_t* q_po
       dsa_host::mark_setup(configured);
     }
   }
+  // the CTAs resident at once: the distance to the row whose scores a CTA prefetches into the L2
+  int ahead = 0;
+  if (rows > dsa_host::device_sm_count()) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_regs_kernel<KPT, NT>, NT, smem) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    ahead = std::max(1, per_sm) * dsa_host::device_sm_count();
+  }
   return dsa_host::launch(topk_regs_kernel<KPT, NT>, dim3((unsigned)rows), dim3(NT), smem, stream, scores, ld,
-                          q_pos, kv_len, T, k, flags, sort_n, idx, status);
+                          q_pos, kv_len, T, k, flags, sort_n, ahead, idx, status);
 }
 
 int launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, const int32_t* kv_len, int B,
