@@ -562,7 +562,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks,
     }
     if producers is not None:
-        line["mla_producers"] = producer_rooflines(producers, peaks)
+        line["mla_producers"] = producer_rooflines(producers, peaks, args.workload)
     if paged is not None:
         line["paged_caches"] = paged_rooflines(paged, units, peaks, args)
     extras = [w for w in (args.extra or "").split(",") if w and w not in (args.workload, "none")]
@@ -693,9 +693,10 @@ def paged_rooflines(t, units, peaks, args):
     return res
 
 
-def producer_rooflines(t, peaks):
+def producer_rooflines(t, peaks, workload=None):
     """Per producer: device time, algorithmic bytes / flops and the HBM roofline (all three are
-    below the bf16 ridge: bound by memory)."""
+    below the bf16 ridge: bound by memory), with the ncu DRAM traffic where a current capture of
+    that producer on this workload is committed."""
     units = producer_units(t["rows"])
     res = {"rows": t["rows"], "timing": "graph of the call alone, L2 flushed before each replay"}
     for name in ("q_absorb", "kv_entry", "out_absorb"):
@@ -704,7 +705,8 @@ def producer_rooflines(t, peaks):
         ach = u["bytes"] / sec / 1e9
         res[name] = {"us": sec * 1e6, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": ach / peaks["hbm_gbs"], "algorithmic_bytes": u["bytes"],
-                     "tflops": u["flops"] / sec / 1e12 if u["flops"] else None}
+                     "tflops": u["flops"] / sec / 1e12 if u["flops"] else None,
+                     "traffic": load_traffic(name, workload) if workload else None}
     return res
 
 

@@ -38,7 +38,7 @@ struct AbsorbParams {
   const float* rope_cs;      // [max_pos][32][2]
   int max_pos;
   int64_t rows;
-  int tiles_per_cta;         // row tiles each CTA runs (for one head and one output part)
+  int tiles_per_cta;         // out_absorb: row tiles each CTA runs (for one head)
   uint16_t* out;             // q_absorb [rows][128][576]; out_absorb [rows][128][128]
   int* status;
 };
@@ -87,47 +87,72 @@ __device__ __forceinline__ void store_bf16_32(uint8_t* dst, const uint32_t (&v)[
 }
 
 // ------------------------------------------------------------------------------------ q_absorb
-// CTA = (group of row tiles, head h, output part n): latent features [256n, 256n + 256) of head h,
-// the part n = 1 also writes the rotated q_pe (features 512..575 follow its 256 features).
-// Shared memory: w_uk[h][:, 256n : 256n+256] as 4 MN-major regions (64 c x 128 d rows), resident;
-// two stages of the q_nope tile (2 K-major regions of 128 rows x 64 d); a staging row per tile row.
+// Work item = (head h, 128-row tile): the whole 576-feature q row of head h for the tile's tokens,
+// so each q_nope tile is read once. Items are ordered head-major and each CTA (one per SM) runs an
+// equal range of them, which crosses into at most a few heads; the head's W_UK[h] (128 KB) stays
+// resident in shared memory until its last item, then the next head's is loaded in its place.
+// Per item the two 256-feature halves accumulate in their own TMEM accumulator (512 columns), so
+// the epilogue drains one half while the MMAs of the other (or of the next tile) run. Each
+// epilogue warp writes its 32 rows in 64-feature chunks through four swizzled 4 KB staging buffers
+// with TMA tensor stores (full 128-byte lines; rows past the end are clipped by the tensor map).
+// Four more warps rotate q_pe (features 512..575, one 128-byte segment per row) for the same
+// items, off the epilogue's path: their position -> table loads are the longest latency here.
 namespace qa {
-constexpr int kOffB = 0;
-constexpr int kOffA = 4 * kRegion;
+constexpr int kThreads = 320;                         // warp 0 TMA, 1 MMA + TMEM owner, 2-5 epilogue, 6-9 RoPE
+constexpr int kOffB = 0;                              // W_UK[h]: 8 MN-major regions (64 c x 128 d rows)
+constexpr int kOffA = 8 * kRegion;                    // the q_nope tile: 2 K-major regions (128 rows x 64 d)
 constexpr int kAStage = 2 * kRegion;
-constexpr int kRowBytes = 656;                        // 640 B (256 + 64 bf16) + 16 B pad
-constexpr int kOffStage = kOffA + 2 * kAStage;
-constexpr int kOffBar = kOffStage + kRows * kRowBytes;
+constexpr int kAStages = 1;                           // an item's drain outlasts the next tile's load
+constexpr int kStageBytes = 32 * 128;                 // one warp's 32 rows x 64 features, 128B swizzle
+constexpr int kStageBufs = 4;                         // staging buffers per epilogue warp (stores in flight)
+constexpr int kOffStage = kOffA + kAStages * kAStage;
+constexpr int kOffBar = kOffStage + 4 * kStageBufs * kStageBytes;
 constexpr int kSmemBytes = kOffBar + 128 + 1024;       // + alignment slack
-constexpr int kTmemCols = 512;                        // two 128 x 256 fp32 accumulators
+constexpr int kTmemCols = 512;                        // the two 128 x 256 fp32 halves of one tile
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+static_assert(kOffStage % 1024 == 0 && kStageBytes % 1024 == 0, "128B-swizzled staging alignment");
 }  // namespace qa
 
-__global__ void __launch_bounds__(kThreads, 1)
+// TMA tensor store of a shared-memory box to (x, y, z) of the map's tensor, in the bulk group.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int32_t x, int32_t y, int32_t z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z) : "memory");
+}
+
+// Wait until at most N of this thread's bulk groups still have to read their shared-memory source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read_n() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
+
+__global__ void __launch_bounds__(qa::kThreads, 1)
     q_absorb_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constant__ CUtensorMap w_map,
-                    const AbsorbParams p) {
+                    const __grid_constant__ CUtensorMap o_map, const AbsorbParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + qa::kOffBar);
-  uint64_t* b_full = bars;               // weights landed
-  uint64_t* a_full = bars + 1;           // [2] q_nope tile landed
-  uint64_t* a_empty = bars + 3;          // [2] MMAs done reading the tile
-  uint64_t* acc_full = bars + 5;         // [2] accumulator ready
-  uint64_t* acc_empty = bars + 7;        // [2] accumulator drained (128 arrivals)
+  uint64_t* w_full = bars;               // a head's weights landed
+  uint64_t* w_empty = bars + 1;          // the MMAs of a head's last item are done with its weights
+  uint64_t* a_full = bars + 2;           // [2] q_nope tile landed
+  uint64_t* a_empty = bars + 4;          // [2] MMAs done reading the tile
+  uint64_t* acc_full = bars + 6;         // [2] half n of the item's product ready
+  uint64_t* acc_empty = bars + 8;        // [2] half n drained (128 arrivals)
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n = blockIdx.x & 1;
-  const int h = (blockIdx.x >> 1) % kHeadsA;
-  const int64_t g = (blockIdx.x >> 1) / kHeadsA;
   const int64_t ntiles = (p.rows + kRows - 1) / kRows;
-  const int64_t tile0 = g * p.tiles_per_cta;
-  const int my_tiles = (int)max((int64_t)0, min((int64_t)p.tiles_per_cta, ntiles - tile0));
+  const int64_t items = (int64_t)kHeadsA * ntiles;
+  const int64_t i0 = (int64_t)blockIdx.x * items / gridDim.x;
+  const int my_items = (int)((int64_t)(blockIdx.x + 1) * items / gridDim.x - i0);
+  const int h0 = (int)(i0 / ntiles);
+  // item j of this CTA: its head, its tile, and whether it is the first of its head here
+  auto head_of = [&](int j) { return (int)((i0 + j) / ntiles); };
+  auto tile_of = [&](int j) { return (i0 + j) % ntiles; };
+  auto new_head = [&](int j) { return j == 0 || tile_of(j) == 0; };
 
   if (tid == 0) {
     abort_flag = 0;
-    mbar_init(b_full, 1);
+    mbar_init(w_full, 1);
+    mbar_init(w_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&a_full[i], 1);
       mbar_init(&a_empty[i], 1);
@@ -149,20 +174,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0 && my_tiles > 0) {
+    if (lane == 0 && my_items > 0) {
       prefetch_tensormap(&a_map);
       prefetch_tensormap(&w_map);
-      mbar_arrive_expect_tx(b_full, 4 * kRegion);
-      for (int j = 0; j < 4; ++j) tma_load_3d(smem + qa::kOffB + j * kRegion, &w_map, b_full, 256 * n + 64 * j, 0, h);
-      // The two CTAs of a head (n = 0, 1) read the same q_nope tiles. Requested at the same moment
-      // both miss the L2; the second trails by the weight load, so its tiles come from the L2.
-      bool go = n == 0 || mbar_wait(b_full, 0, &abort_flag, p.status, DSA_SITE_ABSORB_W);
-      for (int i = 0; go && i < my_tiles; ++i) {
-        const int s = i & 1;
-        if (i >= 2 && !mbar_wait(&a_empty[s], ((i >> 1) + 1) & 1, &abort_flag, p.status, DSA_SITE_ABSORB_A_EMPTY))
+      for (int j = 0; j < my_items; ++j) {
+        const int h = head_of(j);
+        if (new_head(j)) {
+          const int seg = h - h0;
+          if (seg > 0 && !mbar_wait(w_empty, (seg - 1) & 1, &abort_flag, p.status, DSA_SITE_ABSORB_W)) break;
+          mbar_arrive_expect_tx(w_full, 8 * kRegion);
+          for (int r = 0; r < 8; ++r) tma_load_3d(smem + qa::kOffB + r * kRegion, &w_map, w_full, 64 * r, 0, h);
+        }
+        const int s = j % qa::kAStages;
+        if (j >= qa::kAStages &&
+            !mbar_wait(&a_empty[s], (j / qa::kAStages - 1) & 1, &abort_flag, p.status, DSA_SITE_ABSORB_A_EMPTY))
           break;
         mbar_arrive_expect_tx(&a_full[s], qa::kAStage);
-        const int32_t t = (int32_t)((tile0 + i) * kRows);
+        const int32_t t = (int32_t)(tile_of(j) * kRows);
         uint8_t* dst = smem + qa::kOffA + s * qa::kAStage;
         tma_load_3d(dst, &a_map, &a_full[s], 0, h, t);
         tma_load_3d(dst + kRegion, &a_map, &a_full[s], 64, h, t);
@@ -170,66 +198,107 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0 && my_tiles > 0) {
+    if (lane == 0 && my_items > 0) {
       constexpr uint32_t idesc = idesc_f32acc(1, 1, kRows, 256, 0, 1 /*B MN-major*/);
       const uint32_t b_addr = smem_u32(smem + qa::kOffB);
-      bool ok = mbar_wait(b_full, 0, &abort_flag, p.status, DSA_SITE_ABSORB_W);
-      for (int i = 0; ok && i < my_tiles; ++i) {
-        const int s = i & 1, a = i & 1;
-        if (i >= 2 && !mbar_wait(&acc_empty[a], ((i >> 1) + 1) & 1, &abort_flag, p.status, DSA_SITE_ABSORB_ACC_EMPTY))
-          break;
-        if (!mbar_wait(&a_full[s], (i >> 1) & 1, &abort_flag, p.status, DSA_SITE_ABSORB_A_FULL)) break;
-        tc_fence_after();
+      bool ok = true;
+      for (int j = 0; ok && j < my_items; ++j) {
+        if (new_head(j) && !mbar_wait(w_full, (head_of(j) - h0) & 1, &abort_flag, p.status, DSA_SITE_ABSORB_W)) break;
+        const int s = j % qa::kAStages;
+        if (!mbar_wait(&a_full[s], (j / qa::kAStages) & 1, &abort_flag, p.status, DSA_SITE_ABSORB_A_FULL)) break;
         const uint32_t a_addr = smem_u32(smem + qa::kOffA + s * qa::kAStage);
+        for (int n = 0; n < 2; ++n) {
+          if (j >= 1 && !mbar_wait(&acc_empty[n], (j - 1) & 1, &abort_flag, p.status, DSA_SITE_ABSORB_ACC_EMPTY)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < kNope / 16; ++ks) {
-          const uint64_t ad = sdesc_kmajor_sw128(a_addr + (ks >> 2) * kRegion + (ks & 3) * 32);
-          const uint64_t bd = sdesc_mnmajor_sw128(b_addr + ks * 2048, kRegion, 1024);   // 16 d-rows per K-step
-          mma_f16_ss(tmem + a * 256, ad, bd, idesc, ks > 0 ? 1u : 0u);
+          for (int ks = 0; ks < kNope / 16; ++ks) {
+            const uint64_t ad = sdesc_kmajor_sw128(a_addr + (ks >> 2) * kRegion + (ks & 3) * 32);
+            const uint64_t bd = sdesc_mnmajor_sw128(b_addr + n * 4 * kRegion + ks * 2048, kRegion, 1024);
+            mma_f16_ss(tmem + n * 256, ad, bd, idesc, ks > 0 ? 1u : 0u);
+          }
+          mma_commit(&acc_full[n]);
         }
+        if (!ok) break;
         mma_commit(&a_empty[s]);
-        mma_commit(&acc_full[a]);
+        if (j + 1 < my_items && new_head(j + 1)) mma_commit(w_empty);   // the next head may replace the weights
       }
+    }
+  } else if (warp >= 6) {
+    // ------------------------------------------------------------------ RoPE (warps 6-9)
+    // thread = tile row; the next item's position is loaded one item ahead
+    const int r = tid - 6 * 32;
+    auto row_of = [&](int j) { return tile_of(j) * kRows + r; };
+    int pos_next = my_items > 0 && row_of(0) < p.rows ? __ldg(p.pos + row_of(0)) : 0;
+    for (int j = 0; j < my_items; ++j) {
+      const int64_t t = row_of(j);
+      const int pos = pos_next;
+      if (j + 1 < my_items && row_of(j + 1) < p.rows) pos_next = __ldg(p.pos + row_of(j + 1));
+      if (t >= p.rows) continue;
+      const int h = head_of(j);
+      uint4 rv[8];
+      if (!rope_row(p.q_pe + (t * kHeadsA + h) * kRopeD, pos, p, rv)) set_status(p.status, DSA_ERR_DEVICE_BOUNDS);
+      uint4* dst = reinterpret_cast<uint4*>(p.out + (t * kHeadsA + h) * kQk + kLat);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) dst[c] = rv[c];
     }
   } else {
     // ------------------------------------------------------------------ epilogue (warps 2-5)
-    // warp w reads TMEM lane quadrant w % 4: one tile row per thread
+    // warp w reads TMEM lane quadrant w % 4: one tile row per thread, 32 rows per warp
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;
-    uint8_t* srow = smem + qa::kOffStage + r * qa::kRowBytes;
-    for (int i = 0; i < my_tiles; ++i) {
-      const int a = i & 1;
-      const int64_t t = (tile0 + i) * kRows + r;
-      if (i > 0) bulk_wait_read();                   // the previous row's copy has read the staging row
-      // the rotary part first: its loads do not depend on the MMAs and overlap them
-      if (n == 1 && t < p.rows) {
-        const int pos = __ldg(p.pos + t);
-        if (!rope_row(p.q_pe + (t * kHeadsA + h) * kRopeD, pos, p, reinterpret_cast<uint4*>(srow + 512)))
-          set_status(p.status, DSA_ERR_DEVICE_BOUNDS);
-      }
-      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[a], (i >> 1) & 1, &abort_flag, p.status,
-                                             DSA_SITE_ABSORB_ACC_FULL)))
-        break;
-      tc_fence_after();
-      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + a * 256;
-#pragma unroll 1
-      for (int c = 0; c < 8; c += 2) {
-        uint32_t v0[32], v1[32];
-        tmem_ld32(taddr + c * 32, v0);
-        tmem_ld32(taddr + (c + 1) * 32, v1);
-        tmem_ld_wait();
-        store_bf16_32(srow + c * 64, v0);
-        store_bf16_32(srow + (c + 1) * 64, v1);
-      }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[a]);
-      if (t < p.rows) {
-        fence_proxy_async_smem();
-        bulk_store_s2g(p.out + (t * kHeadsA + h) * kQk + 256 * n, smem_u32(srow), n ? 640u : 512u);
+    uint8_t* stage = smem + qa::kOffStage + quad * qa::kStageBufs * qa::kStageBytes;
+    uint32_t chunks = 0;                                     // 64-feature chunks this warp has staged
+    // stage one 64-feature chunk (32 packed bf16 pairs) of this lane's row, then store the warp's box
+    auto put = [&](const uint32_t (&v)[32], int feat, int h, int32_t z, bool live) {
+      uint8_t* buf = stage + (chunks % qa::kStageBufs) * qa::kStageBytes;
+      if (lane == 0 && chunks >= qa::kStageBufs)            // the store that last read this buffer is done
+        bulk_wait_read_n<qa::kStageBufs - 1>();
+      __syncwarp();
+#pragma unroll
+      for (int c = 0; c < 8; ++c)                            // 128B swizzle: 16-byte chunk c of row r at c ^ (r % 8)
+        *reinterpret_cast<uint4*>(buf + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+            make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && live) {
+        tma_store_3d(&o_map, buf, feat, h, z);
         bulk_commit();
       }
+      ++chunks;
+    };
+    for (int j = 0; j < my_items; ++j) {
+      const int h = head_of(j);
+      const int32_t z = (int32_t)(tile_of(j) * kRows + quad * 32);   // this warp's first row
+      const bool live = z < p.rows;
+      bool ok = true;
+      for (int n = 0; n < 2; ++n) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[n], j & 1, &abort_flag, p.status, DSA_SITE_ABSORB_ACC_FULL))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + n * 256;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t x0[32], x1[32], v[32];
+          tmem_ld32(taddr + c * 64, x0);
+          tmem_ld32(taddr + c * 64 + 32, x1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            v[i] = pack_bf16(__uint_as_float(x0[2 * i]), __uint_as_float(x0[2 * i + 1]));
+            v[16 + i] = pack_bf16(__uint_as_float(x1[2 * i]), __uint_as_float(x1[2 * i + 1]));
+          }
+          put(v, 256 * n + 64 * c, h, z, live);
+        }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[n]);
+      }
+      if (!ok) break;
     }
-    bulk_wait_all();
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -712,12 +781,19 @@ int launch_mla_q_absorb(const uint16_t* q_nope, const uint16_t* q_pe, const int3
     return dsa_host::launch(q_absorb_few_kernel, dim3(kHeadsA), dim3(kThreads), fr::kSmemBytes, stream, x_map, w_map,
                             p, n_pad);
   }
-  p.tiles_per_cta = tiles_per_cta(ntiles, 2 * kHeadsA);
+  // the output q [rows][128][576], written in boxes of 32 rows x 64 features of one head
+  CUtensorMap o_map;
+  const uint64_t o_dims[3] = {kQk, kHeadsA, (uint64_t)rows};
+  const uint64_t o_str[2] = {kQk * 2, (uint64_t)kHeadsA * kQk * 2};
+  const uint32_t o_box[3] = {64, 1, 32};
+  if (!dsa_host::encode_tensor_map_3d(&o_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (void*)q_out, o_dims, o_str, o_box,
+                                      CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  p.tiles_per_cta = 0;                       // items are split evenly over one CTA per SM
   p.out = q_out; p.status = status;
-  const int64_t grid = (ntiles + p.tiles_per_cta - 1) / p.tiles_per_cta * 2 * kHeadsA;
-  if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;
-  return dsa_host::launch(q_absorb_kernel, dim3((unsigned)grid), dim3(kThreads), qa::kSmemBytes, stream, a_map, w_map,
-                          p);
+  const int64_t grid = std::min<int64_t>(dsa_host::device_sm_count(), ntiles * kHeadsA);
+  return dsa_host::launch(q_absorb_kernel, dim3((unsigned)grid), dim3(qa::kThreads), qa::kSmemBytes, stream, a_map,
+                          w_map, o_map, p);
 }
 
 int launch_mla_out_absorb(const uint16_t* o, const uint16_t* w_uv, int64_t w_head_stride, int64_t rows,

@@ -45,7 +45,10 @@ def _weights(inp):
     return wkv_b, wkv_b[:, :128], wkv_b[:, 128:]
 
 
-@pytest.mark.parametrize("rows", [1, 8, 33, 64, 65, 130, 300])    # <= 64: one CTA per head
+# <= 64 rows: one CTA per head; above, (head, 128-row tile) items split over one CTA per SM, whose
+# ranges cross from one head to the next (65, 130: one to three items per CTA; 600, 1000: four to
+# seven items, ragged last tiles)
+@pytest.mark.parametrize("rows", [1, 8, 33, 64, 65, 130, 300, 600, 1000])
 def test_q_absorb(table_dev, rows):
     inp = DI.make_mla_producer_inputs(rows, seed=rows)
     _, w_uk, _ = _weights(inp)
