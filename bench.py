@@ -3,9 +3,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode_b64] [--extra prefill_16384]
                     [--impl ours|reference]
 
-A decode step runs, through the C ABI: dsa_index_keys on the new keys (written into the
-resident FP8 K-cache) and on the queries, dsa_index_scores, dsa_topk and dsa_sparse_mla. A
-prefill step runs the same calls over all T queries and S keys. Inputs are seeded synthetic
+A decode step runs, through the C ABI: dsa_index_qk (the dsa_index_keys transform of the new keys,
+written into the resident FP8 K-cache, and of the queries, in one launch), dsa_index_scores,
+dsa_topk and dsa_sparse_mla. A prefill step runs the same calls over all T queries and S keys. Inputs are seeded synthetic
 tensors of the workload's shapes (dsa_inputs); the caches are resident device state.
 
 Timing: W untimed warm-up steps, then K steps, each a replay of a CUDA graph of the step bracketed
@@ -244,7 +244,7 @@ class Step:
         self.h_idx = torch.empty((B, T, self.k), dtype=torch.int32).pin_memory()
         self.h_out = torch.empty((B, T, 128, 512), dtype=torch.bfloat16).pin_memory() if self.out is not None else None
         self.h_lse = torch.empty((B, T, 128), dtype=torch.float32).pin_memory() if self.out is not None else None
-        self.launches_per_step = 4 + (1 if self.kv is not None else 0) + (
+        self.launches_per_step = 3 + (1 if self.kv is not None else 0) + (
             1 if ws > 0 else 0)
 
     def h2d(self):
@@ -286,10 +286,9 @@ class Step:
             ev.setdefault(name, []).append((s, e))
 
         B, T = self.B, self.T
-        rec("index_keys", lambda: (
-            dsa.dsa_index_keys(d["kx"], d["kpos"], self.table, out_fp8=self.kcache, out_scale=self.kscale,
-                               dst_row=d["kdst"]),
-            dsa.dsa_index_keys(d["qx"], d["qpos_flat"], self.table, out_fp8=self.q8, out_scale=self.qs)))
+        rec("index_keys", lambda: dsa.dsa_index_qk(
+            d["kx"], d["kpos"], d["qx"], d["qpos_flat"], self.table, self.kcache, self.kscale, k_dst_row=d["kdst"],
+            q_out_fp8=self.q8, q_out_scale=self.qs))
         rec("index_scores", lambda: dsa.dsa_index_scores(
             self.q8.view(B, T, 64, 128), self.qs.view(B, T, 64), d["w"], self.kcache, self.kscale, d["q_pos"],
             d["kv_len"], scores=self.scores, ld=self.ld))

@@ -125,6 +125,22 @@ DSA_API int dsa_index_keys(const void* x, int x_dtype, int64_t rows, int heads, 
                    dsa_stream_t stream);
 
 /*
+ * dsa_index_qk - the indexer's key and query transforms of one step in a single launch
+ * ([rotate] Indexer.forward applies the same RoPE, rotate_activation and act_quant to the new
+ * key and to the queries before fp8_index). Equivalent to
+ *   dsa_index_keys(kx, x_dtype, k_rows, 1, k_pos, ..., k_out_fp8, k_out_scale, k_dst_row) and
+ *   dsa_index_keys(qx, x_dtype, q_rows, q_heads, q_pos, ..., q_out_fp8, q_out_scale, NULL)
+ * with the same rope_cs, max_pos and flags, bit for bit, and the same argument checks and errors
+ * (either side may have 0 rows; its pointers are then not read). The key outputs and the query
+ * outputs must not overlap (not checked).
+ */
+DSA_API int dsa_index_qk(const void* kx, int64_t k_rows, const int32_t* k_pos, const int64_t* k_dst_row,
+                         uint8_t* k_out_fp8, float* k_out_scale,
+                         const void* qx, int64_t q_rows, int q_heads, const int32_t* q_pos,
+                         uint8_t* q_out_fp8, float* q_out_scale,
+                         int x_dtype, const float* rope_cs, int max_pos, uint32_t flags, dsa_stream_t stream);
+
+/*
  * dsa_index_scores - lightning-indexer scores (fp8_index in Indexer.forward; [dense]
  * S^I_{t,s} = 1/(sqrt 64 sqrt 128) sum_h w_{t,h} ReLU(Q^I_{h,t} . k^I_s)).
  *

@@ -14,8 +14,8 @@ import torch
 
 __all__ = [
     "DsaError", "lib", "lib_path", "DSA_HADAMARD", "DSA_FILL_MASKED", "DSA_SORTED", "DSA_Q_READY", "DSA_F32", "DSA_BF16", "INDEXER_SOFTMAX_SCALE",
-    "MLA_SOFTMAX_SCALE", "dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk", "dsa_index_topk",
-    "dsa_sparse_mla", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_noalloc", "dsa_sparse_mla_heads",
+    "MLA_SOFTMAX_SCALE", "dsa_rope_table", "dsa_index_keys", "dsa_index_qk", "dsa_index_scores", "dsa_topk",
+    "dsa_index_topk", "dsa_sparse_mla", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_noalloc", "dsa_sparse_mla_heads",
     "dsa_sparse_mla_heads_workspace_size",
     "dsa_index_scores_paged", "dsa_sparse_mla_paged", "dsa_mla_q_absorb", "dsa_mla_kv_entry",
     "dsa_mla_out_absorb",
@@ -62,6 +62,7 @@ def _load():
                                   ctypes.c_float, ctypes.c_size_t)
     L.dsa_rope_table.argtypes = [vp, i32]
     L.dsa_index_keys.argtypes = [vp, i32, i64, i32, vp, vp, i32, u32, vp, vp, vp, vp]
+    L.dsa_index_qk.argtypes = [vp, i64, vp, vp, vp, vp, vp, i64, i32, vp, vp, vp, i32, vp, i32, u32, vp]
     L.dsa_index_scores.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, f32, vp, i64, u32, vp]
     L.dsa_topk.argtypes = [vp, i64, vp, vp, i32, i32, i32, u32, vp, vp]
     L.dsa_index_topk.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, f32, i32, u32, vp, vp]
@@ -88,7 +89,7 @@ def _load():
     L.dsa_status_string.restype = ctypes.c_char_p
     L.dsa_device_supported.argtypes = []
     L.dsa_version.restype = ctypes.c_char_p
-    for f in ("dsa_rope_table", "dsa_index_keys", "dsa_index_scores", "dsa_topk", "dsa_index_topk", "dsa_sparse_mla",
+    for f in ("dsa_rope_table", "dsa_index_keys", "dsa_index_qk", "dsa_index_scores", "dsa_topk", "dsa_index_topk", "dsa_sparse_mla",
               "dsa_sparse_mla_ex",
               "dsa_sparse_mla_heads",
               "dsa_sparse_mla_noalloc", "dsa_get_device_status", "dsa_get_error_detail",
@@ -179,6 +180,47 @@ def dsa_index_keys(x, pos, rope_cs, flags: int = DSA_HADAMARD, out_fp8=None, out
                              _ptr(out_fp8), _ptr(out_scale), _ptr(dst_row), _stream(stream))
     _check(rc, "dsa_index_keys")
     return out_fp8, out_scale
+
+
+def dsa_index_qk(kx, k_pos, qx, q_pos, rope_cs, k_out_fp8, k_out_scale, k_dst_row=None, q_out_fp8=None,
+                 q_out_scale=None, flags: int = DSA_HADAMARD, stream=None):
+    """The new keys kx [k_rows, 128] and the queries qx [q_rows, heads, 128] (one dtype, fp32 or
+    bf16) through dsa_index_keys in one launch. The key codes and scales go to k_out_fp8 /
+    k_out_scale (at the rows k_dst_row names, or densely when it is None); returns the query
+    (codes, scales)."""
+    if kx.dtype not in (torch.float32, torch.bfloat16) or qx.dtype != kx.dtype:
+        raise TypeError("kx and qx must be both float32 or both bfloat16")
+    for t, dt, n in ((kx, kx.dtype, "kx"), (qx, qx.dtype, "qx"), (k_pos, torch.int32, "k_pos"),
+                     (q_pos, torch.int32, "q_pos"), (rope_cs, torch.float32, "rope_cs"),
+                     (k_out_fp8, torch.uint8, "k_out_fp8"), (k_out_scale, torch.float32, "k_out_scale")):
+        _need(t, dt, n)
+    if kx.dim() != 2 or kx.shape[-1] != 128 or qx.dim() != 3 or qx.shape[-1] != 128:
+        raise ValueError("kx must be [rows, 128] and qx [rows, heads, 128]")
+    if k_pos.numel() != kx.shape[0] or q_pos.numel() != qx.shape[0]:
+        raise ValueError("k_pos and q_pos must have one entry per row")
+    if k_dst_row is not None:
+        _need(k_dst_row, torch.int64, "k_dst_row")
+        if k_dst_row.numel() != kx.shape[0]:
+            raise ValueError("k_dst_row must have one entry per key row")
+    elif k_out_fp8.numel() < kx.numel() or k_out_scale.numel() < kx.shape[0]:
+        raise ValueError("dense key outputs are smaller than kx")
+    if q_out_fp8 is None:
+        q_out_fp8 = torch.empty(qx.shape, dtype=torch.uint8, device=qx.device)
+    if q_out_scale is None:
+        q_out_scale = torch.empty(qx.shape[:-1], dtype=torch.float32, device=qx.device)
+    _need(q_out_fp8, torch.uint8, "q_out_fp8")
+    _need(q_out_scale, torch.float32, "q_out_scale")
+    if q_out_fp8.numel() < qx.numel() or q_out_scale.numel() < qx.numel() // 128:
+        raise ValueError("query outputs are smaller than qx")
+    devs = {t.device for t in (kx, qx, k_pos, q_pos, rope_cs, k_out_fp8, k_out_scale, q_out_fp8, q_out_scale)}
+    if len(devs) != 1:
+        raise ValueError("all tensors must be on one device")
+    x_dtype = DSA_BF16 if kx.dtype == torch.bfloat16 else DSA_F32
+    rc = _lib.dsa_index_qk(_ptr(kx), kx.shape[0], _ptr(k_pos), _ptr(k_dst_row), _ptr(k_out_fp8), _ptr(k_out_scale),
+                           _ptr(qx), qx.shape[0], qx.shape[1], _ptr(q_pos), _ptr(q_out_fp8), _ptr(q_out_scale),
+                           x_dtype, _ptr(rope_cs), rope_cs.shape[0], int(flags), _stream(stream))
+    _check(rc, "dsa_index_qk")
+    return q_out_fp8, q_out_scale
 
 
 def dsa_index_scores(q8, q_scale, w, k8, k_scale, q_pos, kv_len, softmax_scale: float = INDEXER_SOFTMAX_SCALE,

@@ -257,9 +257,10 @@ int dsa_rope_table(float* table, int max_pos) {
   return DSA_OK;
 }
 
-int dsa_index_keys(const void* x, int x_dtype, int64_t rows, int heads, const int32_t* pos, const float* rope_cs,
-                   int max_pos, uint32_t flags, uint8_t* out_fp8, float* out_scale,
-                   const int64_t* dst_row, dsa_stream_t stream) {
+// The argument checks of dsa_index_keys (no launch): DSA_OK, or DSA_ERR_INVALID_ARG.
+static int index_keys_args(const void* x, int x_dtype, int64_t rows, int heads, const int32_t* pos,
+                           const float* rope_cs, int max_pos, uint32_t flags, const uint8_t* out_fp8,
+                           const float* out_scale, const int64_t* dst_row) {
   if (rows < 0 || heads < 1 || heads > 4096 || max_pos < 1 || max_pos > DSA_MAX_POS ||
       (flags & ~DSA_HADAMARD) != 0 || (x_dtype != DSA_F32 && x_dtype != DSA_BF16))
     return DSA_ERR_INVALID_ARG;
@@ -269,11 +270,38 @@ int dsa_index_keys(const void* x, int x_dtype, int64_t rows, int heads, const in
       !dsa_host::aligned16(out_scale) || (dst_row && !dsa_host::aligned16(dst_row)) ||
       !dsa_host::aligned16(pos))
     return DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
+int dsa_index_keys(const void* x, int x_dtype, int64_t rows, int heads, const int32_t* pos, const float* rope_cs,
+                   int max_pos, uint32_t flags, uint8_t* out_fp8, float* out_scale,
+                   const int64_t* dst_row, dsa_stream_t stream) {
+  int rc = index_keys_args(x, x_dtype, rows, heads, pos, rope_cs, max_pos, flags, out_fp8, out_scale, dst_row);
+  if (rc != DSA_OK || rows == 0) return rc;
   int* status;
-  int rc = prologue(&status);
+  rc = prologue(&status);
   if (rc != DSA_OK) return rc;
   return dsa::launch_index_keys(x, x_dtype, rows, heads, pos, rope_cs, max_pos, flags, out_fp8, out_scale,
                                 dst_row, (cudaStream_t)stream, status);
+}
+
+int dsa_index_qk(const void* kx, int64_t k_rows, const int32_t* k_pos, const int64_t* k_dst_row,
+                 uint8_t* k_out_fp8, float* k_out_scale, const void* qx, int64_t q_rows, int q_heads,
+                 const int32_t* q_pos, uint8_t* q_out_fp8, float* q_out_scale, int x_dtype,
+                 const float* rope_cs, int max_pos, uint32_t flags, dsa_stream_t stream) {
+  int rc = index_keys_args(kx, x_dtype, k_rows, 1, k_pos, rope_cs, max_pos, flags, k_out_fp8, k_out_scale,
+                           k_dst_row);
+  if (rc != DSA_OK) return rc;
+  rc = index_keys_args(qx, x_dtype, q_rows, q_heads, q_pos, rope_cs, max_pos, flags, q_out_fp8, q_out_scale,
+                       nullptr);
+  if (rc != DSA_OK) return rc;
+  if (k_rows == 0 && q_rows == 0) return DSA_OK;
+  int* status;
+  rc = prologue(&status);
+  if (rc != DSA_OK) return rc;
+  return dsa::launch_index_qk(kx, k_rows, k_pos, k_dst_row, k_out_fp8, k_out_scale, qx, q_rows, q_heads, q_pos,
+                              q_out_fp8, q_out_scale, x_dtype, rope_cs, max_pos, flags, (cudaStream_t)stream,
+                              status);
 }
 
 int dsa_index_scores(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8,

@@ -31,27 +31,31 @@ __device__ __forceinline__ float4 load4<uint16_t>(const uint16_t* __restrict__ x
                      __uint_as_float(u.y & 0xffff0000u));
 }
 
+// One transform problem: `blocks` 128-element blocks of x ([rows][heads][128]), their positions
+// and outputs (dense, or scattered to the rows dst_row names).
+struct KeysJob {
+  const void* x;
+  int64_t blocks;
+  int heads;
+  const int32_t* pos;
+  uint8_t* out_fp8;
+  float* out_scale;
+  const int64_t* dst_row;
+};
+
+// One warp transforms block `blk` of job `j`.
 template <typename In>
-__global__ void __launch_bounds__(256) index_keys_kernel(const In* __restrict__ x, int64_t blocks,
-                                                          int heads, const int32_t* __restrict__ pos,
-                                                          const float* __restrict__ rope_cs,
-                                                          int max_pos, uint32_t flags,
-                                                          uint8_t* __restrict__ out_fp8,
-                                                          float* __restrict__ out_scale,
-                                                          const int64_t* __restrict__ dst_row,
-                                                          int* status) {
-  const int lane = threadIdx.x & 31;
-  const int64_t blk = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  grid_dep_wait();
-  grid_dep_launch();
-  if (blk >= blocks) return;
-  const int64_t row = blk / heads;
-  const int head = (int)(blk - row * heads);
+__device__ __forceinline__ void transform_block(const KeysJob& j, int64_t blk, int lane,
+                                                const float* __restrict__ rope_cs, int max_pos, uint32_t flags,
+                                                int* status) {
+  const In* __restrict__ x = static_cast<const In*>(j.x);
+  const int64_t row = blk / j.heads;
+  const int head = (int)(blk - row * j.heads);
   // the three loads that do not depend on the position go out together, before the RoPE table
   // load that does (a warp's only work is this one block, so its latency is the chain of loads)
   const float4 v4 = load4<In>(x, blk, lane);
-  const int64_t dst = dst_row ? __ldg(dst_row + row) : -1;
-  const int p = pos[row];
+  const int64_t dst = j.dst_row ? __ldg(j.dst_row + row) : -1;
+  const int p = j.pos[row];
   if (p < 0 || p >= max_pos) {
     if (lane == 0) set_status(status, DSA_ERR_DEVICE_BOUNDS);
     return;
@@ -113,25 +117,59 @@ __global__ void __launch_bounds__(256) index_keys_kernel(const In* __restrict__ 
                                __NV_SATFINITE, __NV_E4M3);
   const uint32_t packed = (uint32_t)lo | ((uint32_t)hi << 16);
 
-  const int64_t out_blk = dst_row ? dst * heads + head : blk;
-  reinterpret_cast<uint32_t*>(out_fp8 + out_blk * 128)[lane] = packed;
-  if (lane == 0) out_scale[out_blk] = scale;
+  const int64_t out_blk = j.dst_row ? dst * j.heads + head : blk;
+  reinterpret_cast<uint32_t*>(j.out_fp8 + out_blk * 128)[lane] = packed;
+  if (lane == 0) j.out_scale[out_blk] = scale;
+}
+
+constexpr int kKeysWarps = 8;   // blocks (warps) per CTA
+
+// Two jobs in one launch: CTAs [0, a_ctas) transform job a, the rest job b (one block per warp).
+template <typename In>
+__global__ void __launch_bounds__(kKeysWarps * 32) index_keys_kernel(const KeysJob a, const KeysJob b, int64_t a_ctas,
+                                                                     const float* __restrict__ rope_cs, int max_pos,
+                                                                     uint32_t flags, int* status) {
+  const int lane = threadIdx.x & 31;
+  const bool in_a = (int64_t)blockIdx.x < a_ctas;
+  const int64_t cta = in_a ? (int64_t)blockIdx.x : (int64_t)blockIdx.x - a_ctas;
+  const int64_t blk = cta * kKeysWarps + (threadIdx.x >> 5);
+  grid_dep_wait();
+  grid_dep_launch();
+  const KeysJob j = in_a ? a : b;
+  if (blk >= j.blocks) return;
+  transform_block<In>(j, blk, lane, rope_cs, max_pos, flags, status);
+}
+
+int launch_index_qk(const void* kx, int64_t k_rows, const int32_t* k_pos, const int64_t* k_dst_row,
+                    uint8_t* k_out_fp8, float* k_out_scale, const void* qx, int64_t q_rows, int q_heads,
+                    const int32_t* q_pos, uint8_t* q_out_fp8, float* q_out_scale, int x_dtype,
+                    const float* rope_cs, int max_pos, uint32_t flags, cudaStream_t stream, int* status) {
+  const KeysJob a{kx, k_rows, 1, k_pos, k_out_fp8, k_out_scale, k_dst_row};
+  const KeysJob b{qx, q_rows * q_heads, q_heads, q_pos, q_out_fp8, q_out_scale, nullptr};
+  const int64_t a_ctas = (a.blocks + kKeysWarps - 1) / kKeysWarps;
+  const int64_t grid = a_ctas + (b.blocks + kKeysWarps - 1) / kKeysWarps;
+  if (grid == 0) return DSA_OK;
+  if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;
+  if (x_dtype == DSA_BF16)
+    return dsa_host::launch(index_keys_kernel<uint16_t>, dim3((unsigned)grid), dim3(kKeysWarps * 32), 0, stream, a, b,
+                            a_ctas, rope_cs, max_pos, flags, status);
+  return dsa_host::launch(index_keys_kernel<float>, dim3((unsigned)grid), dim3(kKeysWarps * 32), 0, stream, a, b,
+                          a_ctas, rope_cs, max_pos, flags, status);
 }
 
 int launch_index_keys(const void* x, int x_dtype, int64_t rows, int heads, const int32_t* pos,
                       const float* rope_cs, int max_pos, uint32_t flags, uint8_t* out_fp8,
                       float* out_scale, const int64_t* dst_row, cudaStream_t stream, int* status) {
-  const int64_t blocks = rows * heads;
-  if (blocks == 0) return DSA_OK;
-  const int warps = 8;
-  const int64_t grid = (blocks + warps - 1) / warps;
+  const KeysJob a{x, rows * heads, heads, pos, out_fp8, out_scale, dst_row};
+  const KeysJob none{x, 0, 1, pos, out_fp8, out_scale, nullptr};
+  const int64_t grid = (a.blocks + kKeysWarps - 1) / kKeysWarps;
+  if (grid == 0) return DSA_OK;
+  if (grid > 0x7fffffff) return DSA_ERR_INVALID_ARG;
   if (x_dtype == DSA_BF16)
-    return dsa_host::launch(index_keys_kernel<uint16_t>, dim3((unsigned)grid), dim3(warps * 32), 0, stream,
-                            static_cast<const uint16_t*>(x), blocks, heads, pos, rope_cs, max_pos, flags, out_fp8,
-                            out_scale, dst_row, status);
-  return dsa_host::launch(index_keys_kernel<float>, dim3((unsigned)grid), dim3(warps * 32), 0, stream,
-                          static_cast<const float*>(x), blocks, heads, pos, rope_cs, max_pos, flags, out_fp8,
-                          out_scale, dst_row, status);
+    return dsa_host::launch(index_keys_kernel<uint16_t>, dim3((unsigned)grid), dim3(kKeysWarps * 32), 0, stream, a,
+                            none, grid, rope_cs, max_pos, flags, status);
+  return dsa_host::launch(index_keys_kernel<float>, dim3((unsigned)grid), dim3(kKeysWarps * 32), 0, stream, a, none,
+                          grid, rope_cs, max_pos, flags, status);
 }
 
 }  // namespace dsa

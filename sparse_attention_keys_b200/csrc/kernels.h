@@ -10,6 +10,12 @@ namespace dsa {
 int launch_index_keys(const void* x, int x_dtype, int64_t rows, int heads, const int32_t* pos,
                       const float* rope_cs, int max_pos, uint32_t flags, uint8_t* out_fp8,
                       float* out_scale, const int64_t* dst_row, cudaStream_t stream, int* status);
+// dsa_index_keys on the new keys (heads 1, optionally scattered by k_dst_row) and on the queries
+// (q_heads per row, dense) in one launch
+int launch_index_qk(const void* kx, int64_t k_rows, const int32_t* k_pos, const int64_t* k_dst_row,
+                    uint8_t* k_out_fp8, float* k_out_scale, const void* qx, int64_t q_rows, int q_heads,
+                    const int32_t* q_pos, uint8_t* q_out_fp8, float* q_out_scale, int x_dtype,
+                    const float* rope_cs, int max_pos, uint32_t flags, cudaStream_t stream, int* status);
 
 int launch_index_topk(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8,
                       const float* k_scale, const int32_t* q_pos, const int32_t* kv_len, int B, int T,

@@ -63,6 +63,17 @@ def test_invalid_arguments_rejected_before_launch(L):
     assert L.dsa_index_keys(bad, 0, 4, 1, p, p, 10, 1, p, p, n, n) == 1         # misaligned x
     assert L.dsa_index_keys(n, 1, 4, 1, p, p, 10, 1, p, p, n, n) == 1           # null x
     assert L.dsa_index_keys(p, 0, 0, 1, p, p, 10, 1, p, p, n, n) == 0           # empty: nothing to do
+    # dsa_index_qk: (kx, k_rows, k_pos, k_dst_row, k_fp8, k_scale, qx, q_rows, q_heads, q_pos, q_fp8, q_scale,
+    #                x_dtype, rope_cs, max_pos, flags, stream), the checks of dsa_index_keys on each side
+    qk = [p, 4, p, n, p, p, p, 2, 64, p, p, p, 0, p, 10, 1, n]
+    a = list(qk); a[8] = 0; assert L.dsa_index_qk(*a) == 1                    # query heads < 1
+    a = list(qk); a[15] = 8; assert L.dsa_index_qk(*a) == 1                   # unknown flag
+    a = list(qk); a[12] = 2; assert L.dsa_index_qk(*a) == 1                   # unknown input type
+    a = list(qk); a[3] = bad; assert L.dsa_index_qk(*a) == 1                  # misaligned k_dst_row
+    a = list(qk); a[6] = n; assert L.dsa_index_qk(*a) == 1                    # null qx with query rows
+    a = list(qk); a[1] = -1; assert L.dsa_index_qk(*a) == 1                   # negative key rows
+    a = list(qk); a[14] = 0; assert L.dsa_index_qk(*a) == 1                   # max_pos < 1
+    a = list(qk); a[1] = 0; a[7] = 0; assert L.dsa_index_qk(*a) == 0          # both sides empty
     f = ctypes.c_float
     args = [p, p, p, p, p, p, p, 1, 1, 128, f(0.088), p, 128, 0, n]
     a = list(args); a[12] = 126; assert L.dsa_index_scores(*a) == 1          # ld not a multiple of 4

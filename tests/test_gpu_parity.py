@@ -114,6 +114,76 @@ def test_index_keys_position_out_of_range_sets_status(table_dev):
     assert _status() == 5          # DSA_ERR_DEVICE_BOUNDS
 
 
+def _qk_inputs(k_rows, q_rows, dtype, seed):
+    rng = np.random.default_rng(seed)
+    kx = rng.standard_normal((k_rows, 128)).astype(np.float32) * 2.0
+    qx = rng.standard_normal((q_rows, 64, 128)).astype(np.float32)
+    k_pos = rng.integers(0, 16384, k_rows).astype(np.int32)
+    q_pos = rng.integers(0, 16384, q_rows).astype(np.int32)
+    if dtype == "bf16":
+        to = lambda a: torch.from_numpy(DI.bf16_bits_from_f32(a)).cuda().view(torch.bfloat16)
+    else:
+        to = P.to_dev
+    return to(kx), to(qx), P.to_dev(k_pos), P.to_dev(q_pos)
+
+
+@pytest.mark.parametrize("k_rows,q_rows,dtype", [
+    (8, 8, "f32"),          # a decode step of 8 sequences: one key CTA, 64 query CTAs
+    (13, 7, "bf16"),        # ragged: the key CTAs' last one partly empty, the query range 448 blocks
+    (0, 5, "f32"),          # no new keys
+    (9, 0, "f32"),          # no queries
+    (2048, 64, "f32"),      # many key CTAs ahead of the queries
+])
+@pytest.mark.parametrize("scatter", [True, False])
+def test_index_qk_equals_two_index_keys_calls(table_dev, k_rows, q_rows, dtype, scatter):
+    """dsa_index_qk against dsa_index_keys on the keys then on the queries: bit for bit, including
+    the bytes of the cache rows it must not touch."""
+    kx, qx, k_pos, q_pos = _qk_inputs(k_rows, q_rows, dtype, seed=100 + k_rows + q_rows)
+    B, S = 3, 1000
+    dst = (torch.randperm(B * S, device="cuda")[:k_rows].to(torch.int64).contiguous() if scatter else None)
+    shape_k = (B, S, 128) if scatter else (max(k_rows, 1), 128)
+    shape_ks = (B, S) if scatter else (max(k_rows, 1),)
+    want_c = torch.full(shape_k, 0xAB, dtype=torch.uint8, device="cuda")
+    want_s = torch.full(shape_ks, -1.0, dtype=torch.float32, device="cuda")
+    got_c, got_s = want_c.clone(), want_s.clone()
+    if k_rows:
+        dsa.dsa_index_keys(kx, k_pos, table_dev, out_fp8=want_c, out_scale=want_s, dst_row=dst)
+    want_q8, want_qs = (dsa.dsa_index_keys(qx, q_pos, table_dev) if q_rows else
+                        (torch.empty((0, 64, 128), dtype=torch.uint8, device="cuda"),
+                         torch.empty((0, 64), dtype=torch.float32, device="cuda")))
+    got_q8, got_qs = dsa.dsa_index_qk(kx, k_pos, qx, q_pos, table_dev, got_c, got_s, k_dst_row=dst)
+    torch.cuda.synchronize()
+    assert _status() == 0
+    assert torch.equal(got_c, want_c) and torch.equal(got_s, want_s)
+    assert torch.equal(got_q8, want_q8) and torch.equal(got_qs, want_qs)
+
+
+def test_index_qk_against_the_oracle(table_dev):
+    """One decode-shaped call against the oracle's codes for both sides."""
+    rng = np.random.default_rng(7)
+    kx = rng.standard_normal((6, 128)).astype(np.float32)
+    qx = rng.standard_normal((6, 64, 128)).astype(np.float32)
+    pos = rng.integers(0, 16384, 6).astype(np.int32)
+    k8 = torch.empty((6, 128), dtype=torch.uint8, device="cuda")
+    ks = torch.empty((6,), dtype=torch.float32, device="cuda")
+    q8, qs = dsa.dsa_index_qk(P.to_dev(kx), P.to_dev(pos), P.to_dev(qx), P.to_dev(pos), table_dev, k8, ks)
+    torch.cuda.synchronize()
+    assert _status() == 0
+    P.check_codes(k8.cpu().numpy(), ks.cpu().numpy(), kx, pos, TABLE)
+    P.check_codes(q8.cpu().numpy(), qs.cpu().numpy(), qx, pos[:, None], TABLE)
+
+
+def test_index_qk_key_position_out_of_range_sets_status(table_dev):
+    kx = torch.zeros((3, 128), dtype=torch.float32, device="cuda")
+    qx = torch.zeros((2, 64, 128), dtype=torch.float32, device="cuda")
+    k_pos = torch.tensor([0, 20000, 2], dtype=torch.int32, device="cuda")
+    q_pos = torch.tensor([4, 5], dtype=torch.int32, device="cuda")
+    k8 = torch.empty((3, 128), dtype=torch.uint8, device="cuda")
+    ks = torch.empty((3,), dtype=torch.float32, device="cuda")
+    dsa.dsa_index_qk(kx, k_pos, qx, q_pos, table_dev, k8, ks)
+    assert _status() == 5          # DSA_ERR_DEVICE_BOUNDS
+
+
 # ----------------------------------------------------------------------------------- scores
 def _quantised(inp, q_rows=None, k_seqs=None):
     """Oracle-quantised q/k for a workload (the same bytes are fed to the GPU). With q_rows
