@@ -503,6 +503,7 @@ def run_ours(args, rank, world, local_rank):
     t_e2e = timed_rotation(graph_step)
     check_status(dsa, "end-to-end graph steps")
     del graphs
+    link = time_link(slots, streams, args.steps)
     del slots[1:]
 
     producers = None if (args.no_producers or st.kv is None) else time_producers(st, args, dev)
@@ -550,7 +551,8 @@ def run_ours(args, rank, world, local_rank):
                 "graph": {"value": weak_scaling_value(units["pairs"], args.steps, world, t_e2e),
                           "ms_per_step": t_e2e / args.steps * 1e3},
                 "eager": {"value": weak_scaling_value(units["pairs"], args.steps, world, t_e2e_eager),
-                          "ms_per_step": t_e2e_eager / args.steps * 1e3}},
+                          "ms_per_step": t_e2e_eager / args.steps * 1e3},
+                "link": link},
         "gpu_launches": st.launches_per_step * args.steps,
         "timing": ("device: CUDA-graph replay of the step, CUDA events around each replay; kernel_ms and "
                    "roofline: a replay of the same step with CUDA events around each call, after each "
@@ -603,6 +605,38 @@ def time_producers(st, args, dev):
         out[name] = _graph_time(st, fn, args)
     check_status(dsa, "MLA producers")
     return out
+
+
+def time_link(slots, streams, steps):
+    """The host link alone, per step: the step's host -> device copies with nothing else running,
+    its device -> host copies alone, and both directions at once (two slots, two streams). The
+    last is the floor under the end-to-end step time when kernels hide behind the copies."""
+    import torch
+    a, b = streams[0], streams[1 % len(streams)]
+    sa, sb = slots[0], slots[1 % len(slots)]
+
+    def timed(jobs):
+        cur = torch.cuda.current_stream()
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(cur)
+        a.wait_event(s)
+        b.wait_event(s)
+        for _ in range(steps):
+            for stream, fn in jobs:
+                with torch.cuda.stream(stream):
+                    fn()
+        cur.wait_stream(a)
+        cur.wait_stream(b)
+        e.record(cur)
+        torch.cuda.synchronize()
+        return s.elapsed_time(e) / 1e3 / steps
+
+    timed([(a, sa.h2d), (b, sb.d2h)])                   # warm-up
+    t_h, t_d = timed([(a, sa.h2d)]), timed([(b, sb.d2h)])
+    t_both = timed([(a, sa.h2d), (b, sb.d2h)])
+    return {"h2d_ms": t_h * 1e3, "d2h_ms": t_d * 1e3, "both_ms": t_both * 1e3,
+            "h2d_gbs": sa.bytes_h2d() / t_h / 1e9, "d2h_gbs": sb.bytes_d2h() / t_d / 1e9}
 
 
 def _graph_time(st, fn, args):
