@@ -419,14 +419,14 @@ __device__ __forceinline__ void st_shared_if(int32_t* dst, int32_t v, bool pred)
                : "memory");
 }
 
-// Exclusive prefix, in thread order, of one value per thread of the CTA (NT threads); *total gets
-// the sum. One barrier; `tot` (NT / 32 words) is written before it and read after it, so a call
-// must not reuse the `tot` of the previous call before another barrier.
 // Bulk prefetch of [p, p + bytes) into the L2 (p 16-byte aligned, bytes a multiple of 16).
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
+// Exclusive prefix, in thread order, of one value per thread of the CTA (NT threads); *total gets
+// the sum. One barrier; `tot` (NT / 32 words) is written before it and read after it, so a call
+// must not reuse the `tot` of the previous call before another barrier.
 template <int NT>
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tot, uint32_t* total) {
   constexpr int kRegWarps = NT / 32;
